@@ -1,0 +1,234 @@
+/*
+ * ic.h -- C ABI of libic_b200.so: the hot path of DeepSeek Sparse Attention
+ * with IndexCache (lightning indexer -> per-row top-k -> sparse attention, and
+ * the F/S layer stack that shares the index set), hand-written for sm_100a.
+ *
+ * Sources.  "IndexCache: Wie DeepSeek O(NL^2)-Kosten in Sparse Attention um
+ * 75% reduziert" (itoverdose.com): the intro (k = 2048 positions per query;
+ * attention cost O(Lk)), the second paragraph (the indexer scores all previous
+ * tokens), the F/S list and "the first layer is always F", the routing loop of
+ * "Einfache Implementierung, enorme Effizienzgewinne" (I <- Indexer(X);
+ * T <- top-k(I); T_cache <- T / T <- T_cache; X <- SparseAttn(X, T)), the
+ * T_cache paragraph right after it (one buffer, overwritten by every F layer,
+ * no extra memory), "Wie der Indexer funktioniert" (score, ReLU gate, top-k)
+ * and the MLA paragraph (one latent vector shared by all heads).  The
+ * parapluman.nl article, "Aandacht cachen met IndexCache": an S layer reuses
+ * the indices of the nearest preceding F layer.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named in the argument lists are DEVICE pointers unless marked
+ *    "host".  The caller owns every buffer; the library never allocates device
+ *    memory and keeps no state besides a thread-local error message and one
+ *    device error word.
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and the call returns without synchronising.
+ *  - Tensors are dense, row-major, with the layouts given per function.
+ *  - Errors are returned as negative ic_status codes; arguments are checked
+ *    before anything is launched, so a failed call has launched nothing.
+ *    ic_last_error() describes the last failure of the calling thread.
+ *  - Kernels never trap: a device-side wait that runs out of time (2 s)
+ *    records a code in the device error word, abandons its work and returns;
+ *    ic_device_status() reports it (IC_ERR_TIMEOUT).
+ */
+#ifndef IC_H_
+#define IC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int ic_status;
+#define IC_OK 0
+#define IC_ERR_INVALID_ARG (-1) /* bad pointer, size, layout or pattern        */
+#define IC_ERR_UNSUPPORTED (-2) /* valid request this build does not implement */
+#define IC_ERR_WORKSPACE (-3)   /* workspace missing or too small              */
+#define IC_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed           */
+#define IC_ERR_TIMEOUT (-5)     /* a device-side bounded wait gave up          */
+
+typedef enum { IC_F32 = 0, IC_BF16 = 1, IC_E4M3 = 2 } ic_dtype;
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* ic_last_error(void);
+
+/* Library ABI version (major * 100 + minor). */
+int ic_version(void);
+
+/* Synchronise `stream`, then read and clear the device error word.
+ * Returns IC_OK, IC_ERR_TIMEOUT (a bounded device wait gave up since the last
+ * check) or IC_ERR_CUDA. */
+ic_status ic_device_status(void* stream);
+
+/*
+ * Launch tracing, for timing each kernel on the device.  ic_trace_begin records
+ * a start event on `stream`; from then on, every kernel this library launches
+ * from the calling host thread is followed by an event record on its stream
+ * (all calls must use that same stream for the intervals to be meaningful).
+ * ic_trace_end waits for the last event and fills, for launch i (i < capacity):
+ *   ms[i]    device time from the previous event to this launch's event (ms),
+ *   kinds[i] IC_K_* of the launch,
+ *   work[i]  its algorithmic work: flops for the indexer, bytes for the
+ *            memory-bound kernels (each input byte read once, output written once).
+ * Any of ms/kinds/work may be NULL.  Returns the number of launches made while
+ * recording (launches beyond `capacity` are counted but not timed), or a
+ * negative ic_status.  The library creates its events once and keeps them.
+ */
+#define IC_K_INDEXER_BF16 1
+#define IC_K_INDEXER_E4M3 2
+#define IC_K_INDEXER_F32 3
+#define IC_K_FILL_MASKED 4
+#define IC_K_TOPK 5
+#define IC_K_ATTN_MLA 6
+#define IC_K_ATTN_COMBINE 7
+#define IC_K_ATTN_F32 8
+#define IC_K_QUANT 9
+ic_status ic_trace_begin(void* stream, int capacity);
+long ic_trace_end(float* ms, int* kinds, double* work, int capacity);
+
+/*
+ * Per-row e4m3 quantisation (the fp8 variant of the indexer inputs, "per-token
+ * fp32 scales"; OCP 8-bit floating point, E4M3).  For each row of n values:
+ * scale = amax / 448 (1 for an all-zero row), code = E4M3_rne_satfinite(x / scale),
+ * computed in fp32.
+ *   x      [rows, n] of x_dtype (IC_BF16 or IC_F32)
+ *   codes  [rows, n] uint8 (e4m3 bit patterns)
+ *   scales [rows] float
+ * n must be a multiple of 8 and <= 1024.
+ */
+ic_status ic_quant_e4m3_rows(const void* x, ic_dtype x_dtype, long rows, int n, uint8_t* codes,
+                             float* scales, void* stream);
+
+/*
+ * Lightning-indexer scores ("Wie der Indexer funktioniert": a score per
+ * previous position, a ReLU gate, then top-k; the weighted head sum is this
+ * library's reading of that passage):
+ *   I[b, r, s] = sum_h w[b, r, h] * max(0, q[b, r, h, :] . k[b, s, :])
+ * for every key s <= pos0 + r (query row r sits at position pos0 + r), and
+ * I[b, r, s] = -inf for s > pos0 + r (not a candidate).
+ *   q       [batch, rows, H, D]  dt (IC_BF16 / IC_E4M3 codes / IC_F32)
+ *   q_scale [batch, rows, H] f32 (IC_E4M3 only; NULL otherwise): q = code * q_scale
+ *   k       [batch, Lk, D]       dt
+ *   k_scale [batch, Lk] f32      (IC_E4M3 only; NULL otherwise): k = code * k_scale
+ *   w       [batch, rows, H] f32 head weights
+ *   scores  [batch, rows, ld] f32 output, ld >= Lk; columns [0, Lk) are written
+ * IC_BF16 and IC_E4M3 run on the tensor cores and need H = 64, D = 128 (fp32
+ * accumulation); IC_F32 runs on the CUDA cores for any H <= 64, D <= 256.
+ * pos0 >= 0.  Scores are fp32; the fp8 scales are folded in after the dot products.
+ */
+ic_status ic_indexer_scores(const void* q, const float* q_scale, const void* k,
+                            const float* k_scale, const float* w, ic_dtype dt, int batch, int H,
+                            int D, int rows, int Lk, long pos0, float* scores, long ld,
+                            void* stream);
+
+/*
+ * Exact per-row top-k (routing loop: T <- top-k(I); k = 2048 in the pages).
+ * Row r's candidates are columns s < valid(r), where valid(r) = n when
+ * pos0 < 0, else min(n, pos0 + r + 1) (causal rows).  Output idx[r, 0..k):
+ * the min(k, valid(r)) candidates with the largest scores -- ties go to the
+ * lower index and -0 == +0 -- in ascending index order, padded with -1.
+ *   scores [rows, ld] f32 (finite on the candidate columns), ld >= n
+ *   idx    [rows, k] int32
+ * 1 <= k <= 2048.  Bit-exact: the selection is a pure function of the fp32 values.
+ */
+ic_status ic_topk(const float* scores, long rows, int n, long ld, long pos0, int k, int* idx,
+                  void* stream);
+
+/*
+ * Sparse attention of each query over its index set (routing loop:
+ * X <- SparseAttn(X, T); MLA paragraph).  For query (b, r), head h, with
+ * J = { idx[b, r, j] : idx >= 0 } (-1 entries are skipped):
+ *   z_j = scale * q[b, r, h, :dk] . kv[b, j, :dk]
+ *   out[b, r, h, :] = sum_j softmax(z)_j * V[b, j, :dv]
+ *   lse[b, r, h]    = log sum_j exp(z_j)      (natural log; -inf if J is empty)
+ * Two forms:
+ *   v == NULL  absorbed MLA: V = kv[..., :dv] (the first dv latent dims);
+ *              dt = IC_BF16, dk = 576, dv = 512, heads = 16; out bf16.
+ *   v != NULL  MQA with separate values v [batch, Lkv, dv]; dt = IC_F32,
+ *              dk, dv <= 256, heads <= 64; out f32.
+ *   q   [batch, rows, heads, dk]; kv [batch, Lkv, ld_kv] (ld_kv >= dk, elements);
+ *   idx [batch, rows, k] int32 in [-1, Lkv); out [batch, rows, heads, dv];
+ *   lse [batch, rows, heads] f32 or NULL.
+ * workspace (device, may be NULL): with IC_BF16 and rows * batch small, the
+ * index list is split over several CTAs whose partial results go through the
+ * workspace (see ic_attn_workspace_size); with too little workspace the
+ * split is reduced, never an error.
+ */
+ic_status ic_sparse_attn(const void* q, const void* kv, long ld_kv, const void* v, const int* idx,
+                         ic_dtype dt, int batch, int rows, int heads, int dk, int dv, int Lkv,
+                         int k, float scale, void* out, float* lse, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/* Workspace bytes that let ic_sparse_attn use its preferred split for this shape. */
+size_t ic_attn_workspace_size(int batch, int rows, int heads, int dv, int k);
+
+/*
+ * Per-layer inputs of the layer stack.  Every pointer is device memory.
+ * F layers need the indexer fields; S layers ignore them (they may be NULL).
+ */
+typedef struct {
+  const void* q_idx;    /* [batch, R, H, D] indexer queries (idx_dtype)          */
+  const float* q_scale; /* [batch, R, H] (IC_E4M3 only)                          */
+  const void* k_idx;    /* [batch, L, D] indexer keys (idx_dtype)                */
+  const float* k_scale; /* [batch, L] (IC_E4M3 only)                             */
+  const float* w;       /* [batch, R, H] indexer head weights                    */
+  const void* q;        /* [batch, R, heads, dk] attention queries (attn_dtype)  */
+  const void* kv;       /* [batch, L, ld_kv] latent (MLA) or keys (MQA)          */
+  const void* v;        /* [batch, L, dv] values (MQA only; NULL for MLA)        */
+  void* out;            /* [batch, R, heads, dv] attention output                */
+  float* lse;           /* [batch, R, heads] or NULL                             */
+} ic_layer_io;
+
+/*
+ * Shape of a layer stack.
+ *   prefill: batch = 1, R = L query rows at positions 0..L-1 (causal);
+ *   decode:  batch sequences, R = 1 new token each, at position L-1 of a
+ *            context of L tokens (keys 0..L-1).
+ */
+typedef struct {
+  int L;               /* tokens (prefill) / context length (decode)             */
+  int batch;           /* 1 for prefill; sequences for decode                    */
+  int decode;          /* 0 = prefill, 1 = decode                                */
+  int k;               /* top-k (<= 2048)                                        */
+  ic_dtype idx_dtype;  /* IC_BF16, IC_E4M3 (H=64, D=128) or IC_F32              */
+  int H, D;            /* indexer heads and head dim                             */
+  ic_dtype attn_dtype; /* IC_BF16 (absorbed MLA) or IC_F32 (MQA)                 */
+  int heads, dk, dv;   /* attention heads, key dim, value dim                    */
+  long ld_kv;          /* row stride of kv in elements                           */
+  float scale;         /* softmax scale                                          */
+} ic_stack_desc;
+
+/*
+ * The IndexCache layer stack (routing loop of "Einfache Implementierung",
+ * without the FFN): for layer l = 1..N,
+ *   c_l == 'F': T_cache <- top-k(Indexer_l)   (scores stream through `workspace`
+ *               in row blocks; the L x L matrix is never formed)
+ *   c_l == 'S': T_cache is reused unchanged   (zero work: the nearest preceding
+ *               F layer's index set)
+ *   out_l <- SparseAttn_l(T_cache)
+ * pattern: host string of 'F'/'S', optionally separated by ',' or ' '; its
+ * first layer must be 'F'; its layer count must equal nlayers.
+ * layers: host array of nlayers ic_layer_io.  t_cache: device int32
+ * [batch * R, k], caller-owned, holds the last F layer's index set on return.
+ * workspace: device, at least ic_stack_workspace_size(desc) bytes is
+ * recommended; the minimum is one score row block (a smaller workspace means
+ * smaller row blocks, IC_ERR_WORKSPACE only below one row).
+ */
+ic_status ic_layer_stack(const char* pattern, const ic_stack_desc* desc, const ic_layer_io* layers,
+                         int nlayers, int* t_cache, void* workspace, size_t ws_bytes,
+                         void* stream);
+
+/* Decode form of the stack (desc->decode must be 1): same routing per layer,
+ * one query per sequence; t_cache is [batch, k]. */
+ic_status ic_decode_step(const char* pattern, const ic_stack_desc* desc, const ic_layer_io* layers,
+                         int nlayers, int* t_cache, void* workspace, size_t ws_bytes,
+                         void* stream);
+
+/* Recommended workspace bytes for ic_layer_stack / ic_decode_step. */
+size_t ic_stack_workspace_size(const ic_stack_desc* desc);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* IC_H_ */

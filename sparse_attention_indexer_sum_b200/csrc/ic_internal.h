@@ -1,0 +1,60 @@
+// ic_internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/ic.h"
+
+namespace ic {
+
+// Records a formatted message for ic_last_error() and returns `code`.
+ic_status fail(ic_status code, const char* fmt, ...);
+// Checks a CUDA runtime result; on failure records it and returns IC_ERR_CUDA.
+ic_status cuda_check(cudaError_t e, const char* what);
+int num_sms();
+
+// Launch kinds reported by the tracing hook (ic_trace_begin / ic_trace_end).
+enum LaunchKind : int {
+  kKindIndexerBf16 = 1,
+  kKindIndexerE4m3 = 2,
+  kKindIndexerF32 = 3,
+  kKindFillMasked = 4,
+  kKindTopk = 5,
+  kKindAttnMla = 6,
+  kKindAttnCombine = 7,
+  kKindAttnF32 = 8,
+  kKindQuant = 9,
+};
+// Called after every kernel launch: when tracing is on for this host thread,
+// records an event on `stream` with the launch's kind and algorithmic work
+// (flops for the indexer, bytes for the memory-bound kernels).
+void trace_launch(int kind, cudaStream_t stream, double work);
+// Number of (query, key) pairs with key < Lk and key <= pos0 + r over rows r < R.
+long long causal_pairs(long R, long Lk, long pos0);
+
+// Indexer on tensor cores (H = 64, D = 128).  fp8 = e4m3 inputs with scales.
+ic_status launch_indexer_tc(bool fp8, const void* q, const float* q_scale, const void* k,
+                            const float* k_scale, const float* w, int batch, int rows, int Lk,
+                            long pos0, float* scores, long ld, bool fill_tail,
+                            cudaStream_t stream);
+// Indexer on CUDA cores for fp32 inputs (small H, D).
+ic_status launch_indexer_f32(const float* q, const float* k, const float* w, int batch, int H,
+                             int D, int rows, int Lk, long pos0, float* scores, long ld,
+                             cudaStream_t stream);
+ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0, int k, int* idx,
+                      cudaStream_t stream);
+// valid_entries: number of index entries >= 0 over all rows if the caller knows
+// it (the causal stack does), else -1 (rows * k is assumed for tracing only).
+ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* idx, int batch,
+                          int rows, int Lkv, int k, float scale, void* out, float* lse,
+                          void* ws, size_t ws_bytes, long long valid_entries, cudaStream_t stream);
+size_t attn_mla_ws_bytes(int batch, int rows, int k);
+ic_status launch_attn_f32(const float* q, const float* kv, long ld_kv, const float* v,
+                          const int* idx, int batch, int rows, int heads, int dk, int dv,
+                          int Lkv, int k, float scale, float* out, float* lse,
+                          cudaStream_t stream);
+ic_status launch_quant_e4m3(const void* x, bool bf16, long rows, int n, uint8_t* codes,
+                            float* scales, cudaStream_t stream);
+
+}  // namespace ic

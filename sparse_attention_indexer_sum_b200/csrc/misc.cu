@@ -1,0 +1,101 @@
+// misc.cu -- the small kernels of the path:
+//  * per-row e4m3 quantisation of indexer inputs (OCP 8-bit floating point,
+//    E4M3; "per-token fp32 scales" of the fp8 indexer variant);
+//  * the indexer on CUDA cores for fp32 inputs (small head counts and dims:
+//    the fp32 workload has 4 heads of dim 32, far too small for tensor tiles).
+#include "ic_device.cuh"
+#include "ic_internal.h"
+
+namespace ic {
+
+// One warp per row of n (<= 1024, multiple of 8) values:
+//   scale = amax / 448 (1 when amax == 0);  code = e4m3_rn_satfinite(x / scale)
+// Both the scale and the quotient are IEEE fp32 divisions.
+template <typename T>
+__global__ void quant_e4m3_kernel(const T* __restrict__ x, long rows, int n,
+                                  uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  const long row = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const T* xr = x + row * n;
+  float vals[32];
+  float amax = 0.f;
+  int cnt = 0;
+  for (int i = lane; i < n; i += 32, ++cnt) {
+    const float v = static_cast<float>(xr[i]);
+    vals[cnt] = v;
+    amax = fmaxf(amax, fabsf(v));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  if (lane == 0) scales[row] = scale;
+  cnt = 0;
+  for (int i = lane; i < n; i += 32, ++cnt)
+    codes[row * n + i] = static_cast<uint8_t>(
+        __nv_cvt_float_to_fp8(__fdiv_rn(vals[cnt], scale), __NV_SATFINITE, __NV_E4M3));
+}
+
+ic_status launch_quant_e4m3(const void* x, bool bf16, long rows, int n, uint8_t* codes,
+                            float* scales, cudaStream_t stream) {
+  if (rows == 0) return IC_OK;
+  const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  if (bf16)
+    quant_e4m3_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), rows, n, codes, scales);
+  else
+    quant_e4m3_kernel<float><<<blocks, 256, 0, stream>>>(static_cast<const float*>(x), rows, n,
+                                                         codes, scales);
+  ic_status st = cuda_check(cudaGetLastError(), "quant_e4m3_kernel launch");
+  if (!st)
+    trace_launch(kKindQuant, stream,
+                 static_cast<double>(rows) * (n * ((bf16 ? 2.0 : 4.0) + 1.0) + 4.0));
+  return st;
+}
+
+// I[b,r,s] = sum_h w[b,r,h] * max(0, q[b,r,h,:] . k[b,s,:]) on CUDA cores.
+// Grid (batch * rows, ceil(Lk / 128)); one key per thread, the query row in smem.
+__global__ void indexer_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                                   const float* __restrict__ w, int R, int H, int D, int Lk,
+                                   long pos0, float* __restrict__ scores, long ld) {
+  extern __shared__ float qs[];  // [H * D] then w [H]
+  const long row = blockIdx.x;   // b * R + r
+  const long b = row / R, r = row % R;
+  float* ws = qs + H * D;
+  for (int i = threadIdx.x; i < H * D; i += blockDim.x) qs[i] = q[row * H * D + i];
+  for (int i = threadIdx.x; i < H; i += blockDim.x) ws[i] = w[row * H + i];
+  __syncthreads();
+  const long s = static_cast<long>(blockIdx.y) * blockDim.x + threadIdx.x;
+  if (s >= Lk) return;
+  float res = -INFINITY;
+  if (s <= pos0 + r) {
+    const float* ks = k + (b * Lk + s) * D;
+    res = 0.f;
+    for (int h = 0; h < H; ++h) {
+      float dot = 0.f;
+      for (int d = 0; d < D; ++d) dot = fmaf(qs[h * D + d], ks[d], dot);
+      res = fmaf(ws[h], fmaxf(dot, 0.f), res);
+    }
+  }
+  scores[row * ld + s] = res;
+}
+
+ic_status launch_indexer_f32(const float* q, const float* k, const float* w, int batch, int H,
+                             int D, int rows, int Lk, long pos0, float* scores, long ld,
+                             cudaStream_t stream) {
+  if (static_cast<long>(batch) * rows == 0 || Lk == 0) return IC_OK;
+  const int smem = (H * D + H) * static_cast<int>(sizeof(float));
+  ic_status st = cuda_check(
+      cudaFuncSetAttribute(indexer_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+      "cudaFuncSetAttribute(indexer_f32)");
+  if (st) return st;
+  dim3 grid(static_cast<unsigned>(static_cast<long>(batch) * rows), static_cast<unsigned>((Lk + 127) / 128));
+  indexer_f32_kernel<<<grid, 128, smem, stream>>>(q, k, w, rows, H, D, Lk, pos0, scores, ld);
+  st = cuda_check(cudaGetLastError(), "indexer_f32_kernel launch");
+  if (!st)
+    trace_launch(kKindIndexerF32, stream,
+                 2.0 * H * D * static_cast<double>(causal_pairs(rows, Lk, pos0)) * batch);
+  return st;
+}
+
+}  // namespace ic

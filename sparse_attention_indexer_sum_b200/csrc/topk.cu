@@ -1,0 +1,325 @@
+// topk.cu -- exact per-row top-k over fp32 scores (routing loop T <- top-k(I) of
+// "IndexCache: Wie DeepSeek O(NL^2)-Kosten in Sparse Attention um 75% reduziert";
+// k = 2048 in its intro).  Ties go to the lower index, -0 == +0, output in
+// ascending index order padded with -1.
+//
+// One CTA (512 threads) per row.  Scores are mapped to order-preserving
+// 32-bit keys and the k-th largest key is found by radix selection:
+//   1. histogram of the top 12 key bits over the row (shared-memory atomics,
+//      128-bit loads); the bin holding the k-th largest is located with one
+//      block scan.  If that bin holds more than CAP keys (heavily tied data),
+//      further 12/8-bit histogram passes over the row narrow the prefix.
+//   2. one ordered pass over the row (ballot-free block scans over 4-element
+//      chunks) compacts, in index order, the keys strictly above the prefix
+//      (selected for sure) and the keys equal to it (candidates) into shared
+//      memory.
+//   3. the candidates are resolved in shared memory by more radix digits, the
+//      last tie broken by index order, and the two ascending index lists are
+//      merged into the output row.
+// In the common case each score is read twice from global memory (L2).
+#include "ic_device.cuh"
+#include "ic_internal.h"
+
+namespace ic {
+
+constexpr int TK_THREADS = 512;
+constexpr int TK_NW = TK_THREADS / 32;
+constexpr int TK_NBINS = 4096;  // 12-bit digits
+constexpr int TK_CAP = 4096;    // candidates kept in shared memory
+constexpr int TK_MAXK = 2048;
+
+struct TopkSmem {
+  int hist[TK_NBINS];
+  int gt_idx[TK_MAXK];
+  uint32_t cand_key[TK_CAP];
+  int cand_idx[TK_CAP];
+  int sel_idx[TK_MAXK];
+  int scan_tmp[TK_NW];
+  int bcast[4];
+};
+
+// Order-preserving key: a > b as floats  <=>  key(a) > key(b) as unsigned; -0 -> +0.
+__device__ __forceinline__ uint32_t score_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive block-wide prefix sum of v; *total receives the sum over the block.
+__device__ __forceinline__ int block_excl_scan(int v, int* tmp, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) tmp[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int t = (lane < TK_NW) ? tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < TK_NW) tmp[lane] = t;
+  }
+  __syncthreads();
+  const int res = (w > 0 ? tmp[w - 1] : 0) + incl - v;
+  *total = tmp[TK_NW - 1];
+  __syncthreads();
+  return res;
+}
+
+// Finds the bin B (of nbins) with count(bins > B) < need <= count(bins >= B).
+// Writes B to sm.bcast[0] and count(bins > B) to sm.bcast[1].
+__device__ __forceinline__ void find_bin(TopkSmem& sm, int nbins, int need) {
+  const int per = nbins / TK_THREADS;  // 8 (4096 bins) or 0 (256 bins)
+  int local = 0;
+  int b_lo = 0, b_hi = 0;
+  if (per > 0) {
+    b_lo = threadIdx.x * per;
+    b_hi = b_lo + per;
+  } else if (threadIdx.x < nbins) {
+    b_lo = threadIdx.x;
+    b_hi = b_lo + 1;
+  }
+  for (int b = b_lo; b < b_hi; ++b) local += sm.hist[b];
+  int total;
+  const int before = block_excl_scan(local, sm.scan_tmp, &total);
+  int above = total - before - local;  // keys in bins owned by later threads
+  for (int b = b_hi - 1; b >= b_lo; --b) {
+    const int c = sm.hist[b];
+    if (above < need && above + c >= need) {
+      sm.bcast[0] = b;
+      sm.bcast[1] = above;
+    }
+    above += c;
+  }
+  __syncthreads();
+}
+
+template <typename F>
+__device__ __forceinline__ void for_row(const float* x, int nv, bool vec, F&& f) {
+  for (int i0 = 4 * threadIdx.x; i0 < nv; i0 += 4 * TK_THREADS) {
+    if (vec && i0 + 3 < nv) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(x + i0));
+      f(i0, v.x);
+      f(i0 + 1, v.y);
+      f(i0 + 2, v.z);
+      f(i0 + 3, v.w);
+    } else {
+      for (int e = 0; e < 4 && i0 + e < nv; ++e) f(i0 + e, __ldg(x + i0 + e));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restrict__ scores, long ld,
+                                                          int n, long pos0, int k,
+                                                          int* __restrict__ idx) {
+  extern __shared__ uint8_t tk_smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
+  const long row = blockIdx.x;
+  long nvl = (pos0 < 0) ? n : pos0 + row + 1;
+  if (nvl > n) nvl = n;
+  const int nv = static_cast<int>(nvl);
+  int* out = idx + row * k;
+  if (nv <= k) {
+    for (int j = threadIdx.x; j < k; j += TK_THREADS) out[j] = (j < nv) ? j : -1;
+    return;
+  }
+  const float* x = scores + row * ld;
+  const bool vec = ((ld & 3) == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
+
+  // ---------------------------------------------------------------- 1. radix passes
+  uint32_t prefix = 0;
+  int pbits = 0;
+  int k_rem = k;
+  int cand = 0;
+  for (int level = 0; level < 3; ++level) {
+    const int bits = (level < 2) ? 12 : 8;
+    const int shift = 32 - pbits - bits;
+    const int nb = 1 << bits;
+    for (int b = threadIdx.x; b < nb; b += TK_THREADS) sm.hist[b] = 0;
+    __syncthreads();
+    const uint32_t mask = static_cast<uint32_t>(nb - 1);
+    if (level == 0) {
+      for_row(x, nv, vec, [&](int, float v) {
+        atomicAdd(&sm.hist[score_key(v) >> shift], 1);
+      });
+    } else {
+      const int hs = shift + bits;  // = 32 - pbits, in [8, 20]
+      for_row(x, nv, vec, [&](int, float v) {
+        const uint32_t key = score_key(v);
+        if ((key >> hs) == prefix) atomicAdd(&sm.hist[(key >> shift) & mask], 1);
+      });
+    }
+    __syncthreads();
+    find_bin(sm, nb, k_rem);
+    const int B = sm.bcast[0];
+    const int above = sm.bcast[1];
+    cand = sm.hist[B];
+    prefix = (prefix << bits) | static_cast<uint32_t>(B);
+    pbits += bits;
+    k_rem -= above;
+    __syncthreads();
+    if (cand <= TK_CAP) break;
+  }
+
+  // ---------------------------------------------------------------- 2. ordered compaction
+  const int hs = 32 - pbits;  // 20, 8 or 0
+  int g_run = 0, c_run = 0;
+  for (int c0 = 0; c0 < nv; c0 += 4 * TK_THREADS) {
+    const int i0 = c0 + 4 * threadIdx.x;
+    uint32_t keys[4];
+    int cls[4];  // 2 = above the prefix, 1 = candidate, 0 = neither
+    int ng = 0, nc = 0;
+    if (vec && i0 + 3 < nv) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(x + i0));
+      keys[0] = score_key(v.x);
+      keys[1] = score_key(v.y);
+      keys[2] = score_key(v.z);
+      keys[3] = score_key(v.w);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) keys[e] = (i0 + e < nv) ? score_key(__ldg(x + i0 + e)) : 0u;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      cls[e] = 0;
+      if (i0 + e < nv) {
+        const uint32_t kp = (hs >= 32) ? 0u : (keys[e] >> hs);
+        if (kp > prefix) {
+          cls[e] = 2;
+          ++ng;
+        } else if (kp == prefix) {
+          cls[e] = 1;
+          ++nc;
+        }
+      }
+    }
+    int tot;
+    const int ex = block_excl_scan(ng | (nc << 16), sm.scan_tmp, &tot);
+    int gp = g_run + (ex & 0xFFFF), cp = c_run + (ex >> 16);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (cls[e] == 2) {
+        if (gp < TK_MAXK) sm.gt_idx[gp] = i0 + e;
+        ++gp;
+      } else if (cls[e] == 1) {
+        const int lim = (pbits == 32) ? k_rem : TK_CAP;
+        if (cp < lim) {
+          sm.cand_key[cp] = keys[e];
+          sm.cand_idx[cp] = i0 + e;
+        }
+        ++cp;
+      }
+    }
+    g_run += tot & 0xFFFF;
+    c_run += tot >> 16;
+  }
+  __syncthreads();
+  const int G = g_run;
+  if (G + k_rem != k || G >= TK_MAXK) {
+    // cannot happen for finite inputs; leave a recognisable row rather than garbage
+    if (threadIdx.x == 0) record_error(kErrTopkOverflow);
+    for (int j = threadIdx.x; j < k; j += TK_THREADS) out[j] = -1;
+    return;
+  }
+
+  // ---------------------------------------------------------------- 3. resolve candidates
+  int S;
+  if (pbits == 32) {
+    // every candidate carries the same key: the first k_rem in index order win
+    for (int j = threadIdx.x; j < k_rem; j += TK_THREADS) sm.sel_idx[j] = sm.cand_idx[j];
+    S = k_rem;
+  } else {
+    const int C = c_run;  // <= TK_CAP here
+    while (pbits < 32) {
+      const int bits = (32 - pbits) >= 12 ? 12 : (32 - pbits);
+      const int shift = 32 - pbits - bits;
+      const int nb = 1 << bits;
+      const uint32_t mask = static_cast<uint32_t>(nb - 1);
+      const int hsh = shift + bits;
+      for (int b = threadIdx.x; b < nb; b += TK_THREADS) sm.hist[b] = 0;
+      __syncthreads();
+      for (int j = threadIdx.x; j < C; j += TK_THREADS) {
+        const uint32_t key = sm.cand_key[j];
+        if ((key >> hsh) == prefix) atomicAdd(&sm.hist[(key >> shift) & mask], 1);
+      }
+      __syncthreads();
+      find_bin(sm, nb, k_rem);
+      const int B = sm.bcast[0];
+      k_rem -= sm.bcast[1];
+      prefix = (prefix << bits) | static_cast<uint32_t>(B);
+      pbits += bits;
+      __syncthreads();
+    }
+    // prefix is now the exact k-th key T; take every key > T and the first k_rem keys == T
+    const uint32_t T = prefix;
+    const int take_eq = k_rem;
+    int gt_run = 0, eq_run = 0;
+    for (int c0 = 0; c0 < C; c0 += TK_THREADS) {
+      const int j = c0 + threadIdx.x;
+      uint32_t key = 0;
+      int isgt = 0, iseq = 0;
+      if (j < C) {
+        key = sm.cand_key[j];
+        isgt = key > T;
+        iseq = key == T;
+      }
+      int tot;
+      const int ex = block_excl_scan(isgt | (iseq << 16), sm.scan_tmp, &tot);
+      const int gt_before = gt_run + (ex & 0xFFFF);
+      const int eq_rank = eq_run + (ex >> 16);
+      const int pos = gt_before + (eq_rank < take_eq ? eq_rank : take_eq);
+      if (isgt || (iseq && eq_rank < take_eq)) sm.sel_idx[pos] = sm.cand_idx[j];
+      gt_run += tot & 0xFFFF;
+      eq_run += tot >> 16;
+    }
+    S = k - G;
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- merge two ascending lists
+  for (int p = threadIdx.x; p < G; p += TK_THREADS) {
+    const int v = sm.gt_idx[p];
+    int lo = 0, hi = S;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sm.sel_idx[mid] < v) lo = mid + 1; else hi = mid;
+    }
+    out[p + lo] = v;
+  }
+  for (int p = threadIdx.x; p < S; p += TK_THREADS) {
+    const int v = sm.sel_idx[p];
+    int lo = 0, hi = G;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sm.gt_idx[mid] < v) lo = mid + 1; else hi = mid;
+    }
+    out[p + lo] = v;
+  }
+}
+
+ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0, int k, int* idx,
+                      cudaStream_t stream) {
+  if (rows == 0) return IC_OK;
+  const int smem = static_cast<int>(sizeof(TopkSmem));
+  ic_status st = cuda_check(
+      cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+      "cudaFuncSetAttribute(topk)");
+  if (st) return st;
+  topk_kernel<<<static_cast<unsigned>(rows), TK_THREADS, smem, stream>>>(scores, ld, n, pos0, k,
+                                                                         idx);
+  st = cuda_check(cudaGetLastError(), "topk_kernel launch");
+  if (st) return st;
+  // algorithmic bytes: every candidate score read once, the index rows written once
+  const double cand = pos0 < 0 ? static_cast<double>(rows) * n
+                               : static_cast<double>(causal_pairs(rows, n, pos0));
+  trace_launch(kKindTopk, stream, 4.0 * cand + 4.0 * static_cast<double>(rows) * k);
+  return IC_OK;
+}
+
+}  // namespace ic

@@ -1,0 +1,328 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Tolerances: indexer scores rel 1e-2 / abs 1e-3 (bf16 inputs) and rel 5e-2 (fp8);
+top-k bit-exact on the same fp32 scores; index sets may differ from the oracle's
+only on near-ties with the k-th score; attention max-abs 2e-2 and mean-abs 2e-3
+(bf16 output).  Sizes span several tiles with ragged tails; every input is seeded.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_indexer_sum_b200 import binding as ic
+from sparse_attention_indexer_sum_b200 import synth
+from tests.paritylib import (IDX_RTOL_FP8, assert_attn_close, assert_scores_close,
+                             check_index_row)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy() if t.dtype == torch.bfloat16 else t.detach().cpu().numpy()
+
+
+def _sync():
+    ic.ic_device_status()
+
+
+# ------------------------------------------------------------------------------- top-k
+@pytest.mark.parametrize("rows,n,k,pos0", [(64, 5000, 2048, -1), (33, 3000, 64, 0),
+                                           (40, 2100, 2048, 2040), (7, 200000, 2048, -1)])
+def test_topk_bit_exact_random(rows, n, k, pos0):
+    g = torch.Generator().manual_seed(rows * 7 + n)
+    s = torch.randn(rows, n, generator=g)
+    got = ic.ic_topk(s.to(DEV), k, pos0=pos0)
+    _sync()
+    valid = np.full(rows, n, np.int32) if pos0 < 0 else oracle.causal_valid(rows, pos0, n)
+    ref = oracle.topk(s.numpy(), k, valid=valid)
+    np.testing.assert_array_equal(got.cpu().numpy(), ref)
+
+
+def test_topk_ties_signed_zeros_and_degenerate_rows():
+    k = 2048
+    n = 12000
+    rows = []
+    rows.append(np.zeros(n, np.float32))                                   # all zero
+    rows.append(np.full(n, 1.5, np.float32))                               # all equal
+    r = np.zeros(n, np.float32)
+    r[::2] = -0.0
+    rows.append(r)                                                         # -0 / +0 mix
+    g = np.random.default_rng(0)
+    rows.append(g.choice([0.0, 0.25, 0.5, 1.0], size=n).astype(np.float32))  # heavy ties
+    r = g.standard_normal(n).astype(np.float32)
+    r[:9000] = 0.75                                                        # > CAP equal keys
+    rows.append(r)
+    r = np.maximum(g.standard_normal(n), 0).astype(np.float32)             # ReLU-like: many zeros
+    rows.append(r)
+    r = (1.0 + g.integers(0, 3, n) * 2.0 ** -20).astype(np.float32)        # ties in low bits
+    rows.append(r)
+    rows.append(-np.abs(g.standard_normal(n)).astype(np.float32))          # all negative
+    s = np.stack(rows)
+    got = ic.ic_topk(torch.from_numpy(s).to(DEV), k).cpu().numpy()
+    _sync()
+    np.testing.assert_array_equal(got, oracle.topk(s, k))
+
+
+@pytest.mark.parametrize("n", [1, 2047, 2048, 2049, 4096])
+def test_topk_sizes_around_k(n):
+    k = 2048
+    g = torch.Generator().manual_seed(n)
+    s = torch.randn(3, n, generator=g)
+    got = ic.ic_topk(s.to(DEV), k).cpu().numpy()
+    _sync()
+    np.testing.assert_array_equal(got, oracle.topk(s.numpy(), k))
+
+
+def test_topk_strided_rows_and_causal():
+    g = torch.Generator().manual_seed(5)
+    big = torch.randn(50, 3001, generator=g)
+    view = big[:, :2999]                       # ld = 3001 (not a multiple of 4): scalar loads
+    dev = big.to(DEV)
+    got = ic.ic_topk(dev[:, :2999], 100, n=2999, pos0=2950).cpu().numpy()
+    _sync()
+    ref = oracle.topk(view.numpy(), 100, valid=oracle.causal_valid(50, 2950, 2999))
+    np.testing.assert_array_equal(got, ref)
+
+
+# ------------------------------------------------------------------------------- indexer
+def _idx_inputs(B, R, Lk, seed, dtype=torch.bfloat16):
+    g = torch.Generator().manual_seed(seed)
+    q = (torch.randn(B, R, 64, 128, generator=g) / math.sqrt(128)).to(dtype)
+    k = (torch.randn(B, Lk, 128, generator=g) / math.sqrt(128)).to(dtype)
+    w = torch.rand(B, R, 64, generator=g) / 8
+    return q, k, w
+
+
+@pytest.mark.parametrize("B,R,Lk,pos0", [(1, 1000, 1000, 0), (1, 6, 300, 200), (3, 1, 777, 776),
+                                         (2, 130, 259, 0), (1, 4, 129, 125)])
+def test_indexer_bf16_parity(B, R, Lk, pos0):
+    q, k, w = _idx_inputs(B, R, Lk, seed=B * 1000 + R)
+    got = ic.ic_indexer_scores(q.to(DEV), k.to(DEV), w.to(DEV), pos0=pos0)
+    _sync()
+    ref = oracle.indexer_scores(q.float().numpy(), k.float().numpy(), w.numpy(), pos0=pos0)
+    assert_scores_close(got.cpu().numpy(), ref)
+
+
+def test_indexer_bf16_heavy_keys_and_ld():
+    wl = synth.variant("prefill_8k", L=1500)
+    d = synth.indexer_inputs(wl, 0)
+    scores = torch.full((1500, 1600), 7.0, device=DEV)     # ld > Lk: columns >= Lk untouched
+    ic.ic_indexer_scores(d["q_idx"].to(DEV), d["k_idx"].to(DEV), d["w"].to(DEV), scores=scores)
+    _sync()
+    ref = oracle.indexer_scores(d["q_idx"].float().numpy(), d["k_idx"].float().numpy(),
+                                d["w"].numpy())
+    got = scores.cpu().numpy()
+    assert_scores_close(got[:, :1500], ref)
+    assert (got[:, 1500:] == 7.0).all()
+
+
+def test_quant_e4m3_bit_exact():
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(300, 128, generator=g) * torch.rand(300, 1, generator=g) * 5
+    x[7] = 0
+    xb = x.to(torch.bfloat16)
+    codes, scales = ic.ic_quant_e4m3_rows(xb.to(DEV))
+    _sync()
+    rc, rs = oracle.quant_rows_e4m3(xb.float().numpy())
+    np.testing.assert_array_equal(scales.cpu().numpy(), rs)
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
+
+
+@pytest.mark.parametrize("B,R,Lk,pos0", [(1, 700, 700, 0), (4, 1, 1000, 999)])
+def test_indexer_fp8_parity(B, R, Lk, pos0):
+    q, k, w = _idx_inputs(B, R, Lk, seed=77 + R)
+    qc, qs = ic.ic_quant_e4m3_rows(q.to(DEV))
+    kc, ks = ic.ic_quant_e4m3_rows(k.to(DEV))
+    got = ic.ic_indexer_scores(qc, kc, w.to(DEV), pos0=pos0, q_scale=qs, k_scale=ks)
+    _sync()
+    got = got.cpu().numpy()
+    # (i) same e4m3 values: tight
+    ref_q = oracle.indexer_scores_e4m3(qc.cpu().numpy(), qs.cpu().numpy(), kc.cpu().numpy(),
+                                       ks.cpu().numpy(), w.numpy(), pos0=pos0)
+    assert_scores_close(got, ref_q)
+    # (ii) against the unquantised bf16 inputs: rel 5e-2 with a row-RMS floor
+    ref = oracle.indexer_scores(q.float().numpy(), k.float().numpy(), w.numpy(), pos0=pos0)
+    fin = np.isfinite(ref)
+    rms = np.sqrt(np.nanmean(np.where(fin, ref, np.nan) ** 2, axis=-1, keepdims=True))
+    err = np.abs(np.where(fin, got - ref, 0))
+    lim = IDX_RTOL_FP8 * np.maximum(np.abs(np.where(fin, ref, 0)), rms)
+    assert (err <= lim).all(), float((err - lim).max())
+
+
+def test_indexer_f32_parity():
+    wl = synth.WORKLOADS["tiny_stack"]
+    d = synth.indexer_inputs(wl, 2)
+    got = ic.ic_indexer_scores(d["q_idx"].to(DEV), d["k_idx"].to(DEV), d["w"].to(DEV))
+    _sync()
+    ref = oracle.indexer_scores(d["q_idx"].numpy(), d["k_idx"].numpy(), d["w"].numpy())
+    assert_scores_close(got.cpu().numpy(), ref, atol=1e-5, rtol=1e-5)
+
+
+# ------------------------------------------------------------------------------- attention
+def _rand_idx(B, R, k, Lkv, seed, pad_from=None):
+    g = np.random.default_rng(seed)
+    idx = np.stack([np.stack([np.sort(g.permutation(Lkv)[:k]) for _ in range(R)])
+                    for _ in range(B)]).astype(np.int32)
+    if pad_from is not None:
+        for r in range(R):
+            cut = pad_from[r] if hasattr(pad_from, "__len__") else pad_from
+            idx[:, r, cut:] = -1
+    return idx
+
+
+@pytest.mark.parametrize("B,R,k,Lkv", [(1, 37, 2048, 3000), (5, 1, 2048, 2500), (1, 9, 100, 150)])
+def test_attn_mla_parity(B, R, k, Lkv):
+    g = torch.Generator().manual_seed(B * 100 + R)
+    q = torch.randn(B, R, 16, 576, generator=g).to(torch.bfloat16)
+    kv = torch.randn(B, Lkv, 576, generator=g).to(torch.bfloat16)
+    pads = [k - (r * 37) % (k // 2) for r in range(R)]
+    idx = _rand_idx(B, R, k, Lkv, seed=R, pad_from=pads)
+    idx[:, 0, 5] = -1                                   # a hole in the middle
+    scale = 1 / math.sqrt(576)
+    ws = torch.empty(ic.ic_attn_workspace_size(B, R, 16, 512, k) // 4 + 1, device=DEV)
+    lse = torch.empty(B, R, 16, device=DEV)
+    out = ic.ic_sparse_attn(q.to(DEV), kv.to(DEV), torch.from_numpy(idx).to(DEV), scale, lse=lse,
+                            workspace=ws)
+    _sync()
+    ro, rl = oracle.sparse_attn(q.float().numpy(), kv.float().numpy(), idx, scale, dv=512)
+    assert_attn_close(_np(out), ro)
+    np.testing.assert_allclose(lse.cpu().numpy(), rl, atol=2e-3, rtol=1e-3)
+
+
+def test_attn_mla_decode_split_equals_unsplit():
+    B, k, Lkv = 6, 2048, 4000
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(B, 1, 16, 576, generator=g).to(torch.bfloat16).to(DEV)
+    kv = torch.randn(B, Lkv, 576, generator=g).to(torch.bfloat16).to(DEV)
+    idx = torch.from_numpy(_rand_idx(B, 1, k, Lkv, seed=9)).to(DEV)
+    ws = torch.empty(ic.ic_attn_workspace_size(B, 1, 16, 512, k) // 4 + 1, device=DEV)
+    assert ws.numel() > 1
+    o_split = ic.ic_sparse_attn(q, kv, idx, 0.05, workspace=ws)
+    o_one = ic.ic_sparse_attn(q, kv, idx, 0.05)
+    _sync()
+    ro, _ = oracle.sparse_attn(q.float().cpu().numpy(), kv.float().cpu().numpy(),
+                               idx.cpu().numpy(), 0.05, dv=512)
+    assert_attn_close(_np(o_split), ro)
+    assert_attn_close(_np(o_one), ro)
+
+
+def test_attn_f32_mqa_parity():
+    wl = synth.WORKLOADS["tiny_stack"]
+    a = synth.attn_inputs(wl, 1)
+    idx = _rand_idx(1, wl.L, wl.k, wl.L, seed=4)[0]
+    idx[:10, 3:] = -1
+    out = ic.ic_sparse_attn(a["q"].to(DEV), a["kv"].to(DEV), torch.from_numpy(idx).to(DEV),
+                            wl.scale, v=a["v"].to(DEV))
+    _sync()
+    ro, _ = oracle.sparse_attn(a["q"].numpy(), a["kv"].numpy(), idx, wl.scale, v=a["v"].numpy())
+    np.testing.assert_allclose(out.cpu().numpy(), ro, atol=1e-5, rtol=1e-4)
+
+
+# ------------------------------------------------------------------------------- stacks
+def _stack_layers(wl, device, rows=None):
+    layers, host = [], []
+    for l in range(wl.layers):
+        d = synth.indexer_inputs(wl, l)
+        d.update(synth.attn_inputs(wl, l))
+        host.append(d)
+        dd = {k: v.to(device) for k, v in d.items()}
+        layers.append(dd)
+    return layers, host
+
+
+def _desc(wl, idx_dtype):
+    return ic.make_desc(L=wl.L, k=wl.k, H=wl.H, D=wl.D, idx_dtype=idx_dtype, heads=wl.Hq,
+                        dk=wl.Dk, dv=wl.Dv,
+                        attn_dtype=ic.IC_F32 if wl.attn == "mqa" else ic.IC_BF16,
+                        scale=wl.scale, batch=wl.batch, decode=wl.decode)
+
+
+def _run_stack(wl, pattern, layers, idx_dtype, decode=False, ws_bytes=None):
+    desc = _desc(wl, idx_dtype)
+    dev_layers = []
+    for d in layers:
+        R = 1 if decode else wl.L
+        shape = (wl.batch, R, wl.Hq, wl.Dv) if decode else (wl.L, wl.Hq, wl.Dv)
+        e = {"q_idx": d["q_idx"], "k_idx": d["k_idx"], "w": d["w"], "q": d["q"], "kv": d["kv"],
+             "v": d.get("v"), "q_scale": d.get("q_scale"), "k_scale": d.get("k_scale"),
+             "out": torch.empty(shape, dtype=d["q"].dtype, device=DEV),
+             "lse": torch.empty(shape[:-1], dtype=torch.float32, device=DEV)}
+        dev_layers.append(e)
+    nrows = wl.batch if decode else wl.L
+    t_cache = torch.full((nrows, wl.k), -7, dtype=torch.int32, device=DEV)
+    ws_bytes = ws_bytes or ic.ic_stack_workspace_size(desc)
+    ws = torch.empty(ws_bytes // 4 + 1, device=DEV)
+    fn = ic.ic_decode_step if decode else ic.ic_layer_stack
+    fn(pattern, desc, dev_layers, t_cache, ws)
+    _sync()
+    return dev_layers, t_cache
+
+
+def test_stack_tiny_f32_full_parity():
+    """Tiny 4-layer F,S,S,S fp32 stack, full tensors against the oracle stack."""
+    wl = synth.WORKLOADS["tiny_stack"]
+    layers, host = _stack_layers(wl, DEV)
+    dl, t_cache = _run_stack(wl, wl.pattern, layers, ic.IC_F32)
+    ref = oracle.layer_stack(wl.pattern, [{k: v.numpy() for k, v in h.items()} for h in host],
+                             wl.k, wl.scale, keep_scores=True)
+    # the index set: near-ties with the k-th score only
+    diffs = 0
+    T = t_cache.cpu().numpy()
+    for t in range(wl.L):
+        diffs += check_index_row(T[t], ref[0]["scores"][t], wl.k, t + 1, atol=1e-5, rtol=1e-5)
+    assert diffs <= wl.L // 20
+    # attention of every layer over the GPU's own T (S layers reuse it unchanged)
+    for l in range(wl.layers):
+        h = host[l]
+        ro, rl = oracle.sparse_attn(h["q"].numpy(), h["kv"].numpy(), T, wl.scale, v=h["v"].numpy())
+        np.testing.assert_allclose(dl[l]["out"].cpu().numpy(), ro, atol=1e-5, rtol=1e-4)
+        np.testing.assert_allclose(dl[l]["lse"].cpu().numpy(), rl, atol=1e-5, rtol=1e-5)
+
+
+def test_stack_bf16_row_blocks_and_sharing():
+    """bf16 4-layer F,S,F,S stack at L=2600 (k=2048) with a workspace of a few row
+    blocks: sampled rows of T against the oracle's scores, S layers bit-identical."""
+    wl = synth.variant("stack_32k", L=2600, pattern="F,S,F,S")
+    layers, host = _stack_layers(wl, DEV)
+    ws_bytes = 1000 * wl.L * 4                     # 1000-row blocks: ragged last block
+    dl, t_cache = _run_stack(wl, wl.pattern, layers, ic.IC_BF16, ws_bytes=ws_bytes)
+    T = t_cache.cpu().numpy()
+    # T holds the last F layer's (layer 2's) set; compare sampled rows with the oracle
+    rows = synth.sample_rows(wl.L, wl.k, 40, 1000).numpy()
+    ref = oracle.indexer_scores(host[2]["q_idx"].float().numpy(), host[2]["k_idx"].float().numpy(),
+                                host[2]["w"].numpy(), rows_sel=rows)
+    for j, t in enumerate(rows):
+        check_index_row(T[t], ref[j], wl.k, t + 1)
+    # layers 2 and 3 attend over the same T; compare their outputs on the sampled rows
+    for l in (2, 3):
+        h = host[l]
+        ro, _ = oracle.sparse_attn(h["q"][rows].float().numpy(), h["kv"].float().numpy(), T[rows],
+                                   wl.scale, dv=512)
+        assert_attn_close(_np(dl[l]["out"][torch.from_numpy(rows).to(DEV)]), ro)
+
+
+def test_decode_step_parity():
+    """Decode: 6 sequences x 1 token over a 3000-token context, fp8 indexer cache,
+    pattern F,S: T per sequence and both layers' outputs against the oracle."""
+    wl = synth.variant("decode_200k", L=3000, batch=6, pattern="F,S")
+    layers, host = _stack_layers(wl, DEV)
+    for d in layers:
+        d["q_idx"], d["q_scale"] = ic.ic_quant_e4m3_rows(d["q_idx"])
+        d["k_idx"], d["k_scale"] = ic.ic_quant_e4m3_rows(d["k_idx"])
+    dl, t_cache = _run_stack(wl, wl.pattern, layers, ic.IC_E4M3, decode=True)
+    T = t_cache.cpu().numpy()
+    d0 = layers[0]
+    ref = oracle.indexer_scores_e4m3(d0["q_idx"].cpu().numpy(), d0["q_scale"].cpu().numpy(),
+                                     d0["k_idx"].cpu().numpy(), d0["k_scale"].cpu().numpy(),
+                                     d0["w"].cpu().numpy(), pos0=wl.L - 1)
+    for b in range(wl.batch):
+        check_index_row(T[b], ref[b, 0], wl.k, wl.L)
+    for l in range(2):
+        h = host[l]
+        ro, _ = oracle.sparse_attn(h["q"].float().numpy(), h["kv"].float().numpy(), T[:, None, :],
+                                   wl.scale, dv=512)
+        assert_attn_close(_np(dl[l]["out"]), ro)
