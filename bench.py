@@ -1,0 +1,482 @@
+#!/usr/bin/env python
+"""Prefill benchmark of the DSA / IndexCache hot path on B200.
+
+One step = one pass of the whole hot path over one 200000-token prefill: the
+4-layer F,S,S,S stack through ``ic_layer_stack`` (F layer: lightning indexer ->
+exact top-k (k=2048) -> T_cache; every layer: sparse MLA attention over
+T_cache).  Inputs are seeded synthetic tensors resident in HBM (they are larger
+than L2, so no flush is needed between steps).
+
+Rank 0 prints one JSON line.  Besides the contract keys it carries:
+  roofline      the dominant kernel (the tensor-core indexer) against the
+                measured bf16 peak, from CUDA events recorded after every launch
+                inside the timed region (ic_trace_begin / ic_trace_end);
+  stages        per-kernel device time per step and its own roofline;
+  all_f         the same stack with every layer F, and the F,S,S,S speed-up;
+  e2e           the metric through the C ABI with host buffers (H2D of the
+                step's inputs and D2H of its result inside the timed region);
+  cpu_baseline  the fp64 CPU oracle on a bounded sample of rows, extrapolated.
+
+``--impl reference`` times the CPU oracle (the reference of this repository)
+on the same workload, metric and unit instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from sparse_attention_indexer_sum_b200 import synth  # noqa: E402
+
+METRIC = "prefill tokens/s (indexer+top-k+sparse attn) at L=200K; % of roofline"
+UNIT = "tokens/s"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+                "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms; only samples taken inside mark()..stop() count."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str):
+        self.dev = device_id
+        self.proc = None
+        self.t_mark = None
+        self.path = os.path.join("/tmp", "ic_clocks_%d.csv" % os.getpid())
+
+    def mark(self):
+        self.t_mark = time.time()
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception as e:  # pragma: no cover - no nvidia-smi
+            log("clock sampling unavailable:", e)
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        t_end = time.time()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        import datetime
+        with open(self.path) as f:
+            for ln in f:
+                p = [x.strip() for x in ln.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    if self.t_mark is not None and not (self.t_mark <= ts <= t_end + 0.2):
+                        continue
+                    sm.append(float(p[1]))
+                    mx = max(mx, float(p[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, p[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ workload
+def make_inputs(wl, device, pattern_all, fp8: bool, seed: int):
+    """Device tensors for every layer; indexer inputs for every layer that is F in any
+    of the patterns run."""
+    from sparse_attention_indexer_sum_b200 import binding as ic
+    kinds_any = [any(p[i] == "F" for p in pattern_all) for i in range(wl.layers)]
+    layers = []
+    for l in range(wl.layers):
+        d = {}
+        if kinds_any[l]:
+            d.update(synth.indexer_inputs(wl, l, device=device, seed=seed))
+            if fp8:
+                d["q_idx"], d["q_scale"] = ic.ic_quant_e4m3_rows(d["q_idx"])
+                d["k_idx"], d["k_scale"] = ic.ic_quant_e4m3_rows(d["k_idx"])
+        d.update(synth.attn_inputs(wl, l, device=device, seed=seed))
+        d["out"] = torch.empty(wl.L, wl.Hq, wl.Dv, dtype=torch.bfloat16, device=device)
+        d["lse"] = torch.empty(wl.L, wl.Hq, dtype=torch.float32, device=device)
+        layers.append(d)
+        torch.cuda.synchronize()
+    return layers
+
+
+def kinds_of(pattern):
+    return [c for c in pattern if c in "FS"]
+
+
+def run_ours(args, rank, world, local_rank):
+    from sparse_attention_indexer_sum_b200 import binding as ic
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    wl = synth.WORKLOADS[args.workload]
+    assert not wl.decode and wl.attn == "mla", "bench workloads are MLA prefill stacks"
+    pattern = wl.pattern
+    allf = ",".join("F" * wl.layers)
+    fp8 = args.indexer == "e4m3"
+    t0 = time.time()
+    layers = make_inputs(wl, dev, [kinds_of(pattern)] + ([kinds_of(allf)] if args.compare else []),
+                         fp8, seed=rank)
+    log("rank %d: inputs ready in %.1f s (%.1f GB allocated)" %
+        (rank, time.time() - t0, torch.cuda.memory_allocated(dev) / 1e9))
+    desc = ic.make_desc(L=wl.L, k=wl.k, H=wl.H, D=wl.D,
+                        idx_dtype=ic.IC_E4M3 if fp8 else ic.IC_BF16, heads=wl.Hq, dk=wl.Dk,
+                        dv=wl.Dv, attn_dtype=ic.IC_BF16, scale=wl.scale)
+    ws = torch.empty(ic.ic_stack_workspace_size(desc) // 4 + 1, dtype=torch.float32, device=dev)
+    t_cache = torch.empty(wl.L, wl.k, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(pat=pattern):
+        ic.ic_layer_stack(pat, desc, layers, t_cache, ws, stream=stream)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    ic.ic_device_status(stream)
+    barrier()
+    clocks = ClockSampler("GPU-%s" % torch.cuda.get_device_properties(dev).uuid)
+    clocks.start()
+    time.sleep(0.5)
+    clocks.mark()
+    cap = max(4096, 256 * args.steps)
+    ic.ic_trace_begin(cap, stream=stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    n_launch, trace = ic.ic_trace_end(cap)
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms)
+    ic.ic_device_status(stream)
+
+    # per-kernel device time and algorithmic work over the timed region
+    agg = {}
+    for name, kms, work in trace:
+        a = agg.setdefault(name, [0, 0.0, 0.0])
+        a[0] += 1
+        a[1] += kms
+        a[2] += work
+    tot_ms = sum(a[1] for a in agg.values())
+    dom = "indexer_tc_e4m3" if fp8 else "indexer_tc_bf16"
+    d_n, d_ms, d_work = agg.get(dom, [0, 0.0, 0.0])
+    bf16_peak = peaks["bf16_sustained"]
+    peak = bf16_peak * (2.0 if fp8 else 1.0)   # e4m3 dense peak = 2x bf16 (nominal ratio)
+    achieved = d_work / (d_ms * 1e-3) / 1e12 if d_ms > 0 else 0.0
+    stages = {}
+    for name, (n, kms, work) in sorted(agg.items()):
+        st = {"launches_per_step": n / args.steps, "ms_per_step": kms / args.steps,
+              "share": kms / tot_ms if tot_ms else 0.0}
+        if name.startswith("indexer_tc"):
+            st.update(bound="tensor", achieved_tflops=work / (kms * 1e-3) / 1e12,
+                      unit="TFLOP/s")
+        else:
+            st.update(bound="hbm", achieved_gbs=work / (kms * 1e-3) / 1e9,
+                      frac_hbm=work / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"], unit="GB/s")
+        stages[name] = st
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak if peak else None, "traffic": None,
+                "peak_source": "%s bf16 sustained %.1f TFLOP/s%s" % (
+                    peaks["source"], bf16_peak, " x2 (e4m3 nominal ratio)" if fp8 else ""),
+                "work_per_launch": d_work / d_n if d_n else None,
+                "launches": d_n, "ms_per_launch": d_ms / d_n if d_n else None}
+    value = world * wl.L / (ms * 1e-3)
+    log("rank %d: %.2f ms/step, %.0f tokens/s, indexer %.1f TFLOP/s" % (rank, ms, value, achieved))
+
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3+bf16" if fp8 else "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "L": wl.L, "layers": wl.layers, "pattern": pattern,
+                   "k": wl.k, "indexer": "H_I=64 d_I=128 %s (fp32 accumulate)" %
+                   ("e4m3 per-row scales" if fp8 else "bf16"),
+                   "attention": "absorbed MLA 16 heads x 576 -> 512, bf16",
+                   "batch_per_gpu": 1, "parallelism": "independent sequence per GPU" if world > 1
+                   else "single GPU", "l2": "inputs larger than L2 (no flush needed)"},
+        "gpu_launches": n_launch, "roofline": roofline, "stages": stages, "clocks": clk,
+    }
+
+    if args.compare:
+        for _ in range(1):
+            step(allf)
+        barrier()
+        ka = max(2, args.steps // 2)
+        e0.record(stream)
+        for _ in range(ka):
+            step(allf)
+        e1.record(stream)
+        barrier()
+        ms_f = max_over_ranks(e0.elapsed_time(e1) / ka)
+        res["all_f"] = {"pattern": allf, "ms_per_step": ms_f,
+                        "value": world * wl.L / (ms_f * 1e-3),
+                        "speedup_fsss_over_all_f": ms_f / ms}
+
+    if args.e2e:
+        res["e2e"] = run_e2e(wl, layers, pattern, desc, t_cache, ws, stream, dev, args, barrier,
+                             max_over_ranks, world)
+    if args.cpu_baseline and rank == 0 and world == 1:
+        res["cpu_baseline"] = cpu_baseline(wl, layers, budget_s=args.cpu_budget)
+    return res
+
+
+def run_e2e(wl, layers, pattern, desc, t_cache, ws, stream, dev, args, barrier, max_over_ranks,
+            world):
+    """The metric through the C ABI with HOST buffers: every step copies its inputs from
+    pinned host memory and reads its result (last layer's output and the index set) back."""
+    from sparse_attention_indexer_sum_b200 import binding as ic
+    kinds = kinds_of(pattern)
+    names_f = ["q_idx", "q_scale", "k_idx", "k_scale", "w", "q", "kv"]
+    try:
+        host_in = []
+        for l, d in enumerate(layers):
+            hs = {}
+            for n in names_f:
+                if n in d and (kinds[l] == "F" or n in ("q", "kv")):
+                    h = torch.empty(d[n].shape, dtype=d[n].dtype, pin_memory=True)
+                    h.copy_(d[n])
+                    hs[n] = h
+            host_in.append(hs)
+        out_h = torch.empty(layers[-1]["out"].shape, dtype=torch.bfloat16, pin_memory=True)
+        t_h = torch.empty(t_cache.shape, dtype=torch.int32, pin_memory=True)
+    except RuntimeError as e:
+        return {"value": None, "unit": UNIT, "error": "pinned host buffers: %s" % e}
+    h2d = sum(t.numel() * t.element_size() for hs in host_in for t in hs.values())
+    d2h = out_h.numel() * out_h.element_size() + t_h.numel() * t_h.element_size()
+
+    def step():
+        for d, hs in zip(layers, host_in):
+            for n, h in hs.items():
+                d[n].copy_(h, non_blocking=True)
+        ic.ic_layer_stack(pattern, desc, layers, t_cache, ws, stream=stream)
+        out_h.copy_(layers[-1]["out"], non_blocking=True)
+        t_h.copy_(t_cache, non_blocking=True)
+
+    step()
+    barrier()
+    ke = max(2, min(args.steps, 3))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(ke):
+        step()
+    e1.record(stream)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / ke)
+    return {"value": world * wl.L / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke}
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+class OracleSample:
+    """Host (fp64) copies of what the oracle needs for sampled query rows of the stack."""
+
+    def __init__(self, wl, layers_dev):
+        self.wl = wl
+        self.kinds = kinds_of(wl.pattern)
+        self.layers = layers_dev
+        self.k_idx = {}
+        self.kv = []
+        for l, d in enumerate(layers_dev):
+            if self.kinds[l] == "F":
+                self.k_idx[l] = d["k_idx"].double().cpu().numpy()
+            self.kv.append(d["kv"].double().cpu().numpy())
+
+    def run(self, rows, nthreads):
+        """Runs the oracle stack on the query rows `rows`; returns per-stage seconds."""
+        import oracle
+        wl = self.wl
+        rows_t = torch.from_numpy(rows.astype(np.int64)).to(self.layers[0]["q"].device)
+        t_idx = t_topk = t_attn = 0.0
+        T = None
+        for l, d in enumerate(self.layers):
+            if self.kinds[l] == "F":
+                q = d["q_idx"][rows_t].double().cpu().numpy()
+                w = d["w"][rows_t].double().cpu().numpy()
+                t0 = time.perf_counter()
+                I = oracle.indexer_scores_at(q, self.k_idx[l], w, rows, nthreads=nthreads)
+                t_idx += time.perf_counter() - t0
+                I32 = I.astype(np.float32)
+                t0 = time.perf_counter()
+                T = oracle.topk(I32, wl.k, valid=(rows + 1).astype(np.int32), nthreads=nthreads)
+                t_topk += time.perf_counter() - t0
+            qa = d["q"][rows_t].double().cpu().numpy()
+            t0 = time.perf_counter()
+            oracle.sparse_attn(qa, self.kv[l], T, wl.scale, dv=wl.Dv, nthreads=nthreads)
+            t_attn += time.perf_counter() - t0
+        return t_idx, t_topk, t_attn
+
+
+def extrapolate(wl, rows, t_idx, t_topk, t_attn):
+    """Full-workload seconds from the sample: indexer and top-k scale with the causal pair
+    count (sum of t+1 over rows), attention with the row count."""
+    pairs_sample = float((rows.astype(np.float64) + 1).sum())
+    pairs_total = wl.L * (wl.L + 1) / 2.0
+    return (t_idx + t_topk) * pairs_total / pairs_sample + t_attn * wl.L / len(rows)
+
+
+def cpu_baseline(wl, layers_dev, budget_s=15.0):
+    import oracle
+    oracle.build()
+    nthreads = oracle.default_threads()
+    samp = OracleSample(wl, layers_dev)
+    g = np.random.default_rng(1234)
+    # calibrate on one row per thread, then size the sample to the time budget
+    rows = np.sort(g.choice(wl.L, size=nthreads, replace=False)).astype(np.int64)
+    t = samp.run(rows, nthreads)
+    per_round = max(sum(t), 1e-3)
+    rounds = int(max(1, min(64, (budget_s - per_round) / per_round)))
+    more = np.sort(g.choice(wl.L, size=rounds * nthreads, replace=False)).astype(np.int64)
+    t2 = samp.run(more, nthreads)
+    rows_all = np.concatenate([rows, more])
+    t_all = [a + b for a, b in zip(t, t2)]
+    total = extrapolate(wl, rows_all, *t_all)
+    return {"value": wl.L / total, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": "%d random query rows of the %d-token %s stack (fp64 indexer, top-k and "
+                      "attention on all %d layers), %.1f s measured on %d host threads, "
+                      "extrapolated to the full step by causal pair count (indexer, top-k) "
+                      "and row count (attention)" % (len(rows_all), wl.L, wl.pattern, wl.layers,
+                                                     sum(t_all), nthreads),
+            "extrapolated_s_per_step": total}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: each step is a bounded sample of the workload."""
+    import oracle
+    oracle.build()
+    wl = synth.WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    # inputs come from the same generators (drawn on the GPU when there is one)
+    layers = []
+    kinds = kinds_of(wl.pattern)
+    for l in range(wl.layers):
+        d = {}
+        if kinds[l] == "F":
+            d.update(synth.indexer_inputs(wl, l, device=dev))
+        d.update(synth.attn_inputs(wl, l, device=dev))
+        layers.append(d)
+    nthreads = oracle.default_threads()
+    samp = OracleSample(wl, layers)
+    g = np.random.default_rng(99)
+    n = nthreads
+    totals = []
+    for s in range(args.warmup + args.steps):
+        rows = np.sort(g.choice(wl.L, size=n, replace=False)).astype(np.int64)
+        t_idx, t_topk, t_attn = samp.run(rows, nthreads)
+        if s >= args.warmup:
+            totals.append(extrapolate(wl, rows, t_idx, t_topk, t_attn))
+    sec = statistics.mean(totals)
+    value = wl.L / sec
+    sample = ("%d random query rows per step of the %d-token F,S,S,S stack, fp64 oracle on %d "
+              "host threads, extrapolated by causal pair count" % (n, wl.L, nthreads))
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "L": wl.L, "layers": wl.layers,
+                       "pattern": wl.pattern, "k": wl.k},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(nthreads, n),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill_200k",
+                    choices=["prefill_200k", "stack_32k", "prefill_8k"])
+    ap.add_argument("--indexer", default="bf16", choices=["bf16", "e4m3"])
+    ap.add_argument("--no-compare", dest="compare", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("note: fewer than 3 warm-up steps requested")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -138,6 +138,27 @@ def indexer_scores(q, k, w, pos0: int = 0, rows_sel=None, nthreads: int | None =
     return out[0] if squeeze else out
 
 
+def indexer_scores_at(q_rows, k, w_rows, positions, nthreads: int | None = None):
+    """Indexer scores of a few query rows at arbitrary positions (no batch axis).
+
+    q_rows [n, H, D], w_rows [n, H], positions [n]; k [Lk, D].  Row j is scored at
+    position positions[j] (keys s <= positions[j]).  One call of the same routine per
+    row, spread over a thread pool (the C routine releases the GIL).
+    Returns [n, Lk] fp64.
+    """
+    from concurrent.futures import ThreadPoolExecutor
+    q_rows, k, w_rows = _f64(q_rows), _f64(k), _f64(w_rows)
+    pos = [int(p) for p in positions]
+    out = np.empty((len(pos), k.shape[0]), dtype=np.float64)
+
+    def one(j):
+        out[j] = indexer_scores(q_rows[j:j + 1], k, w_rows[j:j + 1], pos0=pos[j], nthreads=1)[0]
+
+    with ThreadPoolExecutor(max_workers=nthreads or default_threads()) as ex:
+        list(ex.map(one, range(len(pos))))
+    return out
+
+
 def indexer_scores_e4m3(q_codes, q_scale, k_codes, k_scale, w, pos0: int = 0, rows_sel=None,
                         nthreads: int | None = None):
     """The indexer on per-row e4m3 inputs: the same definition on the dequantised values
