@@ -144,7 +144,7 @@ ic_status ic_topk(const float* scores, long rows, int n, long ld, long pos0, int
  *   lse[b, r, h]    = log sum_j exp(z_j)      (natural log; -inf if J is empty)
  * Two forms:
  *   v == NULL  absorbed MLA: V = kv[..., :dv] (the first dv latent dims);
- *              dt = IC_BF16, dk = 576, dv = 512, heads = 16; out bf16.
+ *              dt = IC_BF16, dk = 576, dv = 512, heads = 16, k <= 2048; out bf16.
  *   v != NULL  MQA with separate values v [batch, Lkv, dv]; dt = IC_F32,
  *              dk, dv <= 256, heads <= 64; out f32.
  *   q   [batch, rows, heads, dk]; kv [batch, Lkv, ld_kv] (ld_kv >= dk, elements);

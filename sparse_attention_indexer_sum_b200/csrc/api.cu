@@ -132,6 +132,7 @@ static ic_status check_attn(const void* q, const void* kv, long ld_kv, const voi
                   static_cast<int>(dt), heads, dk, dv);
     if (!aligned(q, 16) || !aligned(kv, 16) || (ld_kv % 8) != 0)
       return fail(IC_ERR_INVALID_ARG, "attn: q/kv rows must be 16-byte aligned");
+    if (k > 2048) return fail(IC_ERR_UNSUPPORTED, "attn: absorbed MLA needs k <= 2048");
   } else {
     if (dt != IC_F32 || heads < 1 || heads > 64 || dk < 1 || dk > 256 || dv < 1 || dv > 256)
       return fail(IC_ERR_UNSUPPORTED, "attn: MQA form needs fp32, heads <= 64, dk, dv <= 256");

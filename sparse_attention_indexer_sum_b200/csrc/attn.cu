@@ -7,18 +7,28 @@
 //
 // The work is bound by gathering k latent rows (1152 B each) per query: with
 // 16 heads there are only ~30 flops per gathered byte, far below the tensor
-// ridge.  So the kernel is built around the gather: 16-byte cp.async row copies
-// into a double-buffered shared tile of 32 rows (padded rows: conflict-free
-// ldmatrix), and the two small contractions per tile -- S = Q K^T (16 x 32 x 576)
-// and O += P V (16 x 512 x 32) -- on the warp-level bf16 tensor-core MMA, whose
-// M = 16 matches the 16 heads exactly.  Softmax is online (running max / sum
-// per head, base 2).
-//
-// CTA = 8 warps, one (query, split) item.  QK: warp w covers keys 8(w%4)..+8
-// over dims 288(w/4)..+288 with its slice of Q held in registers; the two
-// half-dim partial scores meet in shared memory.  PV: warp w owns output dims
-// 64w..+64.  Decode-sized batches split each index list over several CTAs;
-// their unnormalised partial outputs are merged by attn_combine_kernel.
+// ridge.  So the kernel is built around the gather:
+//   * one producer warp issues one TMA bulk copy (cp.async.bulk, 1152 B) per
+//     selected row straight into a 4-stage ring of 32-row shared tiles, each
+//     stage completing on an mbarrier by transaction count -- up to 147 KB of
+//     gathers in flight per SM, with no per-thread copy instructions; each
+//     item's index list arrives by one more bulk copy, one item ahead;
+//   * eight consumer warps run S = Q K^T (16 x 32 x 576) and O += P V
+//     (16 x 512 x 32) on the warp-level bf16 tensor-core MMA, whose M = 16 is
+//     exactly the 16 heads, with an online softmax in base 2;
+//   * CTAs are persistent (one per SM) and walk (query, split) items
+//     round-robin, so the producer streams the next query's rows while the
+//     consumers finish the current one, and neighbouring queries (which share
+//     many selected rows) run at the same time and hit in L2.
+// Shared rows are padded to 1168 B so that ldmatrix is bank-conflict free.
+// QK: consumer warp w covers keys 16(w%2)..+16 over dims 144(w/2)..+144 with
+// its quarter of Q in registers (four accumulator chains); the four partial
+// scores meet in shared memory, behind the tile's only barrier.  Every warp
+// then rebuilds the softmax of all 16 heads for the tile directly in its PV
+// A fragments (the running max and sum live, identical, in every warp's
+// registers).  PV: warp w owns output dims 64w..+64.  Decode-sized batches split
+// each index list over several items; their unnormalised partial outputs are
+// merged by attn_combine_kernel.
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
@@ -28,19 +38,27 @@ constexpr int AT_H = 16;
 constexpr int AT_DK = 576;
 constexpr int AT_DV = 512;
 constexpr int AT_BK = 32;                   // keys per tile
-constexpr int AT_THREADS = 256;
+constexpr int AT_STAGES = 4;
+constexpr int AT_MAXK = 2048;               // longest index list of one item
+constexpr int AT_CONSUMERS = 256;           // 8 consumer warps
+constexpr int AT_THREADS = AT_CONSUMERS + 32;
 constexpr int AT_ROWB = AT_DK * 2 + 16;     // padded shared row: 1168 B
-constexpr int AT_CHUNKS = AT_DK * 2 / 16;   // 72 16-byte chunks per row
-constexpr int AT_PROWB = 80;                // padded P row (32 bf16 + 16 B)
+constexpr uint32_t AT_ROW_BYTES = AT_DK * 2;  // 1152 B gathered per row
+
+constexpr int AT_SROW = 40;  // padded partial-score row (floats): conflict-free 64-bit access
 
 struct AttnSmem {
-  alignas(16) uint8_t kv[2][AT_BK][AT_ROWB];  // 74752 B
-  alignas(16) uint8_t q[AT_H][AT_ROWB];       // 18688 B
-  alignas(16) float s_part[2][AT_H][AT_BK];   // 4096 B
-  alignas(16) uint8_t p[AT_H][AT_PROWB];      // 1280 B
-  int idx[2][AT_BK];
-  float m[AT_H], l[AT_H], alpha[AT_H];
-  int last_valid;
+  alignas(128) uint8_t kv[AT_STAGES][AT_BK][AT_ROWB];  // 149504 B
+  alignas(128) uint8_t q[AT_H][AT_ROWB];               // 18688 B
+  alignas(16) float s_part[2][4][AT_H][AT_SROW];       // double-buffered partial scores
+  alignas(16) int ibuf[2][AT_MAXK];                    // index lists: this item / the next
+  unsigned vmask[AT_STAGES];                           // bit j: row j of the stage is valid
+  int last[AT_STAGES];
+  alignas(8) uint64_t full[AT_STAGES];
+  uint64_t empty[AT_STAGES];
+  uint64_t qfull, qempty;
+  uint64_t ifull[2];
+  int abort;
 };
 
 struct AttnArgs {
@@ -51,21 +69,21 @@ struct AttnArgs {
   int B, R, Lkv, k;
   float scale_log2;         // softmax scale * log2(e)
   int nsplit, chunk;        // index list split into nsplit chunks of `chunk` entries
+  long items;               // B * R * nsplit
+  int idx_bulk;             // index rows 16-byte aligned: fetch each list with one bulk copy
   __nv_bfloat16* out;       // [B, R, 16, 512]   (nsplit == 1)
   float* lse;               // [B, R, 16] or null (nsplit == 1)
-  float* part_o;            // [B*R*nsplit, 16, 512] (nsplit > 1)
-  float* part_ml;           // [B*R*nsplit, 16, 2]   (nsplit > 1)
+  float* part_o;            // [items, 16, 512] (nsplit > 1)
+  float* part_ml;           // [items, 16, 2]   (nsplit > 1)
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
@@ -93,203 +111,424 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Issue the copies of tile t (index-list entries j0 .. j0+31, clipped at `end`)
-// into buffer `buf`; rows whose index is < 0 (or past the end) become zeros.
-__device__ __forceinline__ void gather_tile(AttnSmem& sm, const AttnArgs& a, const int* irow,
-                                            const __nv_bfloat16* kvb, int j0, int end, int buf) {
-  for (int c = threadIdx.x; c < AT_BK * AT_CHUNKS; c += AT_THREADS) {
-    const int row = c / AT_CHUNKS, ch = c % AT_CHUNKS;
-    const int j = j0 + row;
-    int s = (j < end) ? __ldg(irow + j) : -1;
-    if (s >= a.Lkv) s = -1;
-    uint8_t* dst = &sm.kv[buf][row][ch * 16];
-    if (s >= 0)
-      cp_async16(smem_u32(dst), reinterpret_cast<const uint8_t*>(kvb + static_cast<long>(s) * a.ld_kv) + ch * 16);
-    else
-      *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-    if (ch == 0) sm.idx[buf][row] = s;
+struct AttnItem {
+  long qrow;
+  int beg, end;
+};
+__device__ __forceinline__ AttnItem attn_item(const AttnArgs& a, long it) {
+  AttnItem x;
+  x.qrow = it / a.nsplit;
+  const int sp = static_cast<int>(it % a.nsplit);
+  x.beg = sp * a.chunk;
+  x.end = min(x.beg + a.chunk, a.k);
+  if (x.end < x.beg) x.end = x.beg;
+  return x;
+}
+
+// ---------------------------------------------------------------- producer warp
+// Starts loading the index list of item `it` into ibuf[b]: one bulk copy when the
+// rows are 16-byte aligned (k % 4 == 0), else plain loads by the warp.
+__device__ __forceinline__ void attn_load_indices(AttnSmem& sm, const AttnArgs& a, long it, int b,
+                                                  bool bulk) {
+  const int lane = threadIdx.x & 31;
+  const AttnItem x = attn_item(a, it);
+  const int cnt = x.end - x.beg;
+  const int* src = a.idx + x.qrow * a.k + x.beg;
+  if (bulk) {
+    if (lane == 0) {
+      const uint32_t bar = smem_u32(&sm.ifull[b]);
+      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(cnt) * 4u);
+      if (cnt > 0) bulk_g2s(smem_u32(&sm.ibuf[b][0]), src, static_cast<uint32_t>(cnt) * 4u, bar);
+    }
+  } else {
+    for (int j = lane; j < cnt; j += 32) sm.ibuf[b][j] = __ldg(src + j);
+    __syncwarp();
   }
 }
 
-__global__ void __launch_bounds__(AT_THREADS, 2) attn_mla_kernel(const AttnArgs a) {
-  extern __shared__ __align__(16) uint8_t at_smem_raw[];
-  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(at_smem_raw);
+__device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
+  const int lane = threadIdx.x & 31;
+  volatile int* abort = &sm.abort;
+  const bool bulk = a.idx_bulk != 0;
+  int stage = 0;
+  uint32_t ph = 0;
+  int qloads = 0;
+  long issued = 0;
+  uint32_t iph[2] = {0u, 0u};
+  int ipending[2] = {0, 0};
+  const uint32_t kv0 = smem_u32(&sm.kv[0][0][0]);
+  int ib = 0;
+  if (blockIdx.x < a.items) {
+    attn_load_indices(sm, a, blockIdx.x, 0, bulk);
+    ipending[0] = bulk;
+  }
+  for (long it = blockIdx.x; it < a.items; it += gridDim.x, ib ^= 1) {
+    const AttnItem x = attn_item(a, it);
+    const int cnt = x.end - x.beg;
+    const long b = x.qrow / a.R;
+    const __nv_bfloat16* kvb = a.kv + b * static_cast<long>(a.Lkv) * a.ld_kv;
+    if (bulk) {
+      if (!mbar_wait(smem_u32(&sm.ifull[ib]), iph[ib], abort, kErrTimeoutProducer)) break;
+      iph[ib] ^= 1;
+      ipending[ib] = 0;
+    }
+    const int* ilist = sm.ibuf[ib];
+    // trailing -1 entries need no tiles: the last valid entry of the list
+    int lv = -1;
+    for (int j = lane; j < cnt; j += 32) {
+      const int s = ilist[j];
+      if (s >= 0 && s < a.Lkv) lv = j;
+    }
+    lv = __reduce_max_sync(0xffffffffu, lv);
+    const int ntiles = (lv >= 0) ? lv / AT_BK + 1 : 0;
+    // the next item's list streams in while this one's rows are gathered
+    const long nit = it + gridDim.x;
+    if (nit < a.items) {
+      attn_load_indices(sm, a, nit, ib ^ 1, bulk);
+      ipending[ib ^ 1] = bulk;
+    }
+    // the item's queries, once the consumers hold the previous ones in registers
+    if (qloads > 0 &&
+        !mbar_wait(smem_u32(&sm.qempty), (qloads - 1) & 1, abort, kErrTimeoutProducer))
+      break;
+    if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sm.qfull), AT_H * AT_ROW_BYTES);
+    __syncwarp();
+    if (lane < AT_H)
+      bulk_g2s(smem_u32(&sm.q[lane][0]), a.q + (x.qrow * AT_H + lane) * AT_DK, AT_ROW_BYTES,
+               smem_u32(&sm.qfull));
+    ++qloads;
+    const int nt = ntiles > 0 ? ntiles : 1;  // an empty item still ends with one (empty) tile
+    bool ok = true;
+    for (int t = 0; t < nt; ++t) {
+      if (!mbar_wait(smem_u32(&sm.empty[stage]), ph ^ 1, abort, kErrTimeoutProducer)) {
+        ok = false;
+        break;
+      }
+      const int j = t * AT_BK + lane;
+      int s = (t < ntiles && j < cnt) ? ilist[j] : -1;
+      if (s >= a.Lkv) s = -1;
+      const unsigned valid = __ballot_sync(0xffffffffu, s >= 0);
+      if (lane == 0) {
+        sm.vmask[stage] = valid;
+        sm.last[stage] = (t == nt - 1);
+      }
+      const uint32_t fb = smem_u32(&sm.full[stage]);
+      if (lane == 0)
+        mbar_arrive_expect_tx(fb, __popc(valid) * AT_ROW_BYTES);
+      else
+        mbar_arrive(fb);
+      if (s >= 0)
+        bulk_g2s(kv0 + (stage * AT_BK + lane) * AT_ROWB, kvb + static_cast<long>(s) * a.ld_kv,
+                 AT_ROW_BYTES, fb);
+      ++issued;
+      if (++stage == AT_STAGES) {
+        stage = 0;
+        ph ^= 1;
+      }
+    }
+    if (!ok) break;
+  }
+  if (*abort) {
+    // let every copy still in flight land before the CTA exits
+    volatile int never = 0;
+    const long n = issued < AT_STAGES ? issued : AT_STAGES;
+    for (long j = issued - n; j < issued; ++j)
+      (void)mbar_wait(smem_u32(&sm.full[j % AT_STAGES]), static_cast<uint32_t>((j / AT_STAGES) & 1),
+                      &never, kErrTimeoutDrain);
+    if (qloads > 0) (void)mbar_wait(smem_u32(&sm.qfull), (qloads - 1) & 1, &never, kErrTimeoutDrain);
+    for (int b2 = 0; b2 < 2; ++b2)
+      if (ipending[b2]) (void)mbar_wait(smem_u32(&sm.ifull[b2]), iph[b2], &never, kErrTimeoutDrain);
+  }
+}
+
+// ---------------------------------------------------------------- consumer warps
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Partial scores of this warp: Q[:, dims 144kq..+144] . K[keys 16kh..16kh+15] of the
+// tile at kvbase, four accumulator chains (c[0..1]: keys +0..7, c[2..3]: keys +8..15).
+__device__ __forceinline__ void attn_qk(uint32_t kvbase, const uint32_t (&qa)[9][4], int kq,
+                                        int kh, int lane, float (&c)[4][4]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) c[u][0] = c[u][1] = c[u][2] = c[u][3] = 0.f;
+  const int krow = 16 * kh + (lane & 7) + 8 * (lane >> 4);
+  const uint32_t rowaddr = kvbase + krow * AT_ROWB;
+#pragma unroll
+  for (int j = 0; j < 9; ++j) {
+    uint32_t b0, b1, b2, b3;
+    const int col = kq * 144 + 16 * j + 8 * ((lane >> 3) & 1);
+    ldsm_x4(rowaddr + col * 2, b0, b1, b2, b3);
+    mma_bf16(c[(j & 1)], qa[j], b0, b1);
+    mma_bf16(c[2 + (j & 1)], qa[j], b2, b3);
+  }
+}
+
+__device__ __forceinline__ void attn_store_partial(float* sp, const float (&c)[4][4], int kh,
+                                                   int g, int cq) {
+  const int k0 = 16 * kh + 2 * cq;
+  *reinterpret_cast<float2*>(sp + g * AT_SROW + k0) =
+      make_float2(c[0][0] + c[1][0], c[0][1] + c[1][1]);
+  *reinterpret_cast<float2*>(sp + (g + 8) * AT_SROW + k0) =
+      make_float2(c[0][2] + c[1][2], c[0][3] + c[1][3]);
+  *reinterpret_cast<float2*>(sp + g * AT_SROW + k0 + 8) =
+      make_float2(c[2][0] + c[3][0], c[2][1] + c[3][1]);
+  *reinterpret_cast<float2*>(sp + (g + 8) * AT_SROW + k0 + 8) =
+      make_float2(c[2][2] + c[3][2], c[2][3] + c[3][3]);
+}
+
+// Online softmax of heads g, g+8 over one tile's 32 keys from the four partials at
+// sp0, written as the two bf16 A fragments of P; rescales o and updates m, l.
+__device__ __forceinline__ void attn_softmax(const float* sp0, unsigned vm, float scale_log2,
+                                             int g, int cq, float& m0, float& m1, float& l0,
+                                             float& l1, float (&o)[8][4], uint32_t (&pa)[2][4]) {
+  constexpr int PSTRIDE = AT_H * AT_SROW;  // floats between the four dim-quarter partials
+  float z[2][2][4];                        // [ks][head g / g+8][key 2c, 2c+1, 2c+8, 2c+9]
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int row = (g + 8 * hh) * AT_SROW + 16 * ks + 2 * cq;
+      float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        const float2 u = *reinterpret_cast<const float2*>(sp0 + qq * PSTRIDE + row);
+        const float2 v = *reinterpret_cast<const float2*>(sp0 + qq * PSTRIDE + row + 8);
+        lo.x += u.x;
+        lo.y += u.y;
+        hi.x += v.x;
+        hi.y += v.y;
+      }
+      z[ks][hh][0] = lo.x * scale_log2;
+      z[ks][hh][1] = lo.y * scale_log2;
+      z[ks][hh][2] = hi.x * scale_log2;
+      z[ks][hh][3] = hi.y * scale_log2;
+    }
+    const int k0 = 16 * ks + 2 * cq;
+    const bool v0 = (vm >> k0) & 1, v1 = (vm >> (k0 + 1)) & 1;
+    const bool v8 = (vm >> (k0 + 8)) & 1, v9 = (vm >> (k0 + 9)) & 1;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      if (!v0) z[ks][hh][0] = -INFINITY;
+      if (!v1) z[ks][hh][1] = -INFINITY;
+      if (!v8) z[ks][hh][2] = -INFINITY;
+      if (!v9) z[ks][hh][3] = -INFINITY;
+    }
+  }
+  float t0 = -INFINITY, t1 = -INFINITY;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      t0 = fmaxf(t0, z[ks][0][e]);
+      t1 = fmaxf(t1, z[ks][1][e]);
+    }
+  t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, 1));
+  t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, 1));
+  t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, 2));
+  t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, 2));
+  const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
+  // a head with no valid key so far keeps weight 0 and scale 1
+  const float al0 = (n0 == -INFINITY) ? 1.f : fast_exp2(m0 - n0);
+  const float al1 = (n1 == -INFINITY) ? 1.f : fast_exp2(m1 - n1);
+  const float b0 = (n0 == -INFINITY) ? 0.f : n0, b1 = (n1 == -INFINITY) ? 0.f : n1;
+  float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    float e0[4], e1[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      e0[e] = fast_exp2(z[ks][0][e] - b0);  // exp2(-inf) = 0
+      e1[e] = fast_exp2(z[ks][1][e] - b1);
+      r0 += e0[e];
+      r1 += e1[e];
+    }
+    pa[ks][0] = pack_bf16(e0[0], e0[1]);
+    pa[ks][1] = pack_bf16(e1[0], e1[1]);
+    pa[ks][2] = pack_bf16(e0[2], e0[3]);
+    pa[ks][3] = pack_bf16(e1[2], e1[3]);
+  }
+  r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+  r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+  r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+  r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+  l0 = l0 * al0 + r0;
+  l1 = l1 * al1 + r1;
+  m0 = n0;
+  m1 = n1;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    o[i][0] *= al0;
+    o[i][1] *= al0;
+    o[i][2] *= al1;
+    o[i][3] *= al1;
+  }
+}
+
+// O[:, 64w..64w+64) += P V for the tile at kvbase.
+__device__ __forceinline__ void attn_pv(uint32_t kvbase, const uint32_t (&pa)[2][4], int warp,
+                                        int lane, float (&o)[8][4]) {
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    const int vrow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+    for (int np = 0; np < 4; ++np) {
+      uint32_t b0, b1, b2, b3;
+      const int col = 64 * warp + 16 * np + 8 * (lane >> 4);
+      ldsm_x4_t(kvbase + vrow * AT_ROWB + col * 2, b0, b1, b2, b3);
+      mma_bf16(o[2 * np], pa[ks], b0, b1);
+      mma_bf16(o[2 * np + 1], pa[ks], b2, b3);
+    }
+  }
+}
+
+// Software-pipelined per item: while tile t's softmax and P V run, the QK of tile
+// t+1 is already in flight; one barrier per tile publishes the partial scores and
+// retires tile t's stage.
+__device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long item = blockIdx.x;  // (b * R + r) * nsplit + sp
-  const long qrow = item / a.nsplit;
-  const int sp = static_cast<int>(item % a.nsplit);
-  const long b = qrow / a.R;
-  const int* irow = a.idx + qrow * a.k;
-  const __nv_bfloat16* kvb = a.kv + b * static_cast<long>(a.Lkv) * a.ld_kv;
-  const int beg = sp * a.chunk;
-  int end = beg + a.chunk;
-  if (end > a.k) end = a.k;
-
-  // q rows of this query -> shared (async), trim trailing -1 entries of the list
-  const __nv_bfloat16* qg = a.q + qrow * (AT_H * AT_DK);
-  for (int c = tid; c < AT_H * AT_CHUNKS; c += AT_THREADS) {
-    const int h = c / AT_CHUNKS, ch = c % AT_CHUNKS;
-    cp_async16(smem_u32(&sm.q[h][ch * 16]), reinterpret_cast<const uint8_t*>(qg + h * AT_DK) + ch * 16);
-  }
-  if (tid == 0) sm.last_valid = beg - 1;
-  if (tid < AT_H) {
-    sm.m[tid] = -INFINITY;
-    sm.l[tid] = 0.f;
-  }
-  __syncthreads();
-  {
-    int lv = beg - 1;
-    for (int j = beg + tid; j < end; j += AT_THREADS)
-      if (__ldg(irow + j) >= 0) lv = j;
-    atomicMax(&sm.last_valid, lv);
-  }
-  __syncthreads();
-  end = sm.last_valid + 1;
-  const int ntiles = (end > beg) ? (end - beg + AT_BK - 1) / AT_BK : 0;
-
-  if (ntiles > 0) gather_tile(sm, a, irow, kvb, beg, end, 0);
-  cp_async_commit();  // group: q + tile 0
-  cp_async_wait<0>();
-  __syncthreads();
-
-  // this warp's slice of Q as A fragments: 18 k-steps of 16 dims
-  const int kh = warp >> 2, kg = warp & 3;
-  uint32_t qa[18][4];
-  {
-    const uint32_t qbase = smem_u32(&sm.q[0][0]);
-    const int r = (lane & 7) + 8 * ((lane >> 3) & 1);
-    const int cofs = 8 * (lane >> 4);
-#pragma unroll
-    for (int j = 0; j < 18; ++j) {
-      const int col = kh * 288 + 16 * j + cofs;
-      ldsm_x4(qbase + r * AT_ROWB + col * 2, qa[j][0], qa[j][1], qa[j][2], qa[j][3]);
-    }
-  }
-  float o[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-
+  volatile int* abort = &sm.abort;
+  const int kq = warp >> 1, kh = warp & 1;  // QK: dim quarter, key half of the tile
   const int g = lane >> 2, cq = lane & 3;
-  for (int t = 0; t < ntiles; ++t) {
-    const int buf = t & 1;
-    if (t + 1 < ntiles) gather_tile(sm, a, irow, kvb, beg + (t + 1) * AT_BK, end, buf ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-
-    // ---- S partial = Q[:, dims of kh] . K[keys 8kg..8kg+7]
+  int stage = 0, sb = 0;
+  uint32_t ph = 0;
+  int qwaits = 0;
+  for (long it = blockIdx.x; it < a.items; it += gridDim.x) {
+    const AttnItem x = attn_item(a, it);
+    if (!mbar_wait(smem_u32(&sm.qfull), qwaits & 1, abort, kErrTimeoutEpilogue)) return;
+    ++qwaits;
+    uint32_t qa[9][4];
     {
-      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t kvbase = smem_u32(&sm.kv[buf][0][0]);
-      const uint32_t rowaddr = kvbase + (8 * kg + (lane & 7)) * AT_ROWB;
+      const uint32_t qbase = smem_u32(&sm.q[0][0]);
+      const int r = (lane & 7) + 8 * ((lane >> 3) & 1);
+      const int cofs = 8 * (lane >> 4);
 #pragma unroll
-      for (int jj = 0; jj < 9; ++jj) {
-        uint32_t b0, b1, b2, b3;
-        const int col = kh * 288 + 32 * jj + 8 * (lane >> 3);
-        ldsm_x4(rowaddr + col * 2, b0, b1, b2, b3);
-        mma_bf16(sacc, qa[2 * jj], b0, b1);
-        mma_bf16(sacc, qa[2 * jj + 1], b2, b3);
-      }
-      sm.s_part[kh][g][8 * kg + 2 * cq] = sacc[0];
-      sm.s_part[kh][g][8 * kg + 2 * cq + 1] = sacc[1];
-      sm.s_part[kh][g + 8][8 * kg + 2 * cq] = sacc[2];
-      sm.s_part[kh][g + 8][8 * kg + 2 * cq + 1] = sacc[3];
-    }
-    __syncthreads();
-
-    // ---- online softmax: thread -> head tid/16, keys 2*(tid%16), +1
-    {
-      const int h = tid >> 4, c = (tid & 15) * 2;
-      const float2 p0 = *reinterpret_cast<const float2*>(&sm.s_part[0][h][c]);
-      const float2 p1 = *reinterpret_cast<const float2*>(&sm.s_part[1][h][c]);
-      float z0 = (p0.x + p1.x) * a.scale_log2;
-      float z1 = (p0.y + p1.y) * a.scale_log2;
-      if (sm.idx[buf][c] < 0) z0 = -INFINITY;
-      if (sm.idx[buf][c + 1] < 0) z1 = -INFINITY;
-      float tmax = fmaxf(z0, z1);
-#pragma unroll
-      for (int off = 8; off > 0; off >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
-      const float m_old = sm.m[h];
-      const float m_new = fmaxf(m_old, tmax);
-      float e0 = 0.f, e1 = 0.f, alpha = 1.f;
-      if (m_new != -INFINITY) {
-        e0 = exp2f(z0 - m_new);
-        e1 = exp2f(z1 - m_new);
-        alpha = exp2f(m_old - m_new);  // 0 when m_old = -inf
-      }
-      float rs = e0 + e1;
-#pragma unroll
-      for (int off = 8; off > 0; off >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
-      *reinterpret_cast<uint32_t*>(&sm.p[h][c * 2]) = pack_bf16(e0, e1);
-      __syncwarp();
-      if ((tid & 15) == 0) {
-        sm.l[h] = sm.l[h] * alpha + rs;
-        sm.m[h] = m_new;
-        sm.alpha[h] = alpha;
+      for (int j = 0; j < 9; ++j) {
+        const int col = kq * 144 + 16 * j + cofs;
+        ldsm_x4(qbase + r * AT_ROWB + col * 2, qa[j][0], qa[j][1], qa[j][2], qa[j][3]);
       }
     }
-    __syncthreads();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&sm.qempty));
+    float o[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads g, g + 8
 
-    // ---- O[:, 64w..64w+64) = alpha * O + P V
+    // prologue: the item's first tile through QK
+    if (!mbar_wait(smem_u32(&sm.full[stage]), ph, abort, kErrTimeoutEpilogue)) return;
+    int cur = stage, cur_sb = sb;
+    int cur_last = sm.last[stage];
+    unsigned cur_vm = sm.vmask[stage];
     {
-      const float al0 = sm.alpha[g], al1 = sm.alpha[g + 8];
+      float c[4][4];
+      attn_qk(smem_u32(&sm.kv[stage][0][0]), qa, kq, kh, lane, c);
+      attn_store_partial(&sm.s_part[sb][kq][0][0], c, kh, g, cq);
+    }
+    if (++stage == AT_STAGES) {
+      stage = 0;
+      ph ^= 1;
+    }
+    sb ^= 1;
+    named_bar_sync(1, AT_CONSUMERS);
+
+    for (;;) {
+      // softmax of the current tile (its partials are complete after the barrier)
+      uint32_t pa[2][4];
+      attn_softmax(&sm.s_part[cur_sb][0][0][0], cur_vm, a.scale_log2, g, cq, m0, m1, l0, l1, o,
+                   pa);
+      // QK of the next tile of this item overlaps the P V of the current one
+      const bool more = !cur_last;
+      float c[4][4];
+      int nxt_last = 1;
+      unsigned nxt_vm = 0u;
+      if (more) {
+        if (!mbar_wait(smem_u32(&sm.full[stage]), ph, abort, kErrTimeoutEpilogue)) return;
+        nxt_last = sm.last[stage];
+        nxt_vm = sm.vmask[stage];
+        attn_qk(smem_u32(&sm.kv[stage][0][0]), qa, kq, kh, lane, c);
+      }
+      attn_pv(smem_u32(&sm.kv[cur][0][0]), pa, warp, lane, o);
+      if (more) attn_store_partial(&sm.s_part[sb][kq][0][0], c, kh, g, cq);
+      named_bar_sync(1, AT_CONSUMERS);
+      // every warp is done with the current tile: its stage can be refilled
+      if (tid == 0) mbar_arrive(smem_u32(&sm.empty[cur]));
+      if (!more) break;
+      cur = stage;
+      cur_sb = sb;
+      cur_last = nxt_last;
+      cur_vm = nxt_vm;
+      if (++stage == AT_STAGES) {
+        stage = 0;
+        ph ^= 1;
+      }
+      sb ^= 1;
+    }
+
+    // ---- item epilogue: every thread holds m, l of its two heads
+    if (a.nsplit == 1) {
+      const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+      __nv_bfloat16* ob = a.out + x.qrow * (AT_H * AT_DV);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        o[i][0] *= al0;
-        o[i][1] *= al0;
-        o[i][2] *= al1;
-        o[i][3] *= al1;
+        const int d = 64 * warp + 8 * i + 2 * cq;
+        *reinterpret_cast<uint32_t*>(ob + g * AT_DV + d) = pack_bf16(o[i][0] * inv0, o[i][1] * inv0);
+        *reinterpret_cast<uint32_t*>(ob + (g + 8) * AT_DV + d) =
+            pack_bf16(o[i][2] * inv1, o[i][3] * inv1);
       }
-      const uint32_t pbase = smem_u32(&sm.p[0][0]);
-      const uint32_t kvbase = smem_u32(&sm.kv[buf][0][0]);
+      if (a.lse && warp == 0 && cq == 0) {
+        a.lse[x.qrow * AT_H + g] = l0 > 0.f ? (m0 + log2f(l0)) * 0.69314718055994531f : -INFINITY;
+        a.lse[x.qrow * AT_H + g + 8] =
+            l1 > 0.f ? (m1 + log2f(l1)) * 0.69314718055994531f : -INFINITY;
+      }
+    } else {
+      float* po = a.part_o + it * (AT_H * AT_DV);
 #pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        uint32_t pa[4];
-        const int pr = (lane & 7) + 8 * ((lane >> 3) & 1);
-        ldsm_x4(pbase + pr * AT_PROWB + (16 * ks + 8 * (lane >> 4)) * 2, pa[0], pa[1], pa[2], pa[3]);
-        const int vrow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t b0, b1, b2, b3;
-          const int col = 64 * warp + 16 * np + 8 * (lane >> 4);
-          ldsm_x4_t(kvbase + vrow * AT_ROWB + col * 2, b0, b1, b2, b3);
-          mma_bf16(o[2 * np], pa, b0, b1);
-          mma_bf16(o[2 * np + 1], pa, b2, b3);
-        }
+      for (int i = 0; i < 8; ++i) {
+        const int d = 64 * warp + 8 * i + 2 * cq;
+        *reinterpret_cast<float2*>(po + g * AT_DV + d) = make_float2(o[i][0], o[i][1]);
+        *reinterpret_cast<float2*>(po + (g + 8) * AT_DV + d) = make_float2(o[i][2], o[i][3]);
+      }
+      if (warp == 0 && cq == 0) {
+        a.part_ml[(it * AT_H + g) * 2] = m0;
+        a.part_ml[(it * AT_H + g) * 2 + 1] = l0;
+        a.part_ml[(it * AT_H + g + 8) * 2] = m1;
+        a.part_ml[(it * AT_H + g + 8) * 2 + 1] = l1;
       }
     }
-    __syncthreads();
   }
-  cp_async_wait<0>();
+}
 
-  // ---- epilogue
-  const float l0 = sm.l[g], l1 = sm.l[g + 8];
-  if (a.nsplit == 1) {
-    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
-    __nv_bfloat16* ob = a.out + qrow * (AT_H * AT_DV);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int d = 64 * warp + 8 * i + 2 * cq;
-      *reinterpret_cast<uint32_t*>(ob + g * AT_DV + d) = pack_bf16(o[i][0] * inv0, o[i][1] * inv0);
-      *reinterpret_cast<uint32_t*>(ob + (g + 8) * AT_DV + d) = pack_bf16(o[i][2] * inv1, o[i][3] * inv1);
+__global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const AttnArgs a) {
+  extern __shared__ uint8_t at_smem_raw[];
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(
+      (reinterpret_cast<uintptr_t>(at_smem_raw) + 127) & ~static_cast<uintptr_t>(127));
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < AT_STAGES; ++s) {
+      mbar_init(smem_u32(&sm.full[s]), 32);
+      mbar_init(smem_u32(&sm.empty[s]), 1);
     }
-    if (a.lse && tid < AT_H) {
-      const float l = sm.l[tid];
-      a.lse[qrow * AT_H + tid] = l > 0.f ? (sm.m[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-    }
-  } else {
-    float* po = a.part_o + item * (AT_H * AT_DV);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int d = 64 * warp + 8 * i + 2 * cq;
-      *reinterpret_cast<float2*>(po + g * AT_DV + d) = make_float2(o[i][0], o[i][1]);
-      *reinterpret_cast<float2*>(po + (g + 8) * AT_DV + d) = make_float2(o[i][2], o[i][3]);
-    }
-    if (tid < AT_H) {
-      a.part_ml[(item * AT_H + tid) * 2] = sm.m[tid];
-      a.part_ml[(item * AT_H + tid) * 2 + 1] = sm.l[tid];
-    }
+    mbar_init(smem_u32(&sm.qfull), 1);
+    mbar_init(smem_u32(&sm.qempty), AT_CONSUMERS / 32);
+    mbar_init(smem_u32(&sm.ifull[0]), 1);
+    mbar_init(smem_u32(&sm.ifull[1]), 1);
+    sm.abort = 0;
+    fence_barrier_init();
   }
+  // rows a tile never receives (index < 0) keep whatever the buffer held; start from
+  // zeros so that those stale rows are always finite (their softmax weight is 0)
+  uint4* z = reinterpret_cast<uint4*>(&sm.kv[0][0][0]);
+  for (int i = threadIdx.x; i < static_cast<int>(sizeof(sm.kv) / 16); i += blockDim.x)
+    z[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x >= AT_CONSUMERS)
+    attn_producer(sm, a);
+  else
+    attn_consumer(sm, a);
+  __syncthreads();
 }
 
 // Merges the nsplit partial results of one query: per head,
@@ -324,7 +563,7 @@ __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, i
 }
 
 static int pick_splits(long items, int k) {
-  const long want = 4L * num_sms();  // 2 resident CTAs per SM, two waves
+  const long want = 4L * num_sms();  // persistent CTAs: about four items per SM
   if (items >= want) return 1;
   long s = (want + items - 1) / items;
   long maxs = (k + 255) / 256;  // at least 256 entries per split
@@ -362,14 +601,17 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
   a.chunk = ((k + ns - 1) / ns + AT_BK - 1) / AT_BK * AT_BK;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse = lse;
+  a.items = items * ns;
+  a.idx_bulk = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
   a.part_o = static_cast<float*>(ws);
   a.part_ml = ns > 1 ? static_cast<float*>(ws) + items * ns * AT_H * AT_DV : nullptr;
-  const int smem = static_cast<int>(sizeof(AttnSmem));
+  const int smem = static_cast<int>(sizeof(AttnSmem)) + 128;
   ic_status st = cuda_check(
       cudaFuncSetAttribute(attn_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
       "cudaFuncSetAttribute(attn)");
   if (st) return st;
-  attn_mla_kernel<<<static_cast<unsigned>(items * ns), AT_THREADS, smem, stream>>>(a);
+  const long grid = a.items < num_sms() ? a.items : num_sms();
+  attn_mla_kernel<<<static_cast<unsigned>(grid), AT_THREADS, smem, stream>>>(a);
   st = cuda_check(cudaGetLastError(), "attn_mla_kernel launch");
   if (st) return st;
   // algorithmic bytes: each selected latent row gathered once, q read once, out written once

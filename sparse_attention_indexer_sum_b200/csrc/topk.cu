@@ -25,7 +25,10 @@ namespace ic {
 constexpr int TK_THREADS = 512;
 constexpr int TK_NW = TK_THREADS / 32;
 constexpr int TK_NBINS = 4096;  // 12-bit digits
-constexpr int TK_CAP = 4096;    // candidates kept in shared memory
+constexpr int TK_CAP = 6144;    // candidates kept in shared memory
+constexpr int TK_SAMPLE = 4096; // keys sampled to estimate the threshold
+constexpr int TK_EPT = 16;      // contiguous scores per thread per step of the ordered pass
+constexpr int TK_CHUNK = TK_THREADS * TK_EPT;
 constexpr int TK_MAXK = 2048;
 
 struct TopkSmem {
@@ -100,8 +103,27 @@ __device__ __forceinline__ void find_bin(TopkSmem& sm, int nbins, int need) {
   __syncthreads();
 }
 
+// Keys of scores [i0, i0 + 16) (0 past nv): four 128-bit loads when aligned and in range.
+__device__ __forceinline__ void load_keys16(const float* __restrict__ x, int nv, bool vec, int i0,
+                                            uint32_t (&k)[TK_EPT]) {
+  if (vec && i0 + TK_EPT - 1 < nv) {
+#pragma unroll
+    for (int v = 0; v < TK_EPT / 4; ++v) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(x + i0 + 4 * v));
+      k[4 * v + 0] = score_key(f.x);
+      k[4 * v + 1] = score_key(f.y);
+      k[4 * v + 2] = score_key(f.z);
+      k[4 * v + 3] = score_key(f.w);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < TK_EPT; ++e) k[e] = (i0 + e < nv) ? score_key(__ldg(x + i0 + e)) : 0u;
+  }
+}
+
 template <typename F>
 __device__ __forceinline__ void for_row(const float* x, int nv, bool vec, F&& f) {
+#pragma unroll 4
   for (int i0 = 4 * threadIdx.x; i0 < nv; i0 += 4 * TK_THREADS) {
     if (vec && i0 + 3 < nv) {
       const float4 v = __ldg(reinterpret_cast<const float4*>(x + i0));
@@ -115,23 +137,12 @@ __device__ __forceinline__ void for_row(const float* x, int nv, bool vec, F&& f)
   }
 }
 
-__global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restrict__ scores, long ld,
-                                                          int n, long pos0, int k,
-                                                          int* __restrict__ idx) {
-  extern __shared__ uint8_t tk_smem_raw[];
-  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
-  const long row = blockIdx.x;
-  long nvl = (pos0 < 0) ? n : pos0 + row + 1;
-  if (nvl > n) nvl = n;
-  const int nv = static_cast<int>(nvl);
-  int* out = idx + row * k;
-  if (nv <= k) {
-    for (int j = threadIdx.x; j < k; j += TK_THREADS) out[j] = (j < nv) ? j : -1;
-    return;
-  }
-  const float* x = scores + row * ld;
-  const bool vec = ((ld & 3) == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
-
+// Exact radix selection over the whole row: 12-bit histogram passes narrow the
+// bin of the k-th key (more passes only for heavily tied rows), one ordered pass
+// compacts the keys above it and its candidates, the candidates are resolved in
+// shared memory and the two ascending lists are merged into `out`.
+__device__ __noinline__ void topk_exact(TopkSmem& sm, const float* __restrict__ x, int nv,
+                                        bool vec, int k, int* __restrict__ out) {
   // ---------------------------------------------------------------- 1. radix passes
   uint32_t prefix = 0;
   int pbits = 0;
@@ -300,6 +311,142 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
       if (sm.gt_idx[mid] < v) lo = mid + 1; else hi = mid;
     }
     out[p + lo] = v;
+  }
+}
+
+// The k-th largest of `count` keys held in shared memory (count >= j >= 1),
+// by 12/12/8-bit histogram rounds over the keys.
+__device__ uint32_t select_kth_smem(TopkSmem& sm, const uint32_t* keys, int count, int j) {
+  uint32_t prefix = 0;
+  int pbits = 0;
+  int need = j;
+  while (pbits < 32) {
+    const int bits = (32 - pbits) >= 12 ? 12 : (32 - pbits);
+    const int shift = 32 - pbits - bits;
+    const int nb = 1 << bits;
+    const uint32_t mask = static_cast<uint32_t>(nb - 1);
+    for (int b = threadIdx.x; b < nb; b += TK_THREADS) sm.hist[b] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < count; i += TK_THREADS) {
+      const uint32_t key = keys[i];
+      if (pbits == 0 || (key >> (shift + bits)) == prefix)
+        atomicAdd(&sm.hist[(key >> shift) & mask], 1);
+    }
+    __syncthreads();
+    find_bin(sm, nb, need);
+    need -= sm.bcast[1];
+    prefix = (prefix << bits) | static_cast<uint32_t>(sm.bcast[0]);
+    pbits += bits;
+    __syncthreads();
+  }
+  return prefix;
+}
+
+__global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restrict__ scores, long ld,
+                                                          int n, long pos0, int k,
+                                                          int* __restrict__ idx) {
+  extern __shared__ uint8_t tk_smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
+  const long row = blockIdx.x;
+  long nvl = (pos0 < 0) ? n : pos0 + row + 1;
+  if (nvl > n) nvl = n;
+  const int nv = static_cast<int>(nvl);
+  int* out = idx + row * k;
+  if (nv <= k) {
+    for (int j = threadIdx.x; j < k; j += TK_THREADS) out[j] = (j < nv) ? j : -1;
+    return;
+  }
+  const float* x = scores + row * ld;
+  const bool vec = ((ld & 3) == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
+
+  // ---- 1. threshold estimate from a sample: the whole row when it is short,
+  //         else 32 evenly spread runs of 128 contiguous scores (2% of a 200K row)
+  uint32_t* samp = sm.cand_key;
+  int m, j;
+  if (nv <= TK_SAMPLE) {
+    m = nv;
+    for (int i = threadIdx.x; i < nv; i += TK_THREADS) samp[i] = score_key(__ldg(x + i));
+    j = k;  // exact k-th key: at least k keys are >= it
+  } else {
+    m = TK_SAMPLE;
+    const int run = TK_SAMPLE / 32;  // 128
+    for (int i = threadIdx.x; i < TK_SAMPLE; i += TK_THREADS) {
+      const int b = i / run, o = i % run;
+      const int start = static_cast<int>((static_cast<long>(b) * (nv - run)) / 31) & ~3;
+      samp[i] = score_key(__ldg(x + start + o));
+    }
+    // aim at ~1.6 k keys above the threshold: enough margin below k, and well under CAP
+    const long jj = (static_cast<long>(k) * 16 * m + 10L * nv - 1) / (10L * nv);
+    j = static_cast<int>(jj < 1 ? 1 : (jj > m ? m : jj));
+  }
+  __syncthreads();
+  const uint32_t tau = select_kth_smem(sm, samp, m, j);
+
+  // ---- 2. one ordered pass: every key >= tau, in index order, into the candidate list.
+  //         Each thread takes 16 contiguous scores per step and prefetches the next 16
+  //         before the block scan, so the loads stay in flight across the barriers.
+  int c_run = 0;
+  uint32_t cur[TK_EPT], nxt[TK_EPT];
+  load_keys16(x, nv, vec, TK_EPT * threadIdx.x, cur);
+  for (int c0 = 0; c0 < nv; c0 += TK_CHUNK) {
+    const int i0 = c0 + TK_EPT * threadIdx.x;
+    if (c0 + TK_CHUNK < nv) load_keys16(x, nv, vec, i0 + TK_CHUNK, nxt);
+    int nc = 0;
+#pragma unroll
+    for (int e = 0; e < TK_EPT; ++e) nc += (i0 + e < nv && cur[e] >= tau) ? 1 : 0;
+    int tot;
+    int cp = c_run + block_excl_scan(nc, sm.scan_tmp, &tot);
+    if (nc) {
+#pragma unroll
+      for (int e = 0; e < TK_EPT; ++e) {
+        if (i0 + e < nv && cur[e] >= tau) {
+          if (cp < TK_CAP) {
+            sm.cand_key[cp] = cur[e];
+            sm.cand_idx[cp] = i0 + e;
+          }
+          ++cp;
+        }
+      }
+    }
+    c_run += tot;
+#pragma unroll
+    for (int e = 0; e < TK_EPT; ++e) cur[e] = nxt[e];
+  }
+  __syncthreads();
+  const int C = c_run;
+  if (C < k || C > TK_CAP) {
+    // the sample misjudged the threshold (or the row is heavily tied): exact path
+    topk_exact(sm, x, nv, vec, k, out);
+    return;
+  }
+
+  // ---- 3. the k-th key T among the candidates; keys > T and the first ties == T win
+  const uint32_t T = select_kth_smem(sm, sm.cand_key, C, k);
+  int gt_total;
+  {
+    int local = 0;
+    for (int i = threadIdx.x; i < C; i += TK_THREADS) local += sm.cand_key[i] > T ? 1 : 0;
+    block_excl_scan(local, sm.scan_tmp, &gt_total);
+  }
+  const int take_eq = k - gt_total;
+  int gt_run = 0, eq_run = 0;
+  for (int c0 = 0; c0 < C; c0 += TK_THREADS) {
+    const int i = c0 + threadIdx.x;
+    int isgt = 0, iseq = 0;
+    if (i < C) {
+      const uint32_t key = sm.cand_key[i];
+      isgt = key > T;
+      iseq = key == T;
+    }
+    int tot;
+    const int ex = block_excl_scan(isgt | (iseq << 16), sm.scan_tmp, &tot);
+    const int gt_before = gt_run + (ex & 0xFFFF);
+    const int eq_rank = eq_run + (ex >> 16);
+    // output slot = rank among the selected, which keep index order
+    if (isgt || (iseq && eq_rank < take_eq))
+      out[gt_before + (eq_rank < take_eq ? eq_rank : take_eq)] = sm.cand_idx[i];
+    gt_run += tot & 0xFFFF;
+    eq_run += tot >> 16;
   }
 }
 

@@ -174,12 +174,13 @@ def _rand_idx(B, R, k, Lkv, seed, pad_from=None):
     return idx
 
 
-@pytest.mark.parametrize("B,R,k,Lkv", [(1, 37, 2048, 3000), (5, 1, 2048, 2500), (1, 9, 100, 150)])
+@pytest.mark.parametrize("B,R,k,Lkv", [(1, 37, 2048, 3000), (5, 1, 2048, 2500), (1, 9, 100, 150),
+                                       (2, 7, 37, 90)])
 def test_attn_mla_parity(B, R, k, Lkv):
     g = torch.Generator().manual_seed(B * 100 + R)
     q = torch.randn(B, R, 16, 576, generator=g).to(torch.bfloat16)
     kv = torch.randn(B, Lkv, 576, generator=g).to(torch.bfloat16)
-    pads = [k - (r * 37) % (k // 2) for r in range(R)]
+    pads = [k - (r * 37) % max(1, k // 2) for r in range(R)]
     idx = _rand_idx(B, R, k, Lkv, seed=R, pad_from=pads)
     idx[:, 0, 5] = -1                                   # a hole in the middle
     scale = 1 / math.sqrt(576)
