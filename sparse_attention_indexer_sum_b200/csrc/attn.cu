@@ -41,7 +41,8 @@ constexpr int AT_BK = 32;                   // keys per tile
 constexpr int AT_STAGES = 4;
 constexpr int AT_MAXK = 2048;               // longest index list of one item
 constexpr int AT_CONSUMERS = 256;           // 8 consumer warps
-constexpr int AT_THREADS = AT_CONSUMERS + 32;
+constexpr int AT_PRODUCERS = 4;             // producer warps; each issues 8 of a tile's 32 rows
+constexpr int AT_THREADS = AT_CONSUMERS + 32 * AT_PRODUCERS;
 constexpr int AT_ROWB = AT_DK * 2 + 16;     // padded shared row: 1168 B
 constexpr uint32_t AT_ROW_BYTES = AT_DK * 2;  // 1152 B gathered per row
 
@@ -58,6 +59,7 @@ struct AttnSmem {
   uint64_t empty[AT_STAGES];
   uint64_t qfull, qempty;
   uint64_t ifull[2];
+  uint64_t pitem;   // producers meet here at every item start
   int abort;
 };
 
@@ -146,8 +148,14 @@ __device__ __forceinline__ void attn_load_indices(AttnSmem& sm, const AttnArgs& 
   }
 }
 
+// Four producer warps walk the same items and tiles in lock step (they wait on the
+// same stage barriers); producer pw issues the bulk copies of rows 8pw..8pw+7 of
+// every tile -- one warp's bulk copies issue one lane at a time, so spreading a
+// tile over four warps quadruples the gather issue rate.  Producer 0 also owns
+// the per-item work: the next index list, the queries, the stage flags.
 __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
   const int lane = threadIdx.x & 31;
+  const int pw = (threadIdx.x - AT_CONSUMERS) >> 5;
   volatile int* abort = &sm.abort;
   const bool bulk = a.idx_bulk != 0;
   int stage = 0;
@@ -157,8 +165,10 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
   uint32_t iph[2] = {0u, 0u};
   int ipending[2] = {0, 0};
   const uint32_t kv0 = smem_u32(&sm.kv[0][0][0]);
+  const bool mine = (lane >> 3) == pw;  // this lane issues its row's copy
   int ib = 0;
-  if (blockIdx.x < a.items) {
+  long nitem = 0;
+  if (pw == 0 && blockIdx.x < a.items) {
     attn_load_indices(sm, a, blockIdx.x, 0, bulk);
     ipending[0] = bulk;
   }
@@ -167,6 +177,17 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
     const int cnt = x.end - x.beg;
     const long b = x.qrow / a.R;
     const __nv_bfloat16* kvb = a.kv + b * static_cast<long>(a.Lkv) * a.ld_kv;
+    // every producer is done with the previous item (and its index list)
+    if (lane == 0) mbar_arrive(smem_u32(&sm.pitem));
+    if (!mbar_wait(smem_u32(&sm.pitem), static_cast<uint32_t>(nitem & 1), abort, kErrTimeoutProducer))
+      break;
+    ++nitem;
+    // the next item's list streams in while this one's rows are gathered
+    const long nit = it + gridDim.x;
+    if (pw == 0 && nit < a.items) {
+      attn_load_indices(sm, a, nit, ib ^ 1, bulk);
+      ipending[ib ^ 1] = bulk;
+    }
     if (bulk) {
       if (!mbar_wait(smem_u32(&sm.ifull[ib]), iph[ib], abort, kErrTimeoutProducer)) break;
       iph[ib] ^= 1;
@@ -181,22 +202,18 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
     }
     lv = __reduce_max_sync(0xffffffffu, lv);
     const int ntiles = (lv >= 0) ? lv / AT_BK + 1 : 0;
-    // the next item's list streams in while this one's rows are gathered
-    const long nit = it + gridDim.x;
-    if (nit < a.items) {
-      attn_load_indices(sm, a, nit, ib ^ 1, bulk);
-      ipending[ib ^ 1] = bulk;
+    if (pw == 0) {
+      // the item's queries, once the consumers hold the previous ones in registers
+      if (qloads > 0 &&
+          !mbar_wait(smem_u32(&sm.qempty), (qloads - 1) & 1, abort, kErrTimeoutProducer))
+        break;
+      if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sm.qfull), AT_H * AT_ROW_BYTES);
+      __syncwarp();
+      if (lane < AT_H)
+        bulk_g2s(smem_u32(&sm.q[lane][0]), a.q + (x.qrow * AT_H + lane) * AT_DK, AT_ROW_BYTES,
+                 smem_u32(&sm.qfull));
+      ++qloads;
     }
-    // the item's queries, once the consumers hold the previous ones in registers
-    if (qloads > 0 &&
-        !mbar_wait(smem_u32(&sm.qempty), (qloads - 1) & 1, abort, kErrTimeoutProducer))
-      break;
-    if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sm.qfull), AT_H * AT_ROW_BYTES);
-    __syncwarp();
-    if (lane < AT_H)
-      bulk_g2s(smem_u32(&sm.q[lane][0]), a.q + (x.qrow * AT_H + lane) * AT_DK, AT_ROW_BYTES,
-               smem_u32(&sm.qfull));
-    ++qloads;
     const int nt = ntiles > 0 ? ntiles : 1;  // an empty item still ends with one (empty) tile
     bool ok = true;
     for (int t = 0; t < nt; ++t) {
@@ -208,16 +225,14 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
       int s = (t < ntiles && j < cnt) ? ilist[j] : -1;
       if (s >= a.Lkv) s = -1;
       const unsigned valid = __ballot_sync(0xffffffffu, s >= 0);
-      if (lane == 0) {
+      if (pw == 0 && lane == 0) {
         sm.vmask[stage] = valid;
         sm.last[stage] = (t == nt - 1);
       }
       const uint32_t fb = smem_u32(&sm.full[stage]);
-      if (lane == 0)
-        mbar_arrive_expect_tx(fb, __popc(valid) * AT_ROW_BYTES);
-      else
-        mbar_arrive(fb);
-      if (s >= 0)
+      if (lane == 0) mbar_arrive_expect_tx(fb, __popc(valid & (0xFFu << (8 * pw))) * AT_ROW_BYTES);
+      __syncwarp();
+      if (mine && s >= 0)
         bulk_g2s(kv0 + (stage * AT_BK + lane) * AT_ROWB, kvb + static_cast<long>(s) * a.ld_kv,
                  AT_ROW_BYTES, fb);
       ++issued;
@@ -507,13 +522,14 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const AttnArgs 
       (reinterpret_cast<uintptr_t>(at_smem_raw) + 127) & ~static_cast<uintptr_t>(127));
   if (threadIdx.x == 0) {
     for (int s = 0; s < AT_STAGES; ++s) {
-      mbar_init(smem_u32(&sm.full[s]), 32);
+      mbar_init(smem_u32(&sm.full[s]), AT_PRODUCERS);
       mbar_init(smem_u32(&sm.empty[s]), 1);
     }
     mbar_init(smem_u32(&sm.qfull), 1);
     mbar_init(smem_u32(&sm.qempty), AT_CONSUMERS / 32);
     mbar_init(smem_u32(&sm.ifull[0]), 1);
     mbar_init(smem_u32(&sm.ifull[1]), 1);
+    mbar_init(smem_u32(&sm.pitem), AT_PRODUCERS);
     sm.abort = 0;
     fence_barrier_init();
   }
