@@ -47,11 +47,15 @@ constexpr int AT_ROWB = AT_DK * 2 + 16;     // padded shared row: 1168 B
 constexpr uint32_t AT_ROW_BYTES = AT_DK * 2;  // 1152 B gathered per row
 
 constexpr int AT_SROW = 40;  // padded partial-score row (floats): conflict-free 64-bit access
+constexpr int AT_PROW = 40;  // padded P row (bf16, 80 B): conflict-free ldmatrix
 
 struct AttnSmem {
   alignas(128) uint8_t kv[AT_STAGES][AT_BK][AT_ROWB];  // 149504 B
   alignas(128) uint8_t q[AT_H][AT_ROWB];               // 18688 B
-  alignas(16) float s_part[2][4][AT_H][AT_SROW];       // double-buffered partial scores
+  alignas(16) float s_part[4][AT_H][AT_SROW];          // partial scores of the 4 dim quarters
+  alignas(16) __nv_bfloat16 p[AT_H][AT_PROW];           // softmax numerators of the tile
+  float alpha[AT_H];                                   // per-head rescale of the tile
+  float fin_m[AT_H], fin_l[AT_H];                      // per-head final max / sum of an item
   alignas(16) int ibuf[2][AT_MAXK];                    // index lists: this item / the next
   unsigned vmask[AT_STAGES];                           // bit j: row j of the stage is valid
   int last[AT_STAGES];
@@ -294,85 +298,9 @@ __device__ __forceinline__ void attn_store_partial(float* sp, const float (&c)[4
       make_float2(c[2][2] + c[3][2], c[2][3] + c[3][3]);
 }
 
-// Online softmax of heads g, g+8 over one tile's 32 keys from the four partials at
-// sp0, written as the two bf16 A fragments of P; rescales o and updates m, l.
-__device__ __forceinline__ void attn_softmax(const float* sp0, unsigned vm, float scale_log2,
-                                             int g, int cq, float& m0, float& m1, float& l0,
-                                             float& l1, float (&o)[8][4], uint32_t (&pa)[2][4]) {
-  constexpr int PSTRIDE = AT_H * AT_SROW;  // floats between the four dim-quarter partials
-  float z[2][2][4];                        // [ks][head g / g+8][key 2c, 2c+1, 2c+8, 2c+9]
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks) {
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int row = (g + 8 * hh) * AT_SROW + 16 * ks + 2 * cq;
-      float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        const float2 u = *reinterpret_cast<const float2*>(sp0 + qq * PSTRIDE + row);
-        const float2 v = *reinterpret_cast<const float2*>(sp0 + qq * PSTRIDE + row + 8);
-        lo.x += u.x;
-        lo.y += u.y;
-        hi.x += v.x;
-        hi.y += v.y;
-      }
-      z[ks][hh][0] = lo.x * scale_log2;
-      z[ks][hh][1] = lo.y * scale_log2;
-      z[ks][hh][2] = hi.x * scale_log2;
-      z[ks][hh][3] = hi.y * scale_log2;
-    }
-    const int k0 = 16 * ks + 2 * cq;
-    const bool v0 = (vm >> k0) & 1, v1 = (vm >> (k0 + 1)) & 1;
-    const bool v8 = (vm >> (k0 + 8)) & 1, v9 = (vm >> (k0 + 9)) & 1;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      if (!v0) z[ks][hh][0] = -INFINITY;
-      if (!v1) z[ks][hh][1] = -INFINITY;
-      if (!v8) z[ks][hh][2] = -INFINITY;
-      if (!v9) z[ks][hh][3] = -INFINITY;
-    }
-  }
-  float t0 = -INFINITY, t1 = -INFINITY;
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      t0 = fmaxf(t0, z[ks][0][e]);
-      t1 = fmaxf(t1, z[ks][1][e]);
-    }
-  t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, 1));
-  t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, 1));
-  t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, 2));
-  t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, 2));
-  const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
-  // a head with no valid key so far keeps weight 0 and scale 1
-  const float al0 = (n0 == -INFINITY) ? 1.f : fast_exp2(m0 - n0);
-  const float al1 = (n1 == -INFINITY) ? 1.f : fast_exp2(m1 - n1);
-  const float b0 = (n0 == -INFINITY) ? 0.f : n0, b1 = (n1 == -INFINITY) ? 0.f : n1;
-  float r0 = 0.f, r1 = 0.f;
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks) {
-    float e0[4], e1[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      e0[e] = fast_exp2(z[ks][0][e] - b0);  // exp2(-inf) = 0
-      e1[e] = fast_exp2(z[ks][1][e] - b1);
-      r0 += e0[e];
-      r1 += e1[e];
-    }
-    pa[ks][0] = pack_bf16(e0[0], e0[1]);
-    pa[ks][1] = pack_bf16(e1[0], e1[1]);
-    pa[ks][2] = pack_bf16(e0[2], e0[3]);
-    pa[ks][3] = pack_bf16(e1[2], e1[3]);
-  }
-  r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
-  r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
-  r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
-  r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
-  l0 = l0 * al0 + r0;
-  l1 = l1 * al1 + r1;
-  m0 = n0;
-  m1 = n1;
+// O[:, 64w..64w+64) = alpha O + P V for the tile at kvbase (P, alpha from shared).
+__device__ __forceinline__ void attn_pv(uint32_t kvbase, uint32_t pbase, float al0, float al1,
+                                        int warp, int lane, float (&o)[8][4]) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     o[i][0] *= al0;
@@ -380,36 +308,37 @@ __device__ __forceinline__ void attn_softmax(const float* sp0, unsigned vm, floa
     o[i][2] *= al1;
     o[i][3] *= al1;
   }
-}
-
-// O[:, 64w..64w+64) += P V for the tile at kvbase.
-__device__ __forceinline__ void attn_pv(uint32_t kvbase, const uint32_t (&pa)[2][4], int warp,
-                                        int lane, float (&o)[8][4]) {
 #pragma unroll
   for (int ks = 0; ks < 2; ++ks) {
+    uint32_t pa[4];
+    const int pr = (lane & 7) + 8 * ((lane >> 3) & 1);
+    ldsm_x4(pbase + (pr * AT_PROW + 16 * ks + 8 * (lane >> 4)) * 2, pa[0], pa[1], pa[2], pa[3]);
     const int vrow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
 #pragma unroll
     for (int np = 0; np < 4; ++np) {
       uint32_t b0, b1, b2, b3;
       const int col = 64 * warp + 16 * np + 8 * (lane >> 4);
       ldsm_x4_t(kvbase + vrow * AT_ROWB + col * 2, b0, b1, b2, b3);
-      mma_bf16(o[2 * np], pa[ks], b0, b1);
-      mma_bf16(o[2 * np + 1], pa[ks], b2, b3);
+      mma_bf16(o[2 * np], pa, b0, b1);
+      mma_bf16(o[2 * np + 1], pa, b2, b3);
     }
   }
 }
 
-// Software-pipelined per item: while tile t's softmax and P V run, the QK of tile
-// t+1 is already in flight; one barrier per tile publishes the partial scores and
-// retires tile t's stage.
+// Per tile: QK partials -> shared -> barrier -> the softmax of heads 2w, 2w+1, done
+// once by warp w (16 lanes per head, 2 keys per lane) -> P, alpha -> barrier ->
+// P V by every warp, with the QK of the next tile issued alongside it.
 __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort = &sm.abort;
   const int kq = warp >> 1, kh = warp & 1;  // QK: dim quarter, key half of the tile
   const int g = lane >> 2, cq = lane & 3;
-  int stage = 0, sb = 0;
+  const int sh = 2 * warp + (lane >> 4);    // softmax: head of this lane
+  const int sk = 2 * (lane & 15);           // and its two keys
+  int stage = 0;
   uint32_t ph = 0;
   int qwaits = 0;
+  int rel = -1;  // stage of the previous tile, released after the next partial barrier
   for (long it = blockIdx.x; it < a.items; it += gridDim.x) {
     const AttnItem x = attn_item(a, it);
     if (!mbar_wait(smem_u32(&sm.qfull), qwaits & 1, abort, kErrTimeoutEpilogue)) return;
@@ -430,61 +359,88 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
     float o[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads g, g + 8
+    float m_run = -INFINITY, l_run = 0.f;  // softmax state of head sh (its 16 lanes agree)
 
-    // prologue: the item's first tile through QK
     if (!mbar_wait(smem_u32(&sm.full[stage]), ph, abort, kErrTimeoutEpilogue)) return;
-    int cur = stage, cur_sb = sb;
+    int cur = stage;
     int cur_last = sm.last[stage];
     unsigned cur_vm = sm.vmask[stage];
     {
       float c[4][4];
       attn_qk(smem_u32(&sm.kv[stage][0][0]), qa, kq, kh, lane, c);
-      attn_store_partial(&sm.s_part[sb][kq][0][0], c, kh, g, cq);
+      attn_store_partial(&sm.s_part[kq][0][0], c, kh, g, cq);
     }
     if (++stage == AT_STAGES) {
       stage = 0;
       ph ^= 1;
     }
-    sb ^= 1;
-    named_bar_sync(1, AT_CONSUMERS);
-
     for (;;) {
-      // softmax of the current tile (its partials are complete after the barrier)
-      uint32_t pa[2][4];
-      attn_softmax(&sm.s_part[cur_sb][0][0][0], cur_vm, a.scale_log2, g, cq, m0, m1, l0, l1, o,
-                   pa);
-      // QK of the next tile of this item overlaps the P V of the current one
+      named_bar_sync(1, AT_CONSUMERS);  // B1: partials of cur complete, P V of prev done
+      if (tid == 0 && rel >= 0) mbar_arrive(smem_u32(&sm.empty[rel]));
+      // ---- softmax of head sh over keys sk, sk+1 (done once)
+      {
+        float2 z = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const float2 u = *reinterpret_cast<const float2*>(&sm.s_part[qq][sh][sk]);
+          z.x += u.x;
+          z.y += u.y;
+        }
+        const float z0 = ((cur_vm >> sk) & 1) ? z.x * a.scale_log2 : -INFINITY;
+        const float z1 = ((cur_vm >> (sk + 1)) & 1) ? z.y * a.scale_log2 : -INFINITY;
+        float t = fmaxf(z0, z1);
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, off));
+        const float n = fmaxf(m_run, t);
+        const float al = (n == -INFINITY) ? 1.f : fast_exp2(m_run - n);
+        const float bse = (n == -INFINITY) ? 0.f : n;
+        const float e0 = fast_exp2(z0 - bse), e1 = fast_exp2(z1 - bse);
+        float rs = e0 + e1;
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
+        l_run = l_run * al + rs;
+        m_run = n;
+        *reinterpret_cast<uint32_t*>(&sm.p[sh][sk]) = pack_bf16(e0, e1);
+        if ((lane & 15) == 0) sm.alpha[sh] = al;
+      }
+      named_bar_sync(1, AT_CONSUMERS);  // B2: P, alpha complete
+      // ---- the next tile's QK goes out alongside this tile's P V
       const bool more = !cur_last;
       float c[4][4];
-      int nxt_last = 1;
+      int nxt = -1, nxt_last = 1;
       unsigned nxt_vm = 0u;
       if (more) {
         if (!mbar_wait(smem_u32(&sm.full[stage]), ph, abort, kErrTimeoutEpilogue)) return;
+        nxt = stage;
         nxt_last = sm.last[stage];
         nxt_vm = sm.vmask[stage];
         attn_qk(smem_u32(&sm.kv[stage][0][0]), qa, kq, kh, lane, c);
+        if (++stage == AT_STAGES) {
+          stage = 0;
+          ph ^= 1;
+        }
       }
-      attn_pv(smem_u32(&sm.kv[cur][0][0]), pa, warp, lane, o);
-      if (more) attn_store_partial(&sm.s_part[sb][kq][0][0], c, kh, g, cq);
-      named_bar_sync(1, AT_CONSUMERS);
-      // every warp is done with the current tile: its stage can be refilled
-      if (tid == 0) mbar_arrive(smem_u32(&sm.empty[cur]));
+      attn_pv(smem_u32(&sm.kv[cur][0][0]), smem_u32(&sm.p[0][0]), sm.alpha[g], sm.alpha[g + 8],
+              warp, lane, o);
+      rel = cur;
       if (!more) break;
-      cur = stage;
-      cur_sb = sb;
+      attn_store_partial(&sm.s_part[kq][0][0], c, kh, g, cq);
+      cur = nxt;
       cur_last = nxt_last;
       cur_vm = nxt_vm;
-      if (++stage == AT_STAGES) {
-        stage = 0;
-        ph ^= 1;
-      }
-      sb ^= 1;
     }
 
-    // ---- item epilogue: every thread holds m, l of its two heads
+    // ---- item epilogue: head h's final max and sum live in warp h/2
+    named_bar_sync(1, AT_CONSUMERS);  // every warp's P V of the item is done
+    if ((lane & 15) == 0) {
+      sm.fin_m[sh] = m_run;
+      sm.fin_l[sh] = l_run;
+    }
+    named_bar_sync(1, AT_CONSUMERS);
+    const float M0 = sm.fin_m[g], M1 = sm.fin_m[g + 8];
+    const float L0 = sm.fin_l[g], L1 = sm.fin_l[g + 8];
     if (a.nsplit == 1) {
-      const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+      const float inv0 = L0 > 0.f ? 1.f / L0 : 0.f, inv1 = L1 > 0.f ? 1.f / L1 : 0.f;
       __nv_bfloat16* ob = a.out + x.qrow * (AT_H * AT_DV);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -494,9 +450,9 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
             pack_bf16(o[i][2] * inv1, o[i][3] * inv1);
       }
       if (a.lse && warp == 0 && cq == 0) {
-        a.lse[x.qrow * AT_H + g] = l0 > 0.f ? (m0 + log2f(l0)) * 0.69314718055994531f : -INFINITY;
+        a.lse[x.qrow * AT_H + g] = L0 > 0.f ? (M0 + log2f(L0)) * 0.69314718055994531f : -INFINITY;
         a.lse[x.qrow * AT_H + g + 8] =
-            l1 > 0.f ? (m1 + log2f(l1)) * 0.69314718055994531f : -INFINITY;
+            L1 > 0.f ? (M1 + log2f(L1)) * 0.69314718055994531f : -INFINITY;
       }
     } else {
       float* po = a.part_o + it * (AT_H * AT_DV);
@@ -507,10 +463,10 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
         *reinterpret_cast<float2*>(po + (g + 8) * AT_DV + d) = make_float2(o[i][2], o[i][3]);
       }
       if (warp == 0 && cq == 0) {
-        a.part_ml[(it * AT_H + g) * 2] = m0;
-        a.part_ml[(it * AT_H + g) * 2 + 1] = l0;
-        a.part_ml[(it * AT_H + g + 8) * 2] = m1;
-        a.part_ml[(it * AT_H + g + 8) * 2 + 1] = l1;
+        a.part_ml[(it * AT_H + g) * 2] = M0;
+        a.part_ml[(it * AT_H + g) * 2 + 1] = L0;
+        a.part_ml[(it * AT_H + g + 8) * 2] = M1;
+        a.part_ml[(it * AT_H + g + 8) * 2 + 1] = L1;
       }
     }
   }
