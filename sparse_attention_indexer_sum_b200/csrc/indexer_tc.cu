@@ -329,21 +329,23 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
           tmem_ld32(taddr, v0);
           tmem_ld32(taddr + 32, v1);
           tmem_ld_wait();
-          const float* wt = wsl + tk * 64;
+          const float4* wt = reinterpret_cast<const float4*>(wsl + tk * 64);
           float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-          for (int h = 0; h < 32; h += 4) {
-            s0 = fmaf(wt[h + 0], fmaxf(v0[h + 0], 0.f), s0);
-            s1 = fmaf(wt[h + 1], fmaxf(v0[h + 1], 0.f), s1);
-            s2 = fmaf(wt[h + 2], fmaxf(v0[h + 2], 0.f), s2);
-            s3 = fmaf(wt[h + 3], fmaxf(v0[h + 3], 0.f), s3);
+          for (int h4 = 0; h4 < 8; ++h4) {
+            const float4 wv = wt[h4];  // same address in every lane: one broadcast
+            s0 = fmaf(wv.x, fmaxf(v0[4 * h4 + 0], 0.f), s0);
+            s1 = fmaf(wv.y, fmaxf(v0[4 * h4 + 1], 0.f), s1);
+            s2 = fmaf(wv.z, fmaxf(v0[4 * h4 + 2], 0.f), s2);
+            s3 = fmaf(wv.w, fmaxf(v0[4 * h4 + 3], 0.f), s3);
           }
 #pragma unroll
-          for (int h = 0; h < 32; h += 4) {
-            s0 = fmaf(wt[32 + h + 0], fmaxf(v1[h + 0], 0.f), s0);
-            s1 = fmaf(wt[32 + h + 1], fmaxf(v1[h + 1], 0.f), s1);
-            s2 = fmaf(wt[32 + h + 2], fmaxf(v1[h + 2], 0.f), s2);
-            s3 = fmaf(wt[32 + h + 3], fmaxf(v1[h + 3], 0.f), s3);
+          for (int h4 = 0; h4 < 8; ++h4) {
+            const float4 wv = wt[8 + h4];
+            s0 = fmaf(wv.x, fmaxf(v1[4 * h4 + 0], 0.f), s0);
+            s1 = fmaf(wv.y, fmaxf(v1[4 * h4 + 1], 0.f), s1);
+            s2 = fmaf(wv.z, fmaxf(v1[4 * h4 + 2], 0.f), s2);
+            s3 = fmaf(wv.w, fmaxf(v1[4 * h4 + 3], 0.f), s3);
           }
           res[tk] = (s0 + s1) + (s2 + s3);
         }
@@ -424,8 +426,8 @@ long long causal_pairs(long R, long Lk, long pos0) {
   long long n = 0;
   const long r_full = Lk - pos0 - 1;  // rows from here on see all Lk keys
   const long r_tri = r_full < 0 ? 0 : (r_full < R ? r_full : R);
-  n += static_cast<long long>(r_tri) * (pos0 + 1) + static_cast<long long>(r_tri) * (r_tri - 1) / 2 +
-       r_tri;  // sum_{r < r_tri} (pos0 + r + 1)
+  n += static_cast<long long>(r_tri) * (pos0 + 1) +
+       static_cast<long long>(r_tri) * (r_tri - 1) / 2;  // sum_{r < r_tri} (pos0 + r + 1)
   n += static_cast<long long>(R - r_tri) * Lk;
   return n;
 }

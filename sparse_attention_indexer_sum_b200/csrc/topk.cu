@@ -3,8 +3,13 @@
 // k = 2048 in its intro).  Ties go to the lower index, -0 == +0, output in
 // ascending index order padded with -1.
 //
-// One CTA (512 threads) per row.  Scores are mapped to order-preserving
-// 32-bit keys and the k-th largest key is found by radix selection:
+// One CTA (512 threads) per row.  Scores are mapped to order-preserving 32-bit
+// keys.  Common path: a threshold estimated from a 2% sample, one streaming pass
+// that collects every key above it (unordered, warp-aggregated shared atomics),
+// the exact k-th key among those candidates by radix selection, ties at it broken
+// toward the lower index, and the selection written in ascending order from a
+// shared-memory bitmap.  When the sample misjudges (or the row is heavily tied
+// or very long), the exact path below runs instead:
 //   1. histogram of the top 12 key bits over the row (shared-memory atomics,
 //      128-bit loads); the bin holding the k-th largest is located with one
 //      block scan.  If that bin holds more than CAP keys (heavily tied data),
@@ -31,14 +36,23 @@ constexpr int TK_EPT = 16;      // contiguous scores per thread per step of the 
 constexpr int TK_CHUNK = TK_THREADS * TK_EPT;
 constexpr int TK_MAXK = 2048;
 
+constexpr int TK_BM_WORDS = 8192;  // selection bitmap: rows of up to 262144 scores
+constexpr int TK_MAXTIE = 512;     // ties at the k-th key resolved in shared memory
+
 struct TopkSmem {
   int hist[TK_NBINS];
-  int gt_idx[TK_MAXK];
   uint32_t cand_key[TK_CAP];
   int cand_idx[TK_CAP];
-  int sel_idx[TK_MAXK];
+  union {
+    struct {
+      int gt_idx[TK_MAXK];
+      int sel_idx[TK_MAXK];
+    } ex;                            // exact path
+    uint32_t bitmap[TK_BM_WORDS];    // fast path: selected indices
+  } u;
   int scan_tmp[TK_NW];
   int bcast[4];
+  int counter, ties;
 };
 
 // Order-preserving key: a > b as floats  <=>  key(a) > key(b) as unsigned; -0 -> +0.
@@ -216,7 +230,7 @@ __device__ __noinline__ void topk_exact(TopkSmem& sm, const float* __restrict__ 
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if (cls[e] == 2) {
-        if (gp < TK_MAXK) sm.gt_idx[gp] = i0 + e;
+        if (gp < TK_MAXK) sm.u.ex.gt_idx[gp] = i0 + e;
         ++gp;
       } else if (cls[e] == 1) {
         const int lim = (pbits == 32) ? k_rem : TK_CAP;
@@ -243,7 +257,7 @@ __device__ __noinline__ void topk_exact(TopkSmem& sm, const float* __restrict__ 
   int S;
   if (pbits == 32) {
     // every candidate carries the same key: the first k_rem in index order win
-    for (int j = threadIdx.x; j < k_rem; j += TK_THREADS) sm.sel_idx[j] = sm.cand_idx[j];
+    for (int j = threadIdx.x; j < k_rem; j += TK_THREADS) sm.u.ex.sel_idx[j] = sm.cand_idx[j];
     S = k_rem;
   } else {
     const int C = c_run;  // <= TK_CAP here
@@ -285,7 +299,7 @@ __device__ __noinline__ void topk_exact(TopkSmem& sm, const float* __restrict__ 
       const int gt_before = gt_run + (ex & 0xFFFF);
       const int eq_rank = eq_run + (ex >> 16);
       const int pos = gt_before + (eq_rank < take_eq ? eq_rank : take_eq);
-      if (isgt || (iseq && eq_rank < take_eq)) sm.sel_idx[pos] = sm.cand_idx[j];
+      if (isgt || (iseq && eq_rank < take_eq)) sm.u.ex.sel_idx[pos] = sm.cand_idx[j];
       gt_run += tot & 0xFFFF;
       eq_run += tot >> 16;
     }
@@ -295,32 +309,35 @@ __device__ __noinline__ void topk_exact(TopkSmem& sm, const float* __restrict__ 
 
   // ---------------------------------------------------------------- merge two ascending lists
   for (int p = threadIdx.x; p < G; p += TK_THREADS) {
-    const int v = sm.gt_idx[p];
+    const int v = sm.u.ex.gt_idx[p];
     int lo = 0, hi = S;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (sm.sel_idx[mid] < v) lo = mid + 1; else hi = mid;
+      if (sm.u.ex.sel_idx[mid] < v) lo = mid + 1; else hi = mid;
     }
     out[p + lo] = v;
   }
   for (int p = threadIdx.x; p < S; p += TK_THREADS) {
-    const int v = sm.sel_idx[p];
+    const int v = sm.u.ex.sel_idx[p];
     int lo = 0, hi = G;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (sm.gt_idx[mid] < v) lo = mid + 1; else hi = mid;
+      if (sm.u.ex.gt_idx[mid] < v) lo = mid + 1; else hi = mid;
     }
     out[p + lo] = v;
   }
 }
 
-// The k-th largest of `count` keys held in shared memory (count >= j >= 1),
-// by 12/12/8-bit histogram rounds over the keys.
-__device__ uint32_t select_kth_smem(TopkSmem& sm, const uint32_t* keys, int count, int j) {
+// The j-th largest of `count` keys held in shared memory (count >= j >= 1), by
+// 12/12/8-bit histogram rounds over the keys.  With bits = 24 it stops after two
+// rounds and returns the lowest key of the j-th key's 24-bit bin (a lower bound:
+// at least j keys are >= it).
+__device__ uint32_t select_kth_smem(TopkSmem& sm, const uint32_t* keys, int count, int j,
+                                    int bits_total = 32) {
   uint32_t prefix = 0;
   int pbits = 0;
   int need = j;
-  while (pbits < 32) {
+  while (pbits < bits_total) {
     const int bits = (32 - pbits) >= 12 ? 12 : (32 - pbits);
     const int shift = 32 - pbits - bits;
     const int nb = 1 << bits;
@@ -339,7 +356,11 @@ __device__ uint32_t select_kth_smem(TopkSmem& sm, const uint32_t* keys, int coun
     pbits += bits;
     __syncthreads();
   }
-  return prefix;
+  return pbits >= 32 ? prefix : (prefix << (32 - pbits));
+}
+
+__device__ __forceinline__ void mark_selected(TopkSmem& sm, int i) {
+  atomicOr(&sm.u.bitmap[i >> 5], 1u << (i & 31));
 }
 
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restrict__ scores, long ld,
@@ -347,106 +368,160 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
                                                           int* __restrict__ idx) {
   extern __shared__ uint8_t tk_smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31;
   const long row = blockIdx.x;
   long nvl = (pos0 < 0) ? n : pos0 + row + 1;
   if (nvl > n) nvl = n;
   const int nv = static_cast<int>(nvl);
   int* out = idx + row * k;
   if (nv <= k) {
-    for (int j = threadIdx.x; j < k; j += TK_THREADS) out[j] = (j < nv) ? j : -1;
+    for (int j = tid; j < k; j += TK_THREADS) out[j] = (j < nv) ? j : -1;
     return;
   }
   const float* x = scores + row * ld;
   const bool vec = ((ld & 3) == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
+  if (nv > TK_BM_WORDS * 32) {  // longer than the selection bitmap: exact multi-pass path
+    topk_exact(sm, x, nv, vec, k, out);
+    return;
+  }
+  const int nwords = (nv + 31) >> 5;
+  for (int w = tid; w < nwords; w += TK_THREADS) sm.u.bitmap[w] = 0u;
+  if (tid == 0) {
+    sm.counter = 0;
+    sm.ties = 0;
+  }
 
-  // ---- 1. threshold estimate from a sample: the whole row when it is short,
-  //         else 32 evenly spread runs of 128 contiguous scores (2% of a 200K row)
+  // ---- 1. threshold from a sample: the whole row when it is short, else 32 evenly
+  //         spread runs of 128 contiguous scores (2% of a 200K row).  tau is a lower
+  //         bound of the sample's j-th key, aimed at ~1.6 k keys >= tau in the row.
   uint32_t* samp = sm.cand_key;
   int m, j;
   if (nv <= TK_SAMPLE) {
     m = nv;
-    for (int i = threadIdx.x; i < nv; i += TK_THREADS) samp[i] = score_key(__ldg(x + i));
-    j = k;  // exact k-th key: at least k keys are >= it
+    for (int i = tid; i < nv; i += TK_THREADS) samp[i] = score_key(__ldg(x + i));
+    j = k;  // at least k keys are >= the k-th key
   } else {
     m = TK_SAMPLE;
     const int run = TK_SAMPLE / 32;  // 128
-    for (int i = threadIdx.x; i < TK_SAMPLE; i += TK_THREADS) {
+    for (int i = tid; i < TK_SAMPLE; i += TK_THREADS) {
       const int b = i / run, o = i % run;
       const int start = static_cast<int>((static_cast<long>(b) * (nv - run)) / 31) & ~3;
       samp[i] = score_key(__ldg(x + start + o));
     }
-    // aim at ~1.6 k keys above the threshold: enough margin below k, and well under CAP
     const long jj = (static_cast<long>(k) * 16 * m + 10L * nv - 1) / (10L * nv);
     j = static_cast<int>(jj < 1 ? 1 : (jj > m ? m : jj));
   }
   __syncthreads();
-  const uint32_t tau = select_kth_smem(sm, samp, m, j);
+  const uint32_t tau = select_kth_smem(sm, samp, m, j, 24);
 
-  // ---- 2. one ordered pass: every key >= tau, in index order, into the candidate list.
-  //         Each thread takes 16 contiguous scores per step and prefetches the next 16
-  //         before the block scan, so the loads stay in flight across the barriers.
-  int c_run = 0;
-  uint32_t cur[TK_EPT], nxt[TK_EPT];
-  load_keys16(x, nv, vec, TK_EPT * threadIdx.x, cur);
-  for (int c0 = 0; c0 < nv; c0 += TK_CHUNK) {
-    const int i0 = c0 + TK_EPT * threadIdx.x;
-    if (c0 + TK_CHUNK < nv) load_keys16(x, nv, vec, i0 + TK_CHUNK, nxt);
-    int nc = 0;
+  // ---- 2. one streaming pass: every key >= tau into the candidate list (unordered;
+  //         one shared atomic per warp and step, no block barriers)
+  {
+    uint32_t cur[TK_EPT], nxt[TK_EPT];
+    load_keys16(x, nv, vec, TK_EPT * tid, cur);
+    for (int c0 = 0; c0 < nv; c0 += TK_CHUNK) {
+      const int i0 = c0 + TK_EPT * tid;
+      if (c0 + TK_CHUNK < nv) load_keys16(x, nv, vec, i0 + TK_CHUNK, nxt);
+      int hits = 0;
 #pragma unroll
-    for (int e = 0; e < TK_EPT; ++e) nc += (i0 + e < nv && cur[e] >= tau) ? 1 : 0;
-    int tot;
-    int cp = c_run + block_excl_scan(nc, sm.scan_tmp, &tot);
-    if (nc) {
+      for (int e = 0; e < TK_EPT; ++e) hits += (i0 + e < nv && cur[e] >= tau) ? 1 : 0;
+      int incl = hits;
 #pragma unroll
-      for (int e = 0; e < TK_EPT; ++e) {
-        if (i0 + e < nv && cur[e] >= tau) {
-          if (cp < TK_CAP) {
-            sm.cand_key[cp] = cur[e];
-            sm.cand_idx[cp] = i0 + e;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+      if (wtot) {
+        int base = 0;
+        if (lane == 31) base = atomicAdd(&sm.counter, wtot);
+        base = __shfl_sync(0xffffffffu, base, 31);
+        int pos = base + incl - hits;
+        if (hits) {
+#pragma unroll
+          for (int e = 0; e < TK_EPT; ++e) {
+            if (i0 + e < nv && cur[e] >= tau) {
+              if (pos < TK_CAP) {
+                sm.cand_key[pos] = cur[e];
+                sm.cand_idx[pos] = i0 + e;
+              }
+              ++pos;
+            }
           }
-          ++cp;
         }
       }
-    }
-    c_run += tot;
 #pragma unroll
-    for (int e = 0; e < TK_EPT; ++e) cur[e] = nxt[e];
+      for (int e = 0; e < TK_EPT; ++e) cur[e] = nxt[e];
+    }
   }
   __syncthreads();
-  const int C = c_run;
+  const int C = sm.counter;
   if (C < k || C > TK_CAP) {
     // the sample misjudged the threshold (or the row is heavily tied): exact path
     topk_exact(sm, x, nv, vec, k, out);
     return;
   }
 
-  // ---- 3. the k-th key T among the candidates; keys > T and the first ties == T win
+  // ---- 3. the exact k-th key T among the candidates
   const uint32_t T = select_kth_smem(sm, sm.cand_key, C, k);
-  int gt_total;
+  int gt_total, eq_total;
   {
-    int local = 0;
-    for (int i = threadIdx.x; i < C; i += TK_THREADS) local += sm.cand_key[i] > T ? 1 : 0;
-    block_excl_scan(local, sm.scan_tmp, &gt_total);
-  }
-  const int take_eq = k - gt_total;
-  int gt_run = 0, eq_run = 0;
-  for (int c0 = 0; c0 < C; c0 += TK_THREADS) {
-    const int i = c0 + threadIdx.x;
-    int isgt = 0, iseq = 0;
-    if (i < C) {
+    int lg = 0, le = 0;
+    for (int i = tid; i < C; i += TK_THREADS) {
       const uint32_t key = sm.cand_key[i];
-      isgt = key > T;
-      iseq = key == T;
+      lg += key > T ? 1 : 0;
+      le += key == T ? 1 : 0;
     }
     int tot;
-    const int ex = block_excl_scan(isgt | (iseq << 16), sm.scan_tmp, &tot);
-    const int gt_before = gt_run + (ex & 0xFFFF);
-    const int eq_rank = eq_run + (ex >> 16);
-    // output slot = rank among the selected, which keep index order
-    if (isgt || (iseq && eq_rank < take_eq))
-      out[gt_before + (eq_rank < take_eq ? eq_rank : take_eq)] = sm.cand_idx[i];
-    gt_run += tot & 0xFFFF;
-    eq_run += tot >> 16;
+    block_excl_scan(lg | (le << 16), sm.scan_tmp, &tot);
+    gt_total = tot & 0xFFFF;
+    eq_total = tot >> 16;
+  }
+  const int take_eq = k - gt_total;  // >= 1
+  if (eq_total > take_eq && eq_total > TK_MAXTIE) {
+    topk_exact(sm, x, nv, vec, k, out);  // many ties at the k-th key: exact path
+    return;
+  }
+
+  // ---- 4. mark the selection: keys > T, and the take_eq lowest indices among ties
+  const bool all_ties = (eq_total == take_eq);
+  for (int i = tid; i < C; i += TK_THREADS) {
+    const uint32_t key = sm.cand_key[i];
+    if (key > T || (all_ties && key == T)) {
+      mark_selected(sm, sm.cand_idx[i]);
+    } else if (key == T) {
+      sm.hist[atomicAdd(&sm.ties, 1)] = sm.cand_idx[i];
+    }
+  }
+  __syncthreads();
+  if (!all_ties) {
+    const int nt = sm.ties;
+    for (int a = tid; a < nt; a += TK_THREADS) {
+      const int v = sm.hist[a];
+      int rank = 0;
+      for (int b = 0; b < nt; ++b) rank += sm.hist[b] < v ? 1 : 0;
+      if (rank < take_eq) mark_selected(sm, v);
+    }
+    __syncthreads();
+  }
+
+  // ---- 5. ascending output: contiguous bitmap words per thread, one block scan
+  {
+    const int wpt = (nwords + TK_THREADS - 1) / TK_THREADS;
+    const int w0 = tid * wpt;
+    const int w1 = min(nwords, w0 + wpt);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(sm.u.bitmap[w]);
+    int tot;
+    int pos = block_excl_scan(cnt, sm.scan_tmp, &tot);
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = sm.u.bitmap[w];
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        out[pos++] = (w << 5) + b;
+        bits &= bits - 1;
+      }
+    }
   }
 }
 

@@ -327,3 +327,18 @@ def test_decode_step_parity():
         ro, _ = oracle.sparse_attn(h["q"].float().numpy(), h["kv"].float().numpy(), T[:, None, :],
                                    wl.scale, dv=512)
         assert_attn_close(_np(dl[l]["out"]), ro)
+
+
+def test_trace_records_every_launch_in_order():
+    q, k, w = _idx_inputs(1, 8, 300, seed=3)
+    q, k, w = q.to(DEV), k.to(DEV), w.to(DEV)
+    ic.ic_indexer_scores(q, k, w, pos0=100)      # warm up (attributes, tensor maps)
+    _sync()
+    ic.ic_trace_begin(16)
+    s = ic.ic_indexer_scores(q, k, w, pos0=100)
+    ic.ic_topk(s[0], 64, pos0=100)
+    n, tr = ic.ic_trace_end(16)
+    assert n == 3
+    assert [t[0] for t in tr] == ["indexer_tc_bf16", "fill_masked", "topk"]
+    assert all(ms > 0 for _, ms, _ in tr)
+    assert tr[0][2] == 2.0 * 64 * 128 * sum(min(300, 100 + r + 1) for r in range(8))
