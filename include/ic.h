@@ -164,6 +164,40 @@ ic_status ic_sparse_attn(const void* q, const void* kv, long ld_kv, const void* 
 size_t ic_attn_workspace_size(int batch, int rows, int heads, int dv, int k);
 
 /*
+ * ic_sparse_attn_noalloc: the absorbed-MLA form of ic_sparse_attn for callers
+ * that cannot allocate device memory -- for example a plugin whose host
+ * framework hands it only its input and output buffers and offers no workspace
+ * hook, or a process whose memory pool has claimed the whole device up front.
+ * The paper has no counterpart; it is a convenience of this library.
+ *
+ * Same arguments, layouts and results as ic_sparse_attn with v = NULL and a
+ * workspace of ic_attn_workspace_size bytes (the same split of the index list
+ * is chosen), minus the workspace.  The split partials go to a fixed array of
+ * IC_NOALLOC_SCRATCH_BYTES (16.06 MiB) inside this library, which every GPU
+ * that loads the library holds until the process exits.  Neither this call
+ * nor anything it calls allocates or frees device memory.
+ *
+ *   batch * rows <= IC_NOALLOC_MAX_QUERIES (64), else IC_ERR_UNSUPPORTED;
+ *   v != NULL (the MQA form, which needs no scratch) -> IC_ERR_UNSUPPORTED;
+ *   other checks and errors as ic_sparse_attn.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress with that device current) and caches it; make that
+ * first call before any stream capture.  All calls share the one array: calls
+ * that overlap on the GPU (other streams, other host threads) race on it and
+ * must be serialised by the caller, e.g. by using a single stream.  Each call
+ * overwrites every partial it later reads, so leftovers from an earlier call
+ * do not matter.  Runs on the calling thread's current device, which must own
+ * `stream`.
+ */
+#define IC_NOALLOC_MAX_QUERIES 64
+#define IC_NOALLOC_SCRATCH_BYTES (64u * 8u * 16u * 514u * 4u)
+ic_status ic_sparse_attn_noalloc(const void* q, const void* kv, long ld_kv, const void* v,
+                                 const int* idx, ic_dtype dt, int batch, int rows, int heads,
+                                 int dk, int dv, int Lkv, int k, float scale, void* out,
+                                 float* lse, void* stream);
+
+/*
  * Per-layer inputs of the layer stack.  Every pointer is device memory.
  * F layers need the indexer fields; S layers ignore them (they may be NULL).
  */

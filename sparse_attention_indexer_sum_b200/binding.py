@@ -28,7 +28,8 @@ IC_F32, IC_BF16, IC_E4M3 = 0, 1, 2
 EXPORTS = ("ic_last_error", "ic_version", "ic_device_status", "ic_trace_begin", "ic_trace_end",
            "ic_quant_e4m3_rows",
            "ic_indexer_scores", "ic_topk", "ic_sparse_attn", "ic_attn_workspace_size",
-           "ic_layer_stack", "ic_decode_step", "ic_stack_workspace_size")
+           "ic_layer_stack", "ic_decode_step", "ic_stack_workspace_size",
+           "ic_sparse_attn_noalloc")
 
 
 class ICError(RuntimeError):
@@ -84,8 +85,9 @@ def lib() -> ctypes.CDLL:
     L.ic_decode_step.argtypes = L.ic_layer_stack.argtypes
     L.ic_stack_workspace_size.argtypes = [ctypes.POINTER(ic_stack_desc)]
     L.ic_stack_workspace_size.restype = S
+    L.ic_sparse_attn_noalloc.argtypes = [P, P, Lg, P, P, I, I, I, I, I, I, I, I, F, P, P, P]
     for name in ("ic_device_status", "ic_quant_e4m3_rows", "ic_indexer_scores", "ic_topk",
-                 "ic_sparse_attn", "ic_layer_stack", "ic_decode_step"):
+                 "ic_sparse_attn", "ic_layer_stack", "ic_decode_step", "ic_sparse_attn_noalloc"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -236,6 +238,27 @@ def ic_sparse_attn(q, kv, idx, scale: float, *, v=None, dv: int | None = None, o
     _check(lib().ic_sparse_attn(_p(q), _p(kv), kv.stride(-2), _p(v), _p(idx), dtype_code(q), B, R,
                                 heads, dk, dv, Lkv, kk, float(scale), _p(out), _p(lse),
                                 _p(workspace), ws_bytes, _stream(stream)))
+    return out
+
+
+def ic_sparse_attn_noalloc(q, kv, idx, scale: float, *, dv: int = 512, out=None, lse=None,
+                           stream=None):
+    """Absorbed-MLA sparse attention whose split scratch is the library's fixed device
+    array rather than a workspace (for callers that cannot allocate; at most
+    IC_NOALLOC_MAX_QUERIES = 64 queries).  q [B?,R,16,576] bf16; kv [B?,Lkv,ld_kv];
+    idx [B?,R,k].  Calls that overlap on the GPU race on the shared array."""
+    _contig(q, idx)
+    if kv.stride(-1) != 1:
+        raise ValueError("kv rows must be contiguous")
+    squeeze = q.dim() == 3
+    B = 1 if squeeze else q.shape[0]
+    R, heads, dk = q.shape[-3:]
+    if out is None:
+        out = torch.empty(q.shape[:-1] + (dv,), dtype=q.dtype, device=q.device)
+    _check(lib().ic_sparse_attn_noalloc(_p(q), _p(kv), kv.stride(-2), None, _p(idx),
+                                        dtype_code(q), B, R, heads, dk, dv, kv.shape[-2],
+                                        idx.shape[-1], float(scale), _p(out), _p(lse),
+                                        _stream(stream)))
     return out
 
 

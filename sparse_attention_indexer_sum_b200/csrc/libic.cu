@@ -5,3 +5,4 @@
 #include "attn.cu"
 #include "misc.cu"
 #include "api.cu"
+#include "noalloc.cu"
