@@ -69,6 +69,8 @@ struct IdxCfg {
   static constexpr int NEPI = 4 * EPG;
   static constexpr int TOK_PER_EW = TPM / EPG;     // tokens per epilogue warp
   static constexpr int THREADS = 64 + 32 * NEPI;
+  // TMEM columns an epilogue thread loads at a time (fewer registers with more warps)
+  static constexpr int EPI_COLS = (NEPI > 8) ? 16 : 32;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_Q = STAGES * A_BYTES;
   static constexpr int OFF_W = OFF_Q + Q_BYTES;
@@ -300,6 +302,11 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
       int acc = 0;
       uint32_t aph = 0;
       int cur_qb = -1;
+      // head weights of this warp's first token, kept in registers while the
+      // query block lasts (any further tokens read theirs from shared memory)
+      float wr[64];
+#pragma unroll
+      for (int h = 0; h < 64; ++h) wr[h] = 0.f;
       for (long i = 0; i < nitems; ++i) {
         const int b = it.qb / a.qb_per_batch, ql = it.qb % a.qb_per_batch;
         const int r0 = ql * TPM + member * C::TOK_PER_EW;
@@ -316,6 +323,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
             wsl[x] = v;
           }
           __syncwarp();
+#pragma unroll
+          for (int h = 0; h < 64; ++h) wr[h] = wsl[h];
           cur_qb = it.qb;
         }
         if (!mbar_wait(accfull_bar(acc), aph, abort_flag, kErrTimeoutEpilogue)) break;
@@ -325,27 +334,27 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
         for (int tk = 0; tk < C::TOK_PER_EW; ++tk) {
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
                                  static_cast<uint32_t>(acc * C::N + (member * C::TOK_PER_EW + tk) * 64);
-          float v0[32], v1[32];
-          tmem_ld32(taddr, v0);
-          tmem_ld32(taddr + 32, v1);
-          tmem_ld_wait();
           const float4* wt = reinterpret_cast<const float4*>(wsl + tk * 64);
           float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-          for (int h4 = 0; h4 < 8; ++h4) {
-            const float4 wv = wt[h4];  // same address in every lane: one broadcast
-            s0 = fmaf(wv.x, fmaxf(v0[4 * h4 + 0], 0.f), s0);
-            s1 = fmaf(wv.y, fmaxf(v0[4 * h4 + 1], 0.f), s1);
-            s2 = fmaf(wv.z, fmaxf(v0[4 * h4 + 2], 0.f), s2);
-            s3 = fmaf(wv.w, fmaxf(v0[4 * h4 + 3], 0.f), s3);
-          }
+          for (int part = 0; part < 64 / C::EPI_COLS; ++part) {  // heads in chunks of EPI_COLS
+            float v[C::EPI_COLS];
+            if constexpr (C::EPI_COLS == 32)
+              tmem_ld32(taddr + 32 * part, *reinterpret_cast<float(*)[32]>(v));
+            else
+              tmem_ld16(taddr + 16 * part, *reinterpret_cast<float(*)[16]>(v));
+            tmem_ld_wait();
 #pragma unroll
-          for (int h4 = 0; h4 < 8; ++h4) {
-            const float4 wv = wt[8 + h4];
-            s0 = fmaf(wv.x, fmaxf(v1[4 * h4 + 0], 0.f), s0);
-            s1 = fmaf(wv.y, fmaxf(v1[4 * h4 + 1], 0.f), s1);
-            s2 = fmaf(wv.z, fmaxf(v1[4 * h4 + 2], 0.f), s2);
-            s3 = fmaf(wv.w, fmaxf(v1[4 * h4 + 3], 0.f), s3);
+            for (int h4 = 0; h4 < C::EPI_COLS / 4; ++h4) {
+              const int h = C::EPI_COLS * part + 4 * h4;
+              // same address in every lane: one broadcast
+              const float4 wv = (tk == 0) ? make_float4(wr[h], wr[h + 1], wr[h + 2], wr[h + 3])
+                                          : wt[h / 4];
+              s0 = fmaf(wv.x, fmaxf(v[4 * h4 + 0], 0.f), s0);
+              s1 = fmaf(wv.y, fmaxf(v[4 * h4 + 1], 0.f), s1);
+              s2 = fmaf(wv.z, fmaxf(v[4 * h4 + 2], 0.f), s2);
+              s3 = fmaf(wv.w, fmaxf(v[4 * h4 + 3], 0.f), s3);
+            }
           }
           res[tk] = (s0 + s1) + (s2 + s3);
         }
