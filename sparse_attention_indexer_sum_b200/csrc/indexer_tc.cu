@@ -69,8 +69,9 @@ struct IdxCfg {
   static constexpr int NEPI = 4 * EPG;
   static constexpr int TOK_PER_EW = TPM / EPG;     // tokens per epilogue warp
   static constexpr int THREADS = 64 + 32 * NEPI;
-  // TMEM columns an epilogue thread loads at a time (fewer registers with more warps)
-  static constexpr int EPI_COLS = (NEPI > 8) ? 16 : 32;
+  // TMEM columns an epilogue thread loads at a time: 16, so that the head
+  // weights of both its tokens fit in registers beside them
+  static constexpr int EPI_COLS = 16;  // matches tmem_ld16
   static constexpr int OFF_A = 0;
   static constexpr int OFF_Q = STAGES * A_BYTES;
   static constexpr int OFF_W = OFF_Q + Q_BYTES;
@@ -302,11 +303,13 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
       int acc = 0;
       uint32_t aph = 0;
       int cur_qb = -1;
-      // head weights of this warp's first token, kept in registers while the
-      // query block lasts (any further tokens read theirs from shared memory)
-      float wr[64];
+      // head weights of this warp's tokens, kept in registers while the query
+      // block lasts (the values are then read from TMEM 16 columns at a time)
+      float wr[C::TOK_PER_EW][64];
 #pragma unroll
-      for (int h = 0; h < 64; ++h) wr[h] = 0.f;
+      for (int t = 0; t < C::TOK_PER_EW; ++t)
+#pragma unroll
+        for (int h = 0; h < 64; ++h) wr[t][h] = 0.f;
       for (long i = 0; i < nitems; ++i) {
         const int b = it.qb / a.qb_per_batch, ql = it.qb % a.qb_per_batch;
         const int r0 = ql * TPM + member * C::TOK_PER_EW;
@@ -324,9 +327,17 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
           }
           __syncwarp();
 #pragma unroll
-          for (int h = 0; h < 64; ++h) wr[h] = wsl[h];
+          for (int t = 0; t < C::TOK_PER_EW; ++t)
+#pragma unroll
+            for (int h = 0; h < 64; ++h) wr[t][h] = wsl[t * 64 + h];
           cur_qb = it.qb;
         }
+        // this lane's key; its fp8 scale is fetched before the wait so the load's
+        // latency hides behind it
+        const int s = it.kt * C::BM + qd * 32 + lane;
+        const bool key_ok = s < a.Lk && b < a.B;
+        float ks = 1.f;
+        if constexpr (FP8) ks = key_ok ? a.k_scale[static_cast<long>(b) * a.Lk + s] : 0.f;
         if (!mbar_wait(accfull_bar(acc), aph, abort_flag, kErrTimeoutEpilogue)) break;
         tc_fence_after();
         float res[C::TOK_PER_EW];
@@ -334,22 +345,16 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
         for (int tk = 0; tk < C::TOK_PER_EW; ++tk) {
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
                                  static_cast<uint32_t>(acc * C::N + (member * C::TOK_PER_EW + tk) * 64);
-          const float4* wt = reinterpret_cast<const float4*>(wsl + tk * 64);
           float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
           for (int part = 0; part < 64 / C::EPI_COLS; ++part) {  // heads in chunks of EPI_COLS
             float v[C::EPI_COLS];
-            if constexpr (C::EPI_COLS == 32)
-              tmem_ld32(taddr + 32 * part, *reinterpret_cast<float(*)[32]>(v));
-            else
-              tmem_ld16(taddr + 16 * part, *reinterpret_cast<float(*)[16]>(v));
+            tmem_ld16(taddr + C::EPI_COLS * part, v);
             tmem_ld_wait();
 #pragma unroll
             for (int h4 = 0; h4 < C::EPI_COLS / 4; ++h4) {
               const int h = C::EPI_COLS * part + 4 * h4;
-              // same address in every lane: one broadcast
-              const float4 wv = (tk == 0) ? make_float4(wr[h], wr[h + 1], wr[h + 2], wr[h + 3])
-                                          : wt[h / 4];
+              const float4 wv = make_float4(wr[tk][h], wr[tk][h + 1], wr[tk][h + 2], wr[tk][h + 3]);
               s0 = fmaf(wv.x, fmaxf(v[4 * h4 + 0], 0.f), s0);
               s1 = fmaf(wv.y, fmaxf(v[4 * h4 + 1], 0.f), s1);
               s2 = fmaf(wv.z, fmaxf(v[4 * h4 + 2], 0.f), s2);
@@ -361,10 +366,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(accempty_bar(acc));
-        const int s = it.kt * C::BM + qd * 32 + lane;
-        if (s < a.Lk && b < a.B) {
-          float ks = 1.f;
-          if constexpr (FP8) ks = a.k_scale[static_cast<long>(b) * a.Lk + s];
+        if (key_ok) {
 #pragma unroll
           for (int tk = 0; tk < C::TOK_PER_EW; ++tk) {
             const int r = r0 + tk;
