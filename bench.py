@@ -15,7 +15,12 @@ Rank 0 prints one JSON line.  Besides the contract keys it carries:
   all_f         the same stack with every layer F, and the F,S,S,S speed-up;
   e2e           the metric through the C ABI with host buffers (H2D of the
                 step's inputs and D2H of its result inside the timed region);
-  cpu_baseline  the fp64 CPU oracle on a bounded sample of rows, extrapolated.
+  cpu_baseline  the fp64 CPU oracle on a bounded sample of rows, extrapolated;
+  decode        64 sequences x 1 new token over a 200000-token context (e4m3
+                indexer key cache, bf16 latent KV cache), F,S,S,S and all-F,
+                against the measured HBM bandwidth;
+  stack_32k     the 8-layer F,S,S,S,F,S,S,S stack at L=32768 against all-F,
+                with the overlap of adjacent layers' index sets under all-F.
 
 ``--impl reference`` times the CPU oracle (the reference of this repository)
 on the same workload, metric and unit instead.
@@ -273,6 +278,171 @@ def run_ours(args, rank, world, local_rank):
                              max_over_ranks, world)
     if args.cpu_baseline and rank == 0 and world == 1:
         res["cpu_baseline"] = cpu_baseline(wl, layers, budget_s=args.cpu_budget)
+    if world == 1 and (args.decode or args.stack32k):
+        del layers, ws, t_cache
+        torch.cuda.empty_cache()
+        if args.decode:
+            res["decode"] = run_decode(args, dev, peaks, barrier)
+            torch.cuda.empty_cache()
+        if args.stack32k:
+            res["stack_32k"] = run_stack32k(args, dev, barrier)
+            torch.cuda.empty_cache()
+    return res
+
+
+def _timed(fn, steps, stream):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def run_decode(args, dev, peaks, barrier):
+    """Config 5: one decode step of 64 sequences (one new token each at position
+    199999) through ic_decode_step, F,S,S,S and all-F.  HBM-bound: the roofline is
+    the algorithmic bytes of the step (fp8 key cache + scales read by the indexer,
+    the scores written and read back by the top-k, the gathered latent rows, q and
+    out of every layer) over the measured copy bandwidth."""
+    from sparse_attention_indexer_sum_b200 import binding as ic
+    wl = synth.WORKLOADS["decode_200k"]
+    B, L, k = wl.batch, wl.L, wl.k
+    layers = []
+    for l in range(wl.layers):
+        d = synth.indexer_inputs(wl, l, device=dev)
+        d["q_idx"], d["q_scale"] = ic.ic_quant_e4m3_rows(d["q_idx"])
+        kb = d.pop("k_idx")
+        d["k_idx"], d["k_scale"] = ic.ic_quant_e4m3_rows(kb)
+        del kb
+        d.update(synth.attn_inputs(wl, l, device=dev))
+        d["out"] = torch.empty(B, 1, wl.Hq, wl.Dv, dtype=torch.bfloat16, device=dev)
+        d["lse"] = torch.empty(B, 1, wl.Hq, dtype=torch.float32, device=dev)
+        layers.append(d)
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+    desc = ic.make_desc(L=L, k=k, H=wl.H, D=wl.D, idx_dtype=ic.IC_E4M3, heads=wl.Hq, dk=wl.Dk,
+                        dv=wl.Dv, attn_dtype=ic.IC_BF16, scale=wl.scale, batch=B, decode=True)
+    ws = torch.empty(ic.ic_stack_workspace_size(desc) // 4 + 1, dtype=torch.float32, device=dev)
+    t_cache = torch.empty(B, k, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    allf = ",".join("F" * wl.layers)
+    steps = 50
+
+    def step(pat):
+        ic.ic_decode_step(pat, desc, layers, t_cache, ws, stream=stream)
+
+    kk = min(k, L)
+    idx_b = B * L * (wl.D + 4)                      # e4m3 key cache + per-token scales
+    score_b = B * L * 4 * 2 + B * kk * 4            # scores out and back in, T out
+    attn_b = B * kk * wl.Dk * 2 + B * wl.Hq * (wl.Dk + wl.Dv) * 2 + B * kk * 4
+
+    def bytes_of(pat):
+        f = sum(1 for c in pat if c == "F")
+        return f * (idx_b + score_b) + wl.layers * attn_b
+
+    out = {"workload": wl.name, "batch": B, "context": L, "k": k, "pattern": wl.pattern,
+           "indexer": "e4m3 key cache + per-token f32 scales", "kv_cache": "bf16 576-d latent",
+           "l2": "inputs larger than L2 (no flush needed)"}
+    for pat, key in ((wl.pattern, None), (allf, "all_f")):
+        for _ in range(max(3, args.warmup)):
+            step(pat)
+        ic.ic_device_status(stream)
+        barrier()
+        cap = 64 * steps
+        ic.ic_trace_begin(cap, stream=stream)
+        ms = _timed(lambda: step(pat), steps, stream)
+        n_launch, trace = ic.ic_trace_end(cap)
+        ic.ic_device_status(stream)
+        hb = bytes_of(pat)
+        gbs = hb / (ms * 1e-3) / 1e9
+        r = {"pattern": pat, "ms_per_step": ms, "value": B / (ms * 1e-3), "unit": "tokens/s",
+             "hbm_bytes_per_step": hb, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+             "frac_hbm": gbs / peaks["hbm_gbs"], "gpu_launches_per_step": n_launch / steps}
+        if key is None:
+            agg = {}
+            for name, kms, work in trace:
+                a = agg.setdefault(name, [0, 0.0, 0.0])
+                a[0] += 1
+                a[1] += kms
+                a[2] += work
+            st = {}
+            for name, (n, kms, work) in sorted(agg.items()):
+                if name.startswith("indexer"):
+                    byt = (idx_b + B * L * 4) * n        # cache read + scores written
+                elif name == "topk":
+                    byt = (B * L * 4 + B * kk * 4) * n
+                else:
+                    byt = work
+                g = byt / (kms * 1e-3) / 1e9
+                st[name] = {"launches_per_step": n / steps, "ms_per_step": kms / steps,
+                            "achieved_gbs": g, "frac_hbm": g / peaks["hbm_gbs"]}
+            r["stages"] = st
+            out.update(r)
+        else:
+            out[key] = r
+    out["speedup_fsss_over_all_f"] = out["all_f"]["ms_per_step"] / out["ms_per_step"]
+    log("decode: %.3f ms/step (%.0f tokens/s), %.0f GB/s = %.2f of HBM; all-F %.3f ms" % (
+        out["ms_per_step"], out["value"], out["achieved_gbs"], out["frac_hbm"],
+        out["all_f"]["ms_per_step"]))
+    return out
+
+
+def _overlap(Ta, Tb):
+    """Mean over rows of |Ta & Tb| / |Ta| for ascending, -1 padded index rows."""
+    big = torch.iinfo(torch.int32).max
+    A = torch.where(Ta < 0, torch.full_like(Ta, big), Ta).contiguous()
+    Bq = torch.where(Tb < 0, torch.full_like(Tb, big), Tb).contiguous()
+    pos = torch.searchsorted(A, Bq).clamp_(max=A.shape[1] - 1)
+    hit = (A.gather(1, pos) == Tb) & (Tb >= 0)
+    n = (Ta >= 0).sum(1).clamp_(min=1)
+    return hit.sum(1).double() / n.double()
+
+
+def run_stack32k(args, dev, barrier):
+    """Config 3: the 8-layer F,S,S,S,F,S,S,S stack at L=32768 against all-F, and the
+    overlap of adjacent layers' index sets when every layer runs its own indexer."""
+    from sparse_attention_indexer_sum_b200 import binding as ic
+    wl = synth.WORKLOADS["stack_32k"]
+    allf = ",".join("F" * wl.layers)
+    layers = make_inputs(wl, dev, [kinds_of(allf)], False, seed=0)
+    desc = ic.make_desc(L=wl.L, k=wl.k, H=wl.H, D=wl.D, idx_dtype=ic.IC_BF16, heads=wl.Hq,
+                        dk=wl.Dk, dv=wl.Dv, attn_dtype=ic.IC_BF16, scale=wl.scale)
+    ws = torch.empty(ic.ic_stack_workspace_size(desc) // 4 + 1, dtype=torch.float32, device=dev)
+    t_cache = torch.empty(wl.L, wl.k, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    steps = 5
+    res = {"workload": wl.name, "L": wl.L, "layers": wl.layers, "k": wl.k,
+           "pattern": wl.pattern}
+    for pat, key in ((wl.pattern, "ms_per_step"), (allf, "all_f_ms_per_step")):
+        for _ in range(max(3, args.warmup)):
+            ic.ic_layer_stack(pat, desc, layers, t_cache, ws, stream=stream)
+        barrier()
+        res[key] = _timed(lambda: ic.ic_layer_stack(pat, desc, layers, t_cache, ws,
+                                                    stream=stream), steps, stream)
+    res["value"] = wl.L / (res["ms_per_step"] * 1e-3)
+    res["all_f_value"] = wl.L / (res["all_f_ms_per_step"] * 1e-3)
+    res["speedup_fs_over_all_f"] = res["all_f_ms_per_step"] / res["ms_per_step"]
+    # every layer F, one at a time, keeping each layer's T
+    prev, ov = None, []
+    rows_ge_k = torch.arange(wl.L, device=dev) >= wl.k - 1
+    for l in range(wl.layers):
+        ic.ic_layer_stack("F", desc, [layers[l]], t_cache, ws, stream=stream)
+        cur = t_cache.clone()
+        if prev is not None:
+            o = _overlap(prev, cur)
+            ov.append((float(o.mean()), float(o[rows_ge_k].mean())))
+        prev = cur
+    ic.ic_device_status(stream)
+    res["overlap_adjacent_all_f"] = {
+        "mean_all_rows": sum(a for a, _ in ov) / len(ov),
+        "mean_rows_with_more_than_k_candidates": sum(b for _, b in ov) / len(ov),
+        "per_pair": [round(b, 4) for _, b in ov],
+        "definition": "|T_l & T_(l+1)| / |T_l| averaged over query rows, every layer F"}
+    log("stack_32k: %.2f ms (F/S) vs %.2f ms (all-F), speed-up %.2fx, adjacent overlap %.3f" % (
+        res["ms_per_step"], res["all_f_ms_per_step"], res["speedup_fs_over_all_f"],
+        res["overlap_adjacent_all_f"]["mean_rows_with_more_than_k_candidates"]))
     return res
 
 
@@ -449,6 +619,10 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-decode", dest="decode", action="store_false",
+                    help="skip the decode (64 x 1 token at 200K context) measurement")
+    ap.add_argument("--no-stack32k", dest="stack32k", action="store_false",
+                    help="skip the 8-layer L=32768 stack and its layer-overlap report")
     args = ap.parse_args()
     if args.warmup < 3:
         log("note: fewer than 3 warm-up steps requested")
