@@ -63,10 +63,15 @@ struct IdxCfg {
   static constexpr int A_BYTES = BM * ROWB;        // one key tile
   static constexpr int Q_BYTES = N * ROWB;         // the query block
   static constexpr int STAGES = FP8 ? 8 : 4;
-  static constexpr int NACC = (TPM == 4) ? 2 : 4;  // TMEM accumulators in the ring
+  static constexpr int NACC = (TPM == 4) ? 2 : 6;  // TMEM accumulators in the ring
   static constexpr int TMEM_COLS = (NACC * N <= 256) ? 256 : 512;
   static constexpr int EPG = (TPM == 4) ? 2 : 1;   // epilogue warps per TMEM lane quadrant
-  static constexpr int NEPI = 4 * EPG;
+  // Epilogue warp sets: set j takes the accumulator slots a with a % NSETS == j, so
+  // each set sees every use of its slots in order.  One-token blocks (decode) have
+  // little epilogue work per tile; several sets overlap consecutive tiles.
+  static constexpr int NSETS = (TPM == 4) ? 1 : 3;
+  static constexpr int SETW = 4 * EPG;             // warps per set
+  static constexpr int NEPI = SETW * NSETS;
   static constexpr int TOK_PER_EW = TPM / EPG;     // tokens per epilogue warp
   static constexpr int THREADS = 64 + 32 * NEPI;
   // TMEM columns an epilogue thread loads at a time: 16, so that the head
@@ -84,6 +89,7 @@ struct IdxCfg {
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(NACC * N <= TMEM_COLS, "TMEM");
+  static_assert(NACC % NSETS == 0, "each epilogue set owns whole accumulator slots");
 };
 
 template <int TPM>
@@ -152,7 +158,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
       }
       for (int i = 0; i < C::NACC; ++i) {
         mbar_init(accfull_bar(i), 1);
-        mbar_init(accempty_bar(i), C::NEPI);
+        mbar_init(accempty_bar(i), C::SETW);
       }
       mbar_init(qfull_bar, 1);
       mbar_init(qempty_bar, 1);
@@ -297,7 +303,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
       // ------------------------------------------------------------ epilogue
       const int e = warp - 2;
       const int qd = warp & 3;     // TMEM lane quadrant this warp may access
-      const int member = e / 4;    // which tokens of the block this warp reduces
+      const int set = e / C::SETW;  // accumulator slots a with a % NSETS == set
+      const int member = (e % C::SETW) / 4;  // which tokens of the block this warp reduces
       float* wsl = w_smem + e * C::TOK_PER_EW * 64;
       WorkIt<TPM> it{start[0], start[1], qb_tiles<TPM>(a, start[0])};
       int acc = 0;
@@ -311,6 +318,14 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
 #pragma unroll
         for (int h = 0; h < 64; ++h) wr[t][h] = 0.f;
       for (long i = 0; i < nitems; ++i) {
+        if (C::NSETS > 1 && acc % C::NSETS != set) {  // another set's slot
+          if (++acc == C::NACC) {
+            acc = 0;
+            aph ^= 1;
+          }
+          it.advance(a);
+          continue;
+        }
         const int b = it.qb / a.qb_per_batch, ql = it.qb % a.qb_per_batch;
         const int r0 = ql * TPM + member * C::TOK_PER_EW;
         if (it.qb != cur_qb) {
