@@ -363,25 +363,76 @@ __device__ __forceinline__ void mark_selected(TopkSmem& sm, int i) {
   atomicOr(&sm.u.bitmap[i >> 5], 1u << (i & 31));
 }
 
+// Every key >= tau among scores [lo, hi) into the candidate list, unordered (one
+// shared atomic per warp and step, no block barriers); the count goes to
+// sm.counter, which may exceed TK_CAP (entries past it are dropped).  lo is a
+// multiple of TK_EPT.
+__device__ __forceinline__ void collect_candidates(TopkSmem& sm, const float* __restrict__ x,
+                                                   int lo, int hi, bool vec, uint32_t tau) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  {
+    uint32_t cur[TK_EPT], nxt[TK_EPT];
+    load_keys16(x, hi, vec, lo + TK_EPT * tid, cur);
+    for (int c0 = lo; c0 < hi; c0 += TK_CHUNK) {
+      const int i0 = c0 + TK_EPT * tid;
+      if (c0 + TK_CHUNK < hi) load_keys16(x, hi, vec, i0 + TK_CHUNK, nxt);
+      int hits = 0;
+#pragma unroll
+      for (int e = 0; e < TK_EPT; ++e) hits += (i0 + e < hi && cur[e] >= tau) ? 1 : 0;
+      int incl = hits;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+      if (wtot) {
+        int base = 0;
+        if (lane == 31) base = atomicAdd(&sm.counter, wtot);
+        base = __shfl_sync(0xffffffffu, base, 31);
+        int pos = base + incl - hits;
+        if (hits) {
+#pragma unroll
+          for (int e = 0; e < TK_EPT; ++e) {
+            if (i0 + e < hi && cur[e] >= tau) {
+              if (pos < TK_CAP) {
+                sm.cand_key[pos] = cur[e];
+                sm.cand_idx[pos] = i0 + e;
+              }
+              ++pos;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < TK_EPT; ++e) cur[e] = nxt[e];
+    }
+  }
+}
+
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restrict__ scores, long ld,
                                                           int n, long pos0, int k,
                                                           int* __restrict__ idx) {
   extern __shared__ uint8_t tk_smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
-  const int tid = threadIdx.x, lane = tid & 31;
-  const long row = blockIdx.x;
+  const int tid = threadIdx.x;
+  // A row is split over the S CTAs of a cluster (S = 1 without clusters): each
+  // collects the candidates of its part, CTA 0 merges them and selects.
+  const uint32_t S = cluster_nctarank(), crank = cluster_ctarank();
+  const long row = blockIdx.x / S;
   long nvl = (pos0 < 0) ? n : pos0 + row + 1;
   if (nvl > n) nvl = n;
   const int nv = static_cast<int>(nvl);
   int* out = idx + row * k;
   if (nv <= k) {
-    for (int j = tid; j < k; j += TK_THREADS) out[j] = (j < nv) ? j : -1;
+    if (crank == 0)
+      for (int j = tid; j < k; j += TK_THREADS) out[j] = (j < nv) ? j : -1;
     return;
   }
   const float* x = scores + row * ld;
   const bool vec = ((ld & 3) == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
   if (nv > TK_BM_WORDS * 32) {  // longer than the selection bitmap: exact multi-pass path
-    topk_exact(sm, x, nv, vec, k, out);
+    if (crank == 0) topk_exact(sm, x, nv, vec, k, out);
     return;
   }
   const int nwords = (nv + 31) >> 5;
@@ -414,47 +465,38 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
   __syncthreads();
   const uint32_t tau = select_kth_smem(sm, samp, m, j, 24);
 
-  // ---- 2. one streaming pass: every key >= tau into the candidate list (unordered;
-  //         one shared atomic per warp and step, no block barriers)
-  {
-    uint32_t cur[TK_EPT], nxt[TK_EPT];
-    load_keys16(x, nv, vec, TK_EPT * tid, cur);
-    for (int c0 = 0; c0 < nv; c0 += TK_CHUNK) {
-      const int i0 = c0 + TK_EPT * tid;
-      if (c0 + TK_CHUNK < nv) load_keys16(x, nv, vec, i0 + TK_CHUNK, nxt);
-      int hits = 0;
-#pragma unroll
-      for (int e = 0; e < TK_EPT; ++e) hits += (i0 + e < nv && cur[e] >= tau) ? 1 : 0;
-      int incl = hits;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const int wtot = __shfl_sync(0xffffffffu, incl, 31);
-      if (wtot) {
-        int base = 0;
-        if (lane == 31) base = atomicAdd(&sm.counter, wtot);
-        base = __shfl_sync(0xffffffffu, base, 31);
-        int pos = base + incl - hits;
-        if (hits) {
-#pragma unroll
-          for (int e = 0; e < TK_EPT; ++e) {
-            if (i0 + e < nv && cur[e] >= tau) {
-              if (pos < TK_CAP) {
-                sm.cand_key[pos] = cur[e];
-                sm.cand_idx[pos] = i0 + e;
-              }
-              ++pos;
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < TK_EPT; ++e) cur[e] = nxt[e];
-    }
-  }
+  // ---- 2. one streaming pass over this CTA's part of the row: every key >= tau into
+  //         the candidate list (unordered; one shared atomic per warp and step)
+  const int seg = ((nv + S - 1) / S + TK_EPT - 1) / TK_EPT * TK_EPT;
+  const int lo = min(nv, static_cast<int>(crank) * seg), hi = min(nv, lo + seg);
+  collect_candidates(sm, x, lo, hi, vec, tau);
   __syncthreads();
+  if (S > 1) {
+    // ---- 2b. the leader appends the other CTAs' candidates (distributed shared memory)
+    cluster_sync_all();  // every CTA's list is complete
+    if (crank == 0) {
+      const int own = sm.counter;
+      int total = own;
+      bool over = own > TK_CAP;
+      for (uint32_t p = 1; p < S; ++p) {
+        const int cnt = static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sm.counter), p)));
+        over = over || cnt > TK_CAP;
+        const int take = (!over && total + cnt <= TK_CAP) ? cnt : 0;
+        const uint32_t rk = mapa_shared(smem_u32(sm.cand_key), p);
+        const uint32_t ri = mapa_shared(smem_u32(sm.cand_idx), p);
+        for (int c = tid; c < take; c += TK_THREADS) {
+          sm.cand_key[total + c] = ld_cluster_u32(rk + 4u * c);
+          sm.cand_idx[total + c] = static_cast<int>(ld_cluster_u32(ri + 4u * c));
+        }
+        total += cnt;
+      }
+      __syncthreads();
+      if (tid == 0) sm.counter = over ? TK_CAP + 1 : total;
+    }
+    cluster_sync_all();  // the leader is done reading the others' lists
+    if (crank != 0) return;
+    __syncthreads();
+  }
   const int C = sm.counter;
   if (C < k || C > TK_CAP) {
     // the sample misjudged the threshold (or the row is heavily tied): exact path
@@ -533,9 +575,33 @@ ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0,
       cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
       "cudaFuncSetAttribute(topk)");
   if (st) return st;
-  topk_kernel<<<static_cast<unsigned>(rows), TK_THREADS, smem, stream>>>(scores, ld, n, pos0, k,
-                                                                         idx);
-  st = cuda_check(cudaGetLastError(), "topk_kernel launch");
+  // Few long rows (decode): split each row over a cluster of S CTAs so that the
+  // grid fills the GPU (two CTAs fit on an SM).
+  int S = 1;
+  if (n >= 32768 && n <= TK_BM_WORDS * 32) {
+    const long slots = 2L * num_sms();
+    while (S < 8 && rows * 2 * S <= slots) S *= 2;
+  }
+  if (S == 1) {
+    topk_kernel<<<static_cast<unsigned>(rows), TK_THREADS, smem, stream>>>(scores, ld, n, pos0, k,
+                                                                           idx);
+    st = cuda_check(cudaGetLastError(), "topk_kernel launch");
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(rows * S));
+    cfg.blockDim = dim3(TK_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    st = cuda_check(cudaLaunchKernelEx(&cfg, topk_kernel, scores, ld, n, pos0, k, idx),
+                    "topk_kernel cluster launch");
+  }
   if (st) return st;
   // algorithmic bytes: every candidate score read once, the index rows written once
   const double cand = pos0 < 0 ? static_cast<double>(rows) * n

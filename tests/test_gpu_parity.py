@@ -67,6 +67,42 @@ def test_topk_ties_signed_zeros_and_degenerate_rows():
     np.testing.assert_array_equal(got, oracle.topk(s, k))
 
 
+@pytest.mark.parametrize("nrows", [8, 17, 64])
+def test_topk_row_clusters_with_ties(nrows):
+    """Few long rows are split over a cluster of CTAs (8, 4 and 2 per row here):
+    degenerate and tie-heavy rows (exact fallback in the merging CTA) and random rows,
+    bit-exact."""
+    k, n = 2048, 40000
+    g = np.random.default_rng(nrows)
+    rows = [np.zeros(n, np.float32), np.full(n, -2.5, np.float32)]
+    r = np.zeros(n, np.float32)
+    r[1::2] = -0.0
+    rows.append(r)
+    rows.append(g.choice([0.0, 0.5, 1.0], size=n).astype(np.float32))
+    r = g.standard_normal(n).astype(np.float32)
+    r[5000:12000] = 1.25                              # ties around the k-th key
+    rows.append(r)
+    r = g.standard_normal(n).astype(np.float32)
+    r[-3000:] = 9.0                                   # the top keys all in the last part
+    rows.append(r)
+    while len(rows) < nrows:
+        rows.append(g.standard_normal(n).astype(np.float32))
+    s = np.stack(rows[:nrows])
+    got = ic.ic_topk(torch.from_numpy(s).to(DEV), k).cpu().numpy()
+    _sync()
+    np.testing.assert_array_equal(got, oracle.topk(s, k))
+
+
+def test_topk_decode_shape_clusters_and_causal():
+    """64 rows of 200000 scores at causal position 199999 (the decode step's shape)."""
+    g = torch.Generator().manual_seed(11)
+    s = torch.randn(64, 200000, generator=g)
+    got = ic.ic_topk(s.to(DEV), 2048, pos0=199999).cpu().numpy()
+    _sync()
+    ref = oracle.topk(s.numpy(), 2048, valid=oracle.causal_valid(64, 199999, 200000))
+    np.testing.assert_array_equal(got, ref)
+
+
 @pytest.mark.parametrize("n", [1, 2047, 2048, 2049, 4096])
 def test_topk_sizes_around_k(n):
     k = 2048
@@ -209,6 +245,29 @@ def test_attn_mla_decode_split_equals_unsplit():
                                idx.cpu().numpy(), 0.05, dv=512)
     assert_attn_close(_np(o_split), ro)
     assert_attn_close(_np(o_one), ro)
+
+
+@pytest.mark.parametrize("B,R,k,Lkv", [(1, 1, 2048, 5000), (2, 1, 2048, 3000), (3, 1, 1000, 1200),
+                                       (1, 2, 33, 40), (64, 1, 2048, 2100)])
+def test_attn_mla_split_pieces(B, R, k, Lkv):
+    """Few queries: the (query, tile) pairs are cut into one range per SM, so a query
+    can be split into up to 64 pieces (one or two tiles each) merged by the combine
+    kernel; ragged lists (-1 tails) and a hole included."""
+    g = torch.Generator().manual_seed(B * 1000 + R * 10 + k)
+    q = torch.randn(B, R, 16, 576, generator=g).to(torch.bfloat16)
+    kv = torch.randn(B, Lkv, 576, generator=g).to(torch.bfloat16)
+    idx = _rand_idx(B, R, k, Lkv, seed=k + B, pad_from=max(1, k - 5))
+    idx[0, 0, 3] = -1
+    scale = 1 / math.sqrt(576)
+    ws = torch.empty(ic.ic_attn_workspace_size(B, R, 16, 512, k) // 4 + 1, device=DEV)
+    assert ws.numel() > 1
+    lse = torch.empty(B, R, 16, device=DEV)
+    out = ic.ic_sparse_attn(q.to(DEV), kv.to(DEV), torch.from_numpy(idx).to(DEV), scale, lse=lse,
+                            workspace=ws)
+    _sync()
+    ro, rl = oracle.sparse_attn(q.float().numpy(), kv.float().numpy(), idx, scale, dv=512)
+    assert_attn_close(_np(out), ro)
+    np.testing.assert_allclose(lse.cpu().numpy(), rl, atol=2e-3, rtol=1e-3)
 
 
 def test_attn_f32_mqa_parity():
