@@ -74,14 +74,26 @@ struct AttnArgs {
   const int* idx;           // [B, R, k]
   int B, R, Lkv, k;
   float scale_log2;         // softmax scale * log2(e)
-  int nsplit, chunk;        // index list split into nsplit chunks of `chunk` entries
-  long items;               // B * R * nsplit
+  long items;               // B * R queries
+  // Split mode (few queries): the B*R*tq (query, 32-key tile) pairs are cut into
+  // gridDim.x equal contiguous ranges, one per CTA; each (query, range) piece
+  // leaves a partial result in slot query * maxp + (its CTA - the query's first CTA).
+  int split;
+  int tq;                   // tiles per query: ceil(k / 32)
+  int maxp;                 // partial slots per query
+  long tot;                 // items * tq
   int idx_bulk;             // index rows 16-byte aligned: fetch each list with one bulk copy
-  __nv_bfloat16* out;       // [B, R, 16, 512]   (nsplit == 1)
-  float* lse;               // [B, R, 16] or null (nsplit == 1)
-  float* part_o;            // [items, 16, 512] (nsplit > 1)
-  float* part_ml;           // [items, 16, 2]   (nsplit > 1)
+  __nv_bfloat16* out;       // [B, R, 16, 512]   (not split)
+  float* lse;               // [B, R, 16] or null (not split)
+  float* part_o;            // [items * maxp, 16, 512] (split)
+  float* part_ml;           // [items * maxp, 16, 2]   (split)
 };
+
+// CTA holding (query, tile) pair t of the split list: the largest c with
+// floor(c * tot / G) <= t.
+__host__ __device__ __forceinline__ long attn_cta_of(long t, long tot, long G) {
+  return (t * G + G - 1) / tot;
+}
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
                                          uint32_t bar) {
@@ -119,15 +131,35 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 struct AttnItem {
   long qrow;
-  int beg, end;
+  int beg, end;  // entries [beg, end) of the query's index list
+  long pslot;    // partial slot (split mode)
 };
-__device__ __forceinline__ AttnItem attn_item(const AttnArgs& a, long it) {
+// Number of items of this CTA.
+__device__ __forceinline__ long attn_nitems(const AttnArgs& a) {
+  if (!a.split)
+    return blockIdx.x < a.items ? (a.items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  const long lo = a.tot * blockIdx.x / gridDim.x, hi = a.tot * (blockIdx.x + 1) / gridDim.x;
+  return hi > lo ? (hi - 1) / a.tq - lo / a.tq + 1 : 0;
+}
+// Item j of this CTA.
+__device__ __forceinline__ AttnItem attn_item(const AttnArgs& a, long j) {
   AttnItem x;
-  x.qrow = it / a.nsplit;
-  const int sp = static_cast<int>(it % a.nsplit);
-  x.beg = sp * a.chunk;
-  x.end = min(x.beg + a.chunk, a.k);
+  if (!a.split) {
+    x.qrow = blockIdx.x + j * gridDim.x;
+    x.beg = 0;
+    x.end = a.k;
+    x.pslot = x.qrow;
+    return x;
+  }
+  const long lo = a.tot * blockIdx.x / gridDim.x, hi = a.tot * (blockIdx.x + 1) / gridDim.x;
+  x.qrow = lo / a.tq + j;
+  const long q0 = x.qrow * a.tq;
+  const long t0 = lo > q0 ? lo : q0;
+  const long t1 = hi < q0 + a.tq ? hi : q0 + a.tq;
+  x.beg = static_cast<int>((t0 - q0) * AT_BK);
+  x.end = min(static_cast<int>((t1 - q0) * AT_BK), a.k);
   if (x.end < x.beg) x.end = x.beg;
+  x.pslot = x.qrow * a.maxp + (blockIdx.x - attn_cta_of(q0, a.tot, gridDim.x));
   return x;
 }
 
@@ -172,11 +204,12 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
   const bool mine = (lane >> 3) == pw;  // this lane issues its row's copy
   int ib = 0;
   long nitem = 0;
-  if (pw == 0 && blockIdx.x < a.items) {
-    attn_load_indices(sm, a, blockIdx.x, 0, bulk);
+  const long nj = attn_nitems(a);
+  if (pw == 0 && nj > 0) {
+    attn_load_indices(sm, a, 0, 0, bulk);
     ipending[0] = bulk;
   }
-  for (long it = blockIdx.x; it < a.items; it += gridDim.x, ib ^= 1) {
+  for (long it = 0; it < nj; ++it, ib ^= 1) {
     const AttnItem x = attn_item(a, it);
     const int cnt = x.end - x.beg;
     const long b = x.qrow / a.R;
@@ -187,8 +220,8 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
       break;
     ++nitem;
     // the next item's list streams in while this one's rows are gathered
-    const long nit = it + gridDim.x;
-    if (pw == 0 && nit < a.items) {
+    const long nit = it + 1;
+    if (pw == 0 && nit < nj) {
       attn_load_indices(sm, a, nit, ib ^ 1, bulk);
       ipending[ib ^ 1] = bulk;
     }
@@ -339,7 +372,8 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
   uint32_t ph = 0;
   int qwaits = 0;
   int rel = -1;  // stage of the previous tile, released after the next partial barrier
-  for (long it = blockIdx.x; it < a.items; it += gridDim.x) {
+  const long nj = attn_nitems(a);
+  for (long it = 0; it < nj; ++it) {
     const AttnItem x = attn_item(a, it);
     if (!mbar_wait(smem_u32(&sm.qfull), qwaits & 1, abort, kErrTimeoutEpilogue)) return;
     ++qwaits;
@@ -439,7 +473,7 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
     named_bar_sync(1, AT_CONSUMERS);
     const float M0 = sm.fin_m[g], M1 = sm.fin_m[g + 8];
     const float L0 = sm.fin_l[g], L1 = sm.fin_l[g + 8];
-    if (a.nsplit == 1) {
+    if (!a.split) {
       const float inv0 = L0 > 0.f ? 1.f / L0 : 0.f, inv1 = L1 > 0.f ? 1.f / L1 : 0.f;
       __nv_bfloat16* ob = a.out + x.qrow * (AT_H * AT_DV);
 #pragma unroll
@@ -455,7 +489,8 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
             L1 > 0.f ? (M1 + log2f(L1)) * 0.69314718055994531f : -INFINITY;
       }
     } else {
-      float* po = a.part_o + it * (AT_H * AT_DV);
+      const long ps = x.pslot;
+      float* po = a.part_o + ps * (AT_H * AT_DV);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int d = 64 * warp + 8 * i + 2 * cq;
@@ -463,10 +498,10 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
         *reinterpret_cast<float2*>(po + (g + 8) * AT_DV + d) = make_float2(o[i][2], o[i][3]);
       }
       if (warp == 0 && cq == 0) {
-        a.part_ml[(it * AT_H + g) * 2] = M0;
-        a.part_ml[(it * AT_H + g) * 2 + 1] = L0;
-        a.part_ml[(it * AT_H + g + 8) * 2] = M1;
-        a.part_ml[(it * AT_H + g + 8) * 2 + 1] = L1;
+        a.part_ml[(ps * AT_H + g) * 2] = M0;
+        a.part_ml[(ps * AT_H + g) * 2 + 1] = L0;
+        a.part_ml[(ps * AT_H + g + 8) * 2] = M1;
+        a.part_ml[(ps * AT_H + g + 8) * 2 + 1] = L1;
       }
     }
   }
@@ -503,21 +538,24 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const AttnArgs 
   __syncthreads();
 }
 
-// Merges the nsplit partial results of one query: per head,
+// Merges the partial results of one query (its pieces in split mode): per head,
 // M = max m_i, L = sum l_i 2^(m_i - M), O = sum O_i 2^(m_i - M) / L.
-__global__ void attn_combine_kernel(const float* part_o, const float* part_ml, int nsplit,
-                                    __nv_bfloat16* out, float* lse) {
+__global__ void attn_combine_kernel(const float* part_o, const float* part_ml, int maxp, long tot,
+                                    int tq, int G, __nv_bfloat16* out, float* lse) {
   const long qrow = blockIdx.x;
   const int h = blockIdx.y;
+  const long c0 = attn_cta_of(qrow * tq, tot, G);
+  const int np = static_cast<int>(attn_cta_of((qrow + 1) * tq - 1, tot, G) - c0 + 1);  // <= 64
+  const long s0 = qrow * maxp;
   __shared__ float wsh[64];
   __shared__ float inv_l;
   if (threadIdx.x == 0) {
     float M = -INFINITY;
-    for (int i = 0; i < nsplit; ++i) M = fmaxf(M, part_ml[((qrow * nsplit + i) * AT_H + h) * 2]);
+    for (int i = 0; i < np; ++i) M = fmaxf(M, part_ml[((s0 + i) * AT_H + h) * 2]);
     float L = 0.f;
-    for (int i = 0; i < nsplit; ++i) {
-      const float mi = part_ml[((qrow * nsplit + i) * AT_H + h) * 2];
-      const float li = part_ml[((qrow * nsplit + i) * AT_H + h) * 2 + 1];
+    for (int i = 0; i < np; ++i) {
+      const float mi = part_ml[((s0 + i) * AT_H + h) * 2];
+      const float li = part_ml[((s0 + i) * AT_H + h) * 2 + 1];
       const float wi = (mi == -INFINITY) ? 0.f : exp2f(mi - M);
       wsh[i] = wi;
       L += li * wi;
@@ -528,27 +566,43 @@ __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, i
   __syncthreads();
   for (int d = threadIdx.x; d < AT_DV; d += blockDim.x) {
     float acc = 0.f;
-    for (int i = 0; i < nsplit; ++i)
-      acc += wsh[i] * part_o[((qrow * nsplit + i) * AT_H + h) * AT_DV + d];
+    for (int i = 0; i < np; ++i) acc += wsh[i] * part_o[((s0 + i) * AT_H + h) * AT_DV + d];
     out[(qrow * AT_H + h) * AT_DV + d] = __float2bfloat16_rn(acc * inv_l);
   }
 }
 
-static int pick_splits(long items, int k) {
-  const long want = 4L * num_sms();  // persistent CTAs: about four items per SM
-  if (items >= want) return 1;
-  long s = (want + items - 1) / items;
-  long maxs = (k + 255) / 256;  // at least 256 entries per split
-  if (s > maxs) s = maxs;
-  if (s > 64) s = 64;
-  return s < 1 ? 1 : static_cast<int>(s);
+// Split plan for few queries: G CTAs over the items*tq (query, tile) pairs, each
+// query cut into at most 64 pieces (G <= 63 * items keeps a range >= tq / 63 tiles).
+struct SplitPlan {
+  bool split;
+  int G, tq, maxp;
+  long tot;
+};
+static SplitPlan split_plan(long items, int k) {
+  SplitPlan p{false, 0, 0, 0, 0};
+  const long nsm = num_sms();
+  if (items <= 0 || items >= 4 * nsm) return p;  // enough queries for every SM
+  p.tq = (k + AT_BK - 1) / AT_BK;
+  p.tot = items * p.tq;
+  long G = nsm;
+  if (G > p.tot) G = p.tot;
+  if (G > 63 * items) G = 63 * items;
+  p.G = static_cast<int>(G);
+  int mx = 1;
+  for (long q = 0; q < items; ++q) {
+    const long np = attn_cta_of((q + 1) * p.tq - 1, p.tot, G) - attn_cta_of(q * p.tq, p.tot, G) + 1;
+    if (np > mx) mx = static_cast<int>(np);
+  }
+  p.maxp = mx;
+  p.split = p.G > 1 || items > 1;
+  return p;
 }
 
 size_t attn_mla_ws_bytes(int batch, int rows, int k) {
   const long items = static_cast<long>(batch) * rows;
-  const int ns = pick_splits(items, k);
-  if (ns <= 1) return 0;
-  return static_cast<size_t>(items) * ns * AT_H * (AT_DV + 2) * sizeof(float);
+  const SplitPlan p = split_plan(items, k);
+  if (!p.split) return 0;
+  return static_cast<size_t>(items) * p.maxp * AT_H * (AT_DV + 2) * sizeof(float);
 }
 
 ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* idx, int batch,
@@ -556,9 +610,9 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
                           size_t ws_bytes, long long valid_entries, cudaStream_t stream) {
   const long items = static_cast<long>(batch) * rows;
   if (items == 0) return IC_OK;
-  int ns = pick_splits(items, k);
-  const size_t per_split = static_cast<size_t>(items) * AT_H * (AT_DV + 2) * sizeof(float);
-  while (ns > 1 && (ws == nullptr || per_split * ns > ws_bytes)) --ns;
+  SplitPlan p = split_plan(items, k);
+  const size_t need = static_cast<size_t>(items) * p.maxp * AT_H * (AT_DV + 2) * sizeof(float);
+  if (p.split && (ws == nullptr || need > ws_bytes)) p.split = false;  // no room: one CTA per query
   AttnArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.kv = static_cast<const __nv_bfloat16*>(kv);
@@ -569,20 +623,22 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
   a.Lkv = Lkv;
   a.k = k;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.nsplit = ns;
-  a.chunk = ((k + ns - 1) / ns + AT_BK - 1) / AT_BK * AT_BK;
+  a.items = items;
+  a.split = p.split ? 1 : 0;
+  a.tq = p.tq;
+  a.maxp = p.maxp;
+  a.tot = p.tot;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse = lse;
-  a.items = items * ns;
   a.idx_bulk = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
-  a.part_o = static_cast<float*>(ws);
-  a.part_ml = ns > 1 ? static_cast<float*>(ws) + items * ns * AT_H * AT_DV : nullptr;
+  a.part_o = p.split ? static_cast<float*>(ws) : nullptr;
+  a.part_ml = p.split ? static_cast<float*>(ws) + items * p.maxp * AT_H * AT_DV : nullptr;
   const int smem = static_cast<int>(sizeof(AttnSmem)) + 128;
   ic_status st = cuda_check(
       cudaFuncSetAttribute(attn_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
       "cudaFuncSetAttribute(attn)");
   if (st) return st;
-  const long grid = a.items < num_sms() ? a.items : num_sms();
+  const long grid = p.split ? p.G : (items < num_sms() ? items : num_sms());
   attn_mla_kernel<<<static_cast<unsigned>(grid), AT_THREADS, smem, stream>>>(a);
   st = cuda_check(cudaGetLastError(), "attn_mla_kernel launch");
   if (st) return st;
@@ -591,13 +647,16 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
                                        : static_cast<double>(items) * k;
   const double io = static_cast<double>(items) * AT_H * (AT_DK + AT_DV) * 2.0;
   trace_launch(kKindAttnMla, stream, ve * AT_DK * 2.0 + io + 4.0 * static_cast<double>(items) * k);
-  if (ns == 1) return IC_OK;
+  if (!p.split) return IC_OK;
   attn_combine_kernel<<<dim3(static_cast<unsigned>(items), AT_H), 128, 0, stream>>>(
-      a.part_o, a.part_ml, ns, a.out, lse);
+      a.part_o, a.part_ml, p.maxp, p.tot, p.tq, p.G, a.out, lse);
   st = cuda_check(cudaGetLastError(), "attn_combine_kernel launch");
-  if (!st)
+  if (!st) {
+    // pieces actually written: every (query, CTA) overlap
+    const double pieces = static_cast<double>(p.G) + static_cast<double>(items) - 1.0;
     trace_launch(kKindAttnCombine, stream,
-                 static_cast<double>(items) * AT_H * (ns * (AT_DV + 2) * 4.0 + AT_DV * 2.0));
+                 pieces * AT_H * (AT_DV + 2) * 4.0 + static_cast<double>(items) * AT_H * AT_DV * 2.0);
+  }
   return st;
 }
 

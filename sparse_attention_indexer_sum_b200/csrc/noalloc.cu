@@ -2,12 +2,13 @@
 // its split-KV scratch held in a fixed device array of this library instead of
 // a caller-supplied workspace, for callers that cannot allocate device memory.
 //
-// The scratch is the per-split partial output and softmax state that the
-// split-KV form writes before its merge kernel combines them: per query, per
-// split, 16 heads x (512 output floats + running max + running sum).  The
-// entry point accepts at most IC_NOALLOC_MAX_QUERIES queries (batch * rows);
-// the split rule never uses more than eight splits at k <= 2048, so the array
-// is IC_NOALLOC_MAX_QUERIES x 8 x 16 x 514 floats.
+// The scratch is the partial output and softmax state that the split form writes
+// before its merge kernel combines them: per piece of a query, 16 heads x (512
+// output floats + running max + running sum).  The entry point accepts at most
+// IC_NOALLOC_MAX_QUERIES queries (batch * rows).  The split plan cuts their
+// (query, 32-key tile) pairs into one contiguous range per SM, so a call makes at
+// most SMs + 2 x queries pieces (276 on a 148-SM B200); the array holds
+// IC_NOALLOC_MAX_QUERIES x 8 pieces and a call that would need more is refused.
 #include <mutex>
 
 #include "ic_device.cuh"
