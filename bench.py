@@ -126,6 +126,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------------------------------ ranks
+def reduce_max(x: float, world: int, device) -> float:
+    """The largest of every rank's x (one all-reduce; the identity on one rank).
+    Every rank must call it the same number of times, in the same order."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank processes its own sequence (weak scaling) and
+    the job takes as long as its slowest rank."""
+    return world * tokens_per_rank / (ms_max * 1e-3)
+
+
 # ------------------------------------------------------------------------------ workload
 def make_inputs(wl, device, pattern_all, fp8: bool, seed: int):
     """Device tensors for every layer; indexer inputs for every layer that is F in any
@@ -184,11 +201,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -242,7 +255,7 @@ def run_ours(args, rank, world, local_rank):
                     peaks["source"], bf16_peak, " x2 (e4m3 nominal ratio)" if fp8 else ""),
                 "work_per_launch": d_work / d_n if d_n else None,
                 "launches": d_n, "ms_per_launch": d_ms / d_n if d_n else None}
-    value = world * wl.L / (ms * 1e-3)
+    value = job_throughput(wl.L, world, ms)
     log("rank %d: %.2f ms/step, %.0f tokens/s, indexer %.1f TFLOP/s" % (rank, ms, value, achieved))
 
     res = {

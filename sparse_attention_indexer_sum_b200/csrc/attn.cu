@@ -358,9 +358,10 @@ __device__ __forceinline__ void attn_pv(uint32_t kvbase, uint32_t pbase, float a
   }
 }
 
-// Per tile: QK partials -> shared -> barrier -> the softmax of heads 2w, 2w+1, done
-// once by warp w (16 lanes per head, 2 keys per lane) -> P, alpha -> barrier ->
-// P V by every warp, with the QK of the next tile issued alongside it.
+// Per tile: QK partials -> shared -> barrier -> the next tile's QK is issued, then
+// the softmax of heads 2w, 2w+1, done once by warp w (16 lanes per head, 2 keys
+// per lane), runs while those MMAs execute -> P, alpha -> barrier -> P V by every
+// warp.
 __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort = &sm.abort;
@@ -411,6 +412,22 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
     for (;;) {
       named_bar_sync(1, AT_CONSUMERS);  // B1: partials of cur complete, P V of prev done
       if (tid == 0 && rel >= 0) mbar_arrive(smem_u32(&sm.empty[rel]));
+      // ---- the next tile's QK goes out first: its MMAs run under this tile's softmax
+      const bool more = !cur_last;
+      float c[4][4];
+      int nxt = -1, nxt_last = 1;
+      unsigned nxt_vm = 0u;
+      if (more) {
+        if (!mbar_wait(smem_u32(&sm.full[stage]), ph, abort, kErrTimeoutEpilogue)) return;
+        nxt = stage;
+        nxt_last = sm.last[stage];
+        nxt_vm = sm.vmask[stage];
+        attn_qk(smem_u32(&sm.kv[stage][0][0]), qa, kq, kh, lane, c);
+        if (++stage == AT_STAGES) {
+          stage = 0;
+          ph ^= 1;
+        }
+      }
       // ---- softmax of head sh over keys sk, sk+1 (done once)
       {
         float2 z = make_float2(0.f, 0.f);
@@ -438,22 +455,6 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
         if ((lane & 15) == 0) sm.alpha[sh] = al;
       }
       named_bar_sync(1, AT_CONSUMERS);  // B2: P, alpha complete
-      // ---- the next tile's QK goes out alongside this tile's P V
-      const bool more = !cur_last;
-      float c[4][4];
-      int nxt = -1, nxt_last = 1;
-      unsigned nxt_vm = 0u;
-      if (more) {
-        if (!mbar_wait(smem_u32(&sm.full[stage]), ph, abort, kErrTimeoutEpilogue)) return;
-        nxt = stage;
-        nxt_last = sm.last[stage];
-        nxt_vm = sm.vmask[stage];
-        attn_qk(smem_u32(&sm.kv[stage][0][0]), qa, kq, kh, lane, c);
-        if (++stage == AT_STAGES) {
-          stage = 0;
-          ph ^= 1;
-        }
-      }
       attn_pv(smem_u32(&sm.kv[cur][0][0]), smem_u32(&sm.p[0][0]), sm.alpha[g], sm.alpha[g + 8],
               warp, lane, o);
       rel = cur;
