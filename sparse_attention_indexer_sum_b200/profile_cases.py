@@ -1,0 +1,131 @@
+"""Small, fixed cases of each hot kernel, for capturing them under a profiler.
+
+    python -m sparse_attention_indexer_sum_b200.profile_cases indexer_longrows
+    python -m sparse_attention_indexer_sum_b200.profile_cases attn_tail4k
+    python -m sparse_attention_indexer_sum_b200.profile_cases decode_indexer
+
+Each case builds its inputs once, on the GPU, with seeded generators. It runs the
+kernels through the C ABI, 2 warm-up rounds then 3 traced rounds, and prints
+each traced launch's time and throughput. With ncu, `-s 2 -c 1` on the kernel's
+name captures a warm launch. Every case fits in a few GB of device memory.
+
+  indexer_longrows  512 query rows at causal positions 100000..100511 against
+                    100512 keys (bf16, H=64, d=128, w ~ U(0,1)/8): ic_indexer_scores,
+                    then ic_topk (k = 2048) on the same rows.
+  attn_tail4k       the last 4096 query rows of the 200000-token prefill workload,
+                    with index sets from the indexer + top-k on those rows, then
+                    ic_sparse_attn over the full 200000-row latent KV.
+  decode_indexer    64 sequences x 1 query at position 199999 over an e4m3 key
+                    cache of 200000 keys (per-token scales), then ic_topk.
+"""
+from __future__ import annotations
+
+import math
+import sys
+
+import torch
+
+from . import binding as ic
+from . import synth
+
+
+def _report(trace):
+    for name, ms, work in trace:
+        unit = "TFLOP/s" if name.startswith("indexer_tc") else "GB/s"
+        rate = work / ms / 1e9 if unit == "TFLOP/s" else work / ms / 1e6
+        print("%-18s %9.3f ms  %10.1f %s" % (name, ms, rate, unit))
+
+
+def _rounds(fn, warm=2, timed=3):
+    for _ in range(warm):
+        fn()
+    ic.ic_device_status()
+    ic.ic_trace_begin(256)
+    for _ in range(timed):
+        fn()
+    _, trace = ic.ic_trace_end(256)
+    _report(trace)
+
+
+def indexer_longrows():
+    torch.manual_seed(0)
+    dev = "cuda"
+    R, P0 = 512, 100000
+    Lk = P0 + R
+    q = (torch.randn(R, 64, 128, device=dev) / math.sqrt(128)).to(torch.bfloat16)
+    k = (torch.randn(Lk, 128, device=dev) / math.sqrt(128)).to(torch.bfloat16)
+    w = torch.rand(R, 64, device=dev) / 8
+    scores = torch.empty(R, Lk, device=dev)
+    idx = torch.empty(R, 2048, dtype=torch.int32, device=dev)
+
+    def rnd():
+        ic.ic_indexer_scores(q, k, w, scores=scores, pos0=P0)
+        ic.ic_topk(scores, 2048, pos0=P0, idx=idx)
+    _rounds(rnd)
+
+
+def attn_tail4k():
+    dev = "cuda"
+    wl = synth.WORKLOADS["prefill_200k"]
+    L, R = wl.L, 4096
+    P0 = L - R
+    d = synth.indexer_inputs(wl, 0, device=dev)
+    q_idx = d["q_idx"][P0:].clone()
+    w = d["w"][P0:].clone()
+    k_idx = d["k_idx"]
+    del d
+    torch.cuda.empty_cache()
+    scores = torch.empty(R, L, device=dev)
+    idx = torch.empty(R, wl.k, dtype=torch.int32, device=dev)
+    ic.ic_indexer_scores(q_idx, k_idx, w, scores=scores, pos0=P0)
+    ic.ic_topk(scores, wl.k, pos0=P0, idx=idx)
+    ic.ic_device_status()
+    del scores, q_idx, k_idx
+    torch.cuda.empty_cache()
+    a = synth.attn_inputs(wl, 0, device=dev)
+    q = a["q"][P0:].clone()
+    kv = a["kv"]
+    del a
+    torch.cuda.empty_cache()
+    out = torch.empty(R, 16, 512, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(R, 16, device=dev)
+    _rounds(lambda: ic.ic_sparse_attn(q, kv, idx, wl.scale, out=out, lse=lse))
+
+
+def decode_indexer():
+    dev = "cuda"
+    B, L = 64, 200000
+    g = torch.Generator(device=dev).manual_seed(0)
+    q = (torch.randn(B, 1, 64, 128, device=dev, generator=g) / math.sqrt(128)).to(torch.bfloat16)
+    q8, qs = ic.ic_quant_e4m3_rows(q)
+    k8 = torch.empty(B, L, 128, dtype=torch.uint8, device=dev)
+    ks = torch.empty(B, L, dtype=torch.float32, device=dev)
+    for b in range(B):
+        kb = (torch.randn(L, 128, device=dev, generator=g) / math.sqrt(128)).to(torch.bfloat16)
+        ic.ic_quant_e4m3_rows(kb, codes=k8[b], scales=ks[b])
+    w = torch.rand(B, 1, 64, device=dev, generator=g) / 8
+    scores = torch.empty(B, 1, L, device=dev)
+    idx = torch.empty(B, 1, 2048, dtype=torch.int32, device=dev)
+
+    def rnd():
+        ic.ic_indexer_scores(q8, k8, w, scores=scores, pos0=L - 1, q_scale=qs, k_scale=ks)
+        ic.ic_topk(scores.view(B, L), 2048, pos0=L - 1, idx=idx.view(B, 2048))
+    _rounds(rnd)
+
+
+CASES = {"indexer_longrows": indexer_longrows, "attn_tail4k": attn_tail4k,
+         "decode_indexer": decode_indexer}
+
+
+def main(argv=None) -> int:
+    argv = sys.argv[1:] if argv is None else argv
+    if len(argv) != 1 or argv[0] not in CASES:
+        print("usage: python -m sparse_attention_indexer_sum_b200.profile_cases {%s}" %
+              ",".join(CASES), file=sys.stderr)
+        return 2
+    CASES[argv[0]]()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
