@@ -8,27 +8,26 @@
 // The work is bound by gathering k latent rows (1152 B each) per query: with
 // 16 heads there are only ~30 flops per gathered byte, far below the tensor
 // ridge.  So the kernel is built around the gather:
-//   * one producer warp issues one TMA bulk copy (cp.async.bulk, 1152 B) per
-//     selected row straight into a 4-stage ring of 32-row shared tiles, each
-//     stage completing on an mbarrier by transaction count -- up to 147 KB of
-//     gathers in flight per SM, with no per-thread copy instructions; each
-//     item's index list arrives by one more bulk copy, one item ahead;
+//   * four producer warps issue one TMA bulk copy (cp.async.bulk, 1152 B) per
+//     selected row (8 rows of each 32-row tile per warp) straight into a
+//     4-stage ring of shared tiles, each stage completing on an mbarrier by
+//     transaction count; producer 0 also fetches each item's index list (one
+//     bulk copy, one item ahead) and its 16 query rows;
 //   * eight consumer warps run S = Q K^T (16 x 32 x 576) and O += P V
 //     (16 x 512 x 32) on the warp-level bf16 tensor-core MMA, whose M = 16 is
-//     exactly the 16 heads, with an online softmax in base 2;
-//   * CTAs are persistent (one per SM) and walk (query, split) items
-//     round-robin, so the producer streams the next query's rows while the
-//     consumers finish the current one, and neighbouring queries (which share
-//     many selected rows) run at the same time and hit in L2.
+//     exactly the 16 heads, with an online softmax in base 2.  QK: warp w covers
+//     keys 16(w%2)..+16 over dims 144(w/2)..+144 with its quarter of Q in
+//     registers; the four partial scores meet in shared memory.  The next tile's
+//     QK is issued, then warp w computes the softmax of heads 2w, 2w+1 once
+//     (16 lanes per head) and leaves P (bf16) and the rescale factors in shared
+//     memory.  PV: warp w owns output dims 64w..+64;
+//   * CTAs are persistent (one per SM).  With many queries, they walk the
+//     queries round-robin, so neighbouring queries (which share many selected
+//     rows) run at the same time and hit in L2.  With few queries (decode), the
+//     (query, tile) pairs are cut into one contiguous range per CTA.  Each
+//     (query, range) piece leaves an unnormalised partial in the workspace, and
+//     attn_combine_kernel merges them.
 // Shared rows are padded to 1168 B so that ldmatrix is bank-conflict free.
-// QK: consumer warp w covers keys 16(w%2)..+16 over dims 144(w/2)..+144 with
-// its quarter of Q in registers (four accumulator chains); the four partial
-// scores meet in shared memory, behind the tile's only barrier.  Every warp
-// then rebuilds the softmax of all 16 heads for the tile directly in its PV
-// A fragments (the running max and sum live, identical, in every warp's
-// registers).  PV: warp w owns output dims 64w..+64.  Decode-sized batches split
-// each index list over several items; their unnormalised partial outputs are
-// merged by attn_combine_kernel.
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
@@ -540,7 +539,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const AttnArgs 
 }
 
 // Merges the partial results of one query (its pieces in split mode): per head,
-// M = max m_i, L = sum l_i 2^(m_i - M), O = sum O_i 2^(m_i - M) / L.
+// M = max m_i, L = sum l_i 2^(m_i - M), O = sum O_i 2^(m_i - M) / L.  Warp 0 reads
+// the pieces' (m, l) in parallel (lane i: pieces i and i + 32) and reduces them
+// with shuffles; then every thread accumulates its output dims over the pieces.
 __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, int maxp, long tot,
                                     int tq, int G, __nv_bfloat16* out, float* lse) {
   const long qrow = blockIdx.x;
@@ -550,25 +551,44 @@ __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, i
   const long s0 = qrow * maxp;
   __shared__ float wsh[64];
   __shared__ float inv_l;
-  if (threadIdx.x == 0) {
-    float M = -INFINITY;
-    for (int i = 0; i < np; ++i) M = fmaxf(M, part_ml[((s0 + i) * AT_H + h) * 2]);
-    float L = 0.f;
-    for (int i = 0; i < np; ++i) {
-      const float mi = part_ml[((s0 + i) * AT_H + h) * 2];
-      const float li = part_ml[((s0 + i) * AT_H + h) * 2 + 1];
-      const float wi = (mi == -INFINITY) ? 0.f : exp2f(mi - M);
-      wsh[i] = wi;
-      L += li * wi;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    if (lane < np) {
+      m0 = part_ml[((s0 + lane) * AT_H + h) * 2];
+      l0 = part_ml[((s0 + lane) * AT_H + h) * 2 + 1];
     }
-    inv_l = L > 0.f ? 1.f / L : 0.f;
-    if (lse) lse[qrow * AT_H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    if (lane + 32 < np) {
+      m1 = part_ml[((s0 + lane + 32) * AT_H + h) * 2];
+      l1 = part_ml[((s0 + lane + 32) * AT_H + h) * 2 + 1];
+    }
+    float M = fmaxf(m0, m1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M);
+    const float w1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M);
+    float L = l0 * w0 + l1 * w1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane < np) wsh[lane] = w0;
+    if (lane + 32 < np) wsh[lane + 32] = w1;
+    if (lane == 0) {
+      inv_l = L > 0.f ? 1.f / L : 0.f;
+      if (lse) lse[qrow * AT_H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    }
   }
   __syncthreads();
+  const float* po = part_o + (s0 * AT_H + h) * AT_DV;
+  const long pstride = static_cast<long>(AT_H) * AT_DV;
   for (int d = threadIdx.x; d < AT_DV; d += blockDim.x) {
-    float acc = 0.f;
-    for (int i = 0; i < np; ++i) acc += wsh[i] * part_o[((s0 + i) * AT_H + h) * AT_DV + d];
-    out[(qrow * AT_H + h) * AT_DV + d] = __float2bfloat16_rn(acc * inv_l);
+    float a0 = 0.f, a1 = 0.f;
+    int i = 0;
+    for (; i + 1 < np; i += 2) {  // two independent loads in flight per step
+      a0 += wsh[i] * po[i * pstride + d];
+      a1 += wsh[i + 1] * po[(i + 1) * pstride + d];
+    }
+    if (i < np) a0 += wsh[i] * po[i * pstride + d];
+    out[(qrow * AT_H + h) * AT_DV + d] = __float2bfloat16_rn((a0 + a1) * inv_l);
   }
 }
 

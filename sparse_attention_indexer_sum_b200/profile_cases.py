@@ -3,6 +3,7 @@
     python -m sparse_attention_indexer_sum_b200.profile_cases indexer_longrows
     python -m sparse_attention_indexer_sum_b200.profile_cases attn_tail4k
     python -m sparse_attention_indexer_sum_b200.profile_cases decode_indexer
+    python -m sparse_attention_indexer_sum_b200.profile_cases decode_attn
 
 Each case builds its inputs once, on the GPU, with seeded generators. It runs the
 kernels through the C ABI, 2 warm-up rounds then 3 traced rounds, and prints
@@ -17,6 +18,10 @@ name captures a warm launch. Every case fits in a few GB of device memory.
                     ic_sparse_attn over the full 200000-row latent KV.
   decode_indexer    64 sequences x 1 query at position 199999 over an e4m3 key
                     cache of 200000 keys (per-token scales), then ic_topk.
+  decode_attn       one decode layer's attention: 64 sequences x 1 query, each
+                    over 2048 random distinct rows of its own 20000-row latent KV
+                    (1.5 GB in all, far beyond L2); split over the SMs, partials
+                    merged by the combine kernel.
 """
 from __future__ import annotations
 
@@ -113,8 +118,23 @@ def decode_indexer():
     _rounds(rnd)
 
 
+def decode_attn():
+    dev = "cuda"
+    wl = synth.variant("decode_200k", L=20000)
+    B, L, k = wl.batch, wl.L, wl.k
+    a = synth.attn_inputs(wl, 0, device=dev)
+    q, kv = a["q"], a["kv"]
+    g = torch.Generator(device=dev).manual_seed(0)
+    idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
+    for b in range(B):
+        idx[b, 0] = torch.sort(torch.randperm(L, device=dev, generator=g)[:k]).values.int()
+    ws = torch.empty(ic.ic_attn_workspace_size(B, 1, wl.Hq, wl.Dv, k) // 4 + 1, device=dev)
+    out = torch.empty(B, 1, wl.Hq, wl.Dv, dtype=torch.bfloat16, device=dev)
+    _rounds(lambda: ic.ic_sparse_attn(q, kv, idx, wl.scale, out=out, workspace=ws))
+
+
 CASES = {"indexer_longrows": indexer_longrows, "attn_tail4k": attn_tail4k,
-         "decode_indexer": decode_indexer}
+         "decode_indexer": decode_indexer, "decode_attn": decode_attn}
 
 
 def main(argv=None) -> int:
