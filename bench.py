@@ -473,7 +473,13 @@ def run_stack32k(args, dev, barrier):
 def run_e2e(wl, layers, pattern, desc, t_cache, ws, stream, dev, args, barrier, max_over_ranks,
             world):
     """The metric through the C ABI with HOST buffers: every step copies its inputs from
-    pinned host memory and reads its result (last layer's output and the index set) back."""
+    pinned host memory and reads its result (last layer's output and the index set) back.
+
+    Steps are pipelined over three streams, as a serving loop would run them: while
+    step s computes, step s+1's inputs stream in (host -> device) and step s-1's
+    result streams out (device -> host). Inputs and results are double-buffered on
+    the device. The timed region opens before the first input copy and closes after
+    the last result has reached the host, so every byte of every step is inside it."""
     from sparse_attention_indexer_sum_b200 import binding as ic
     kinds = kinds_of(pattern)
     names_f = ["q_idx", "q_scale", "k_idx", "k_scale", "w", "q", "kv"]
@@ -494,26 +500,71 @@ def run_e2e(wl, layers, pattern, desc, t_cache, ws, stream, dev, args, barrier, 
     h2d = sum(t.numel() * t.element_size() for hs in host_in for t in hs.values())
     d2h = out_h.numel() * out_h.element_size() + t_h.numel() * t_h.element_size()
 
-    def step():
-        for d, hs in zip(layers, host_in):
-            for n, h in hs.items():
-                d[n].copy_(h, non_blocking=True)
-        ic.ic_layer_stack(pattern, desc, layers, t_cache, ws, stream=stream)
-        out_h.copy_(layers[-1]["out"], non_blocking=True)
-        t_h.copy_(t_cache, non_blocking=True)
+    # device buffer set 1: fresh tensors for everything copied in or read back
+    sets = [layers, []]
+    for l, d in enumerate(layers):
+        e = dict(d)
+        for n in host_in[l]:
+            e[n] = torch.empty_like(d[n])
+        if l == len(layers) - 1:
+            e["out"] = torch.empty_like(d["out"])
+        sets[1].append(e)
+    t_caches = [t_cache, torch.empty_like(t_cache)]
+    copy_s, back_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, in_free, done, back_done = ([ev(), ev()] for _ in range(4))
+    for b in range(2):  # every buffer starts free
+        in_free[b].record(stream)
+        back_done[b].record(back_s)
 
-    step()
+    def copy_in(b):
+        copy_s.wait_event(in_free[b])
+        with torch.cuda.stream(copy_s):
+            for d, hs in zip(sets[b], host_in):
+                for n, h in hs.items():
+                    d[n].copy_(h, non_blocking=True)
+        in_ready[b].record(copy_s)
+
+    def compute(b):
+        stream.wait_event(in_ready[b])
+        stream.wait_event(back_done[b])  # the last read-back of this set's result is done
+        ic.ic_layer_stack(pattern, desc, sets[b], t_caches[b], ws, stream=stream)
+        in_free[b].record(stream)
+        done[b].record(stream)
+
+    def copy_back(b):
+        back_s.wait_event(done[b])
+        with torch.cuda.stream(back_s):
+            out_h.copy_(sets[b][-1]["out"], non_blocking=True)
+            t_h.copy_(t_caches[b], non_blocking=True)
+        back_done[b].record(back_s)
+
+    def run(nsteps, t0=None):
+        if t0 is not None:
+            copy_s.wait_event(t0)
+        copy_in(0)
+        for i in range(nsteps):
+            if i + 1 < nsteps:
+                copy_in((i + 1) % 2)  # next step's inputs, alongside this step's compute
+            compute(i % 2)
+            copy_back(i % 2)
+        stream.wait_stream(back_s)
+        stream.wait_stream(copy_s)
+
+    run(2)  # warm-up
     barrier()
-    ke = max(2, min(args.steps, 3))
+    ke = max(2, args.steps)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(ke):
-        step()
+    run(ke, t0=e0)
     e1.record(stream)
     barrier()
     ms = max_over_ranks(e0.elapsed_time(e1) / ke)
     return {"value": world * wl.L / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke,
+            "pipelined": "inputs of step s+1 copied in and result of step s copied out "
+                         "while step s+1 / s computes; first copy-in and last copy-out "
+                         "inside the timed region"}
 
 
 # ------------------------------------------------------------------------------ CPU oracle
