@@ -185,9 +185,12 @@ def run_ours(args, rank, world, local_rank):
     pattern = wl.pattern
     allf = ",".join("F" * wl.layers)
     fp8 = args.indexer == "e4m3"
+    shard = args.shard == "rows"
     t0 = time.time()
+    # weak scaling: every rank its own sequence (seed = rank); rows sharding: every rank
+    # the same sequence, running only its zig-zag share of the query rows
     layers = make_inputs(wl, dev, [kinds_of(pattern)] + ([kinds_of(allf)] if args.compare else []),
-                         fp8, seed=rank)
+                         fp8, seed=0 if shard else rank)
     log("rank %d: inputs ready in %.1f s (%.1f GB allocated)" %
         (rank, time.time() - t0, torch.cuda.memory_allocated(dev) / 1e9))
     desc = ic.make_desc(L=wl.L, k=wl.k, H=wl.H, D=wl.D,
@@ -197,8 +200,21 @@ def run_ours(args, rank, world, local_rank):
     t_cache = torch.empty(wl.L, wl.k, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(pat=pattern):
-        ic.ic_layer_stack(pat, desc, layers, t_cache, ws, stream=stream)
+    if shard:
+        from sparse_attention_indexer_sum_b200.sharding import zigzag_row_ranges
+        row_names = ("q_idx", "q_scale", "w", "q", "out", "lse")
+        pieces = []
+        for r0, n in zigzag_row_ranges(wl.L, world, rank):
+            lay = [{f: (v[r0:r0 + n] if f in row_names else v) for f, v in d.items()}
+                   for d in layers]
+            pieces.append((r0, n, lay, t_cache[r0:r0 + n]))
+
+        def step(pat=pattern):
+            for r0, n, lay, tc in pieces:
+                ic.ic_layer_stack_rows(pat, desc, lay, r0, n, tc, ws, stream=stream)
+    else:
+        def step(pat=pattern):
+            ic.ic_layer_stack(pat, desc, layers, t_cache, ws, stream=stream)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -266,19 +282,23 @@ def run_ours(args, rank, world, local_rank):
                     peaks["source"], bf16_peak, " x2 (e4m3 nominal ratio)" if fp8 else ""),
                 "work_per_launch": d_work / d_n if d_n else None,
                 "launches": d_n, "ms_per_launch": d_ms / d_n if d_n else None}
-    value = job_throughput(wl.L, world, ms)
+    value = wl.L / (ms * 1e-3) if shard else job_throughput(wl.L, world, ms)
     log("rank %d: %.2f ms/step, %.0f tokens/s, indexer %.1f TFLOP/s" % (rank, ms, value, achieved))
 
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong" if shard else "weak",
         "vs_baseline": None, "dtype": "e4m3+bf16" if fp8 else "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "L": wl.L, "layers": wl.layers, "pattern": pattern,
                    "k": wl.k, "indexer": "H_I=64 d_I=128 %s (fp32 accumulate)" %
                    ("e4m3 per-row scales" if fp8 else "bf16"),
                    "attention": "absorbed MLA 16 heads x 576 -> 512, bf16",
-                   "batch_per_gpu": 1, "parallelism": "independent sequence per GPU" if world > 1
-                   else "single GPU", "l2": "inputs larger than L2 (no flush needed)"},
+                   "batch_per_gpu": 1,
+                   "parallelism": ("one sequence, query rows in zig-zag shares per GPU" if shard
+                                   else "independent sequence per GPU" if world > 1
+                                   else "single GPU"),
+                   "l2": "inputs larger than L2 (no flush needed)"},
         "gpu_launches": n_launch, "roofline": roofline, "stages": stages, "clocks": clk,
     }
 
@@ -294,10 +314,13 @@ def run_ours(args, rank, world, local_rank):
         barrier()
         ms_f = max_over_ranks(e0.elapsed_time(e1) / ka)
         res["all_f"] = {"pattern": allf, "ms_per_step": ms_f,
-                        "value": world * wl.L / (ms_f * 1e-3),
+                        "value": (1 if shard else world) * wl.L / (ms_f * 1e-3),
                         "speedup_fsss_over_all_f": ms_f / ms}
 
-    if args.e2e:
+    if args.e2e and shard:
+        res["e2e"] = {"value": None, "unit": UNIT,
+                      "note": "not measured in the rows-sharded mode (run the default mode)"}
+    elif args.e2e:
         res["e2e"] = run_e2e(wl, layers, pattern, desc, t_cache, ws, stream, dev, args, barrier,
                              max_over_ranks, world)
     if args.cpu_baseline and rank == 0 and world == 1:
@@ -694,6 +717,10 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--shard", default="sequences", choices=["sequences", "rows"],
+                    help="sequences: one independent 200K prefill per GPU (weak scaling, the "
+                         "default); rows: one prefill, its query rows shared out over the GPUs "
+                         "in zig-zag chunks (strong scaling)")
     ap.add_argument("--no-decode", dest="decode", action="store_false",
                     help="skip the decode (64 x 1 token at 200K context) measurement")
     ap.add_argument("--no-stack32k", dest="stack32k", action="store_false",

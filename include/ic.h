@@ -254,6 +254,21 @@ ic_status ic_layer_stack(const char* pattern, const ic_stack_desc* desc, const i
                          int nlayers, int* t_cache, void* workspace, size_t ws_bytes,
                          void* stream);
 
+/*
+ * The prefill stack for query rows [row0, row0 + rows) of the desc->L-token
+ * sequence only, so one long prefill can be shared out by rows (for example
+ * over GPUs). Row r of the call sits at position row0 + r and attends causally
+ * over keys 0..row0 + r. Per-row results are identical to ic_layer_stack's rows.
+ * The row-indexed tensors of `layers` (q_idx, q_scale, w, q, out, lse) and
+ * t_cache [rows, k] hold just these rows. k_idx, k_scale and kv hold all L keys.
+ * ic_layer_stack is this call with row0 = 0, rows = desc->L.
+ * 0 <= row0, row0 + rows <= desc->L, desc->decode = 0.  Other rules, the
+ * workspace and the errors are as ic_layer_stack.
+ */
+ic_status ic_layer_stack_rows(const char* pattern, const ic_stack_desc* desc,
+                              const ic_layer_io* layers, int nlayers, long row0, long rows,
+                              int* t_cache, void* workspace, size_t ws_bytes, void* stream);
+
 /* Decode form of the stack (desc->decode must be 1): same routing per layer,
  * one query per sequence; t_cache is [batch, k]. */
 ic_status ic_decode_step(const char* pattern, const ic_stack_desc* desc, const ic_layer_io* layers,

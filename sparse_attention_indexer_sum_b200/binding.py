@@ -29,7 +29,7 @@ EXPORTS = ("ic_last_error", "ic_version", "ic_device_status", "ic_trace_begin", 
            "ic_quant_e4m3_rows",
            "ic_indexer_scores", "ic_topk", "ic_sparse_attn", "ic_attn_workspace_size",
            "ic_layer_stack", "ic_decode_step", "ic_stack_workspace_size",
-           "ic_sparse_attn_noalloc")
+           "ic_sparse_attn_noalloc", "ic_layer_stack_rows")
 
 
 class ICError(RuntimeError):
@@ -83,11 +83,14 @@ def lib() -> ctypes.CDLL:
     L.ic_layer_stack.argtypes = [ctypes.c_char_p, ctypes.POINTER(ic_stack_desc),
                                  ctypes.POINTER(ic_layer_io), I, P, P, S, P]
     L.ic_decode_step.argtypes = L.ic_layer_stack.argtypes
+    L.ic_layer_stack_rows.argtypes = [ctypes.c_char_p, ctypes.POINTER(ic_stack_desc),
+                                      ctypes.POINTER(ic_layer_io), I, Lg, Lg, P, P, S, P]
     L.ic_stack_workspace_size.argtypes = [ctypes.POINTER(ic_stack_desc)]
     L.ic_stack_workspace_size.restype = S
     L.ic_sparse_attn_noalloc.argtypes = [P, P, Lg, P, P, I, I, I, I, I, I, I, I, F, P, P, P]
     for name in ("ic_device_status", "ic_quant_e4m3_rows", "ic_indexer_scores", "ic_topk",
-                 "ic_sparse_attn", "ic_layer_stack", "ic_decode_step", "ic_sparse_attn_noalloc"):
+                 "ic_sparse_attn", "ic_layer_stack", "ic_decode_step", "ic_sparse_attn_noalloc",
+                 "ic_layer_stack_rows"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -288,6 +291,18 @@ def ic_layer_stack(pattern: str, desc: ic_stack_desc, layers: list[dict], t_cach
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib().ic_layer_stack(pattern.encode(), ctypes.byref(desc), arr, len(layers),
                                 _p(t_cache), _p(workspace), ws_bytes, _stream(stream)))
+
+
+def ic_layer_stack_rows(pattern: str, desc: ic_stack_desc, layers: list[dict], row0: int,
+                        rows: int, t_cache, workspace, stream=None):
+    """Prefill stack for query rows [row0, row0 + rows) of the desc.L-token sequence.
+    Row-indexed layer tensors (q_idx, q_scale, w, q, out, lse) and t_cache hold just
+    those rows; k_idx, k_scale and kv hold all desc.L keys."""
+    arr = _layers(layers)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().ic_layer_stack_rows(pattern.encode(), ctypes.byref(desc), arr, len(layers),
+                                     int(row0), int(rows), _p(t_cache), _p(workspace), ws_bytes,
+                                     _stream(stream)))
 
 
 def ic_decode_step(pattern: str, desc: ic_stack_desc, layers: list[dict], t_cache, workspace,

@@ -174,11 +174,17 @@ static long score_rows(size_t ws_bytes, long L, long want) {
   return rb;
 }
 
+// Prefill runs query rows [row0, row0 + rows) of the L-token sequence (keys are
+// always 0..L-1); decode runs every sequence's one query (row0 = 0, rows = L unused).
 static ic_status run_stack(const char* pattern, const ic_stack_desc* d, const ic_layer_io* layers,
                            int nlayers, int* t_cache, void* workspace, size_t ws_bytes,
-                           void* stream_v, bool decode) {
+                           void* stream_v, bool decode, long row0 = 0, long rows = -1) {
   ic_status st = check_desc(d, decode);
   if (st) return st;
+  if (rows < 0) rows = d->L;
+  if (!decode && (row0 < 0 || rows < 0 || row0 + rows > d->L))
+    return fail(IC_ERR_INVALID_ARG, "stack: rows [%ld, %ld) outside the %d-token sequence", row0,
+                row0 + rows, d->L);
   std::vector<char> kinds;
   st = parse_pattern(pattern, &kinds);
   if (st) return st;
@@ -186,8 +192,8 @@ static ic_status run_stack(const char* pattern, const ic_stack_desc* d, const ic
     return fail(IC_ERR_INVALID_ARG, "pattern has %zu layers, nlayers is %d", kinds.size(), nlayers);
   if (!layers || !t_cache) return fail(IC_ERR_INVALID_ARG, "stack: NULL layers or t_cache");
   const int B = d->batch;
-  const int R = decode ? 1 : d->L;  // query rows per sequence
-  const long pos0 = decode ? d->L - 1 : 0;
+  const int R = decode ? 1 : static_cast<int>(rows);  // query rows per sequence
+  const long pos0 = decode ? d->L - 1 : row0;
   for (int l = 0; l < nlayers; ++l) {
     const ic_layer_io& io = layers[l];
     if (kinds[l] == 'F') {
@@ -220,13 +226,14 @@ static ic_status run_stack(const char* pattern, const ic_stack_desc* d, const ic
         const uint8_t* qi = static_cast<const uint8_t*>(io.q_idx);
         const float* qs = io.q_scale;
         if (!decode) {
-          // query rows u0 .. u0+nu-1 of the one sequence, at positions u0.., keys 0..u0+nu-1
-          const int Lk = static_cast<int>(u0 + nu);
+          // local query rows u0 .. u0+nu-1 sit at positions row0 + u0.., keys 0..row0+u0+nu-1
+          const long p0 = row0 + u0;
+          const int Lk = static_cast<int>(p0 + nu);
           st = run_indexer(qi + u0 * qrow_b, qs ? qs + u0 * d->H : nullptr, io.k_idx, io.k_scale,
                            io.w + u0 * d->H, d->idx_dtype, 1, d->H, d->D, static_cast<int>(nu), Lk,
-                           u0, scores, d->L, false, stream);
+                           p0, scores, d->L, false, stream);
           if (st) return st;
-          st = launch_topk(scores, nu, Lk, d->L, u0, d->k, t_cache + u0 * d->k, stream);
+          st = launch_topk(scores, nu, Lk, d->L, p0, d->k, t_cache + u0 * d->k, stream);
         } else {
           // sequences u0 .. u0+nu-1, one query each at position L-1 over L keys
           const uint8_t* ki = static_cast<const uint8_t*>(io.k_idx);
@@ -244,7 +251,7 @@ static ic_status run_stack(const char* pattern, const ic_stack_desc* d, const ic
     // S layers: T_cache is reused as is (the nearest preceding F layer's set)
     // out_l <- SparseAttn_l(T_cache); the score workspace is free again here
     const long long valid = decode ? static_cast<long long>(B) * (d->k < d->L ? d->k : d->L)
-                                   : causal_pairs(R, d->k, 0);
+                                   : causal_pairs(R, d->k, row0);
     st = run_attn(io.q, io.kv, d->ld_kv, io.v, t_cache, B, R, d->heads, d->dk, d->dv, d->L, d->k,
                   d->scale, io.out, io.lse, workspace, ws_bytes, valid, stream);
     if (st) return st;
@@ -371,6 +378,16 @@ ic_status ic_layer_stack(const char* pattern, const ic_stack_desc* desc, const i
                          int nlayers, int* t_cache, void* workspace, size_t ws_bytes,
                          void* stream) {
   return run_stack(pattern, desc, layers, nlayers, t_cache, workspace, ws_bytes, stream, false);
+}
+
+ic_status ic_layer_stack_rows(const char* pattern, const ic_stack_desc* desc,
+                              const ic_layer_io* layers, int nlayers, long row0, long rows,
+                              int* t_cache, void* workspace, size_t ws_bytes, void* stream) {
+  if (desc && (row0 < 0 || rows < 0 || row0 + rows > desc->L))
+    return fail(IC_ERR_INVALID_ARG, "stack: rows [%ld, %ld) outside the %d-token sequence", row0,
+                row0 + rows, desc->L);
+  return run_stack(pattern, desc, layers, nlayers, t_cache, workspace, ws_bytes, stream, false,
+                   row0, rows);
 }
 
 ic_status ic_decode_step(const char* pattern, const ic_stack_desc* desc, const ic_layer_io* layers,

@@ -97,3 +97,17 @@ def test_workspace_sizes(lib):
                           dk=576, dv=512, attn_dtype=binding.IC_BF16, scale=576 ** -0.5)
     assert binding.ic_stack_workspace_size(d) == 4096 * 200000 * 4
     assert binding.ic_attn_workspace_size(1, 200000, 16, 512, 2048) == 0  # no split at prefill
+
+
+def test_row_range_stack_rejects_rows_outside_the_sequence(lib):
+    desc = binding.make_desc(L=16, k=4, H=4, D=32, idx_dtype=binding.IC_F32, heads=4, dk=64, dv=64,
+                             attn_dtype=binding.IC_F32, scale=0.125)
+    arr = (binding.ic_layer_io * 1)()
+    for row0, rows in ((10, 7), (-1, 4), (0, -2)):
+        assert lib.ic_layer_stack_rows(b"F", ctypes.byref(desc), arr, 1, row0, rows, None, None, 0,
+                                       None) == binding.IC_ERR_INVALID_ARG
+        assert "outside" in binding.ic_last_error()
+    # a valid range gets as far as the NULL layer inputs
+    assert lib.ic_layer_stack_rows(b"F", ctypes.byref(desc), arr, 1, 4, 8, None, None, 0,
+                                   None) == binding.IC_ERR_INVALID_ARG
+    assert "NULL" in binding.ic_last_error()

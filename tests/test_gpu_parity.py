@@ -365,6 +365,33 @@ def test_stack_bf16_row_blocks_and_sharing():
         assert_attn_close(_np(dl[l]["out"][torch.from_numpy(rows).to(DEV)]), ro)
 
 
+def test_stack_rows_zigzag_pieces_equal_the_whole_stack():
+    """ic_layer_stack_rows over the zig-zag row pieces of 2 ranks (run one after the
+    other here) gives the whole stack's index sets bit for bit and its outputs within
+    the attention tolerance."""
+    from sparse_attention_indexer_sum_b200.sharding import zigzag_row_ranges
+    wl = synth.variant("prefill_8k", L=2600, pattern="F,S")
+    layers, _ = _stack_layers(wl, DEV)
+    full, t_full = _run_stack(wl, wl.pattern, layers, ic.IC_BF16)
+    desc = _desc(wl, ic.IC_BF16)
+    ws = torch.empty(ic.ic_stack_workspace_size(desc) // 4 + 1, device=DEV)
+    seen = 0
+    for rank in range(2):
+        for r0, n in zigzag_row_ranges(wl.L, 2, rank):
+            lay = [{"q_idx": d["q_idx"][r0:r0 + n], "w": d["w"][r0:r0 + n], "k_idx": d["k_idx"],
+                    "q": d["q"][r0:r0 + n], "kv": d["kv"],
+                    "out": torch.empty(n, wl.Hq, wl.Dv, dtype=torch.bfloat16, device=DEV),
+                    "lse": torch.empty(n, wl.Hq, device=DEV)} for d in layers]
+            t = torch.full((n, wl.k), -7, dtype=torch.int32, device=DEV)
+            ic.ic_layer_stack_rows(wl.pattern, desc, lay, r0, n, t, ws)
+            _sync()
+            assert torch.equal(t, t_full[r0:r0 + n]), (rank, r0, n)
+            for l in range(len(lay)):
+                assert_attn_close(_np(lay[l]["out"]), _np(full[l]["out"][r0:r0 + n]))
+            seen += n
+    assert seen == wl.L
+
+
 def test_decode_step_parity():
     """Decode: 6 sequences x 1 token over a 3000-token context, fp8 indexer cache,
     pattern F,S: T per sequence and both layers' outputs against the oracle."""

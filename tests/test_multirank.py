@@ -114,3 +114,53 @@ def test_reference_arm_does_no_work_on_other_ranks():
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+# ------------------------------------------------------------------ sharding one prefill
+def test_zigzag_plan_covers_every_row_once_and_balances_the_causal_work():
+    sys.path.insert(0, ROOT)
+    from sparse_attention_indexer_sum_b200.sharding import causal_pairs, zigzag_row_ranges
+    for L, W in ((200000, 8), (200000, 2), (1000, 3), (7, 4), (5, 1)):
+        covered = []
+        work = []
+        for r in range(W):
+            rr = zigzag_row_ranges(L, W, r)
+            covered += [t for r0, n in rr for t in range(r0, r0 + n)]
+            work.append(sum(causal_pairs(r0, n) for r0, n in rr))
+        assert sorted(covered) == list(range(L))
+        assert sum(work) == L * (L + 1) // 2
+        if L >= 1000:
+            assert max(work) / min(work) < 1.01, (L, W, work)
+    # contiguous ranges would not balance: the last of 8 ranks has 15x the first's work
+    assert causal_pairs(175000, 25000) > 14 * causal_pairs(0, 25000)
+    with pytest.raises(ValueError):
+        zigzag_row_ranges(10, 2, 2)
+
+
+def _plan_worker(rank, world, port, q):
+    _init(rank, world, port, 60)
+    import torch
+    from sparse_attention_indexer_sum_b200.sharding import zigzag_row_ranges
+    try:
+        mine = torch.tensor(zigzag_row_ranges(200000, world, rank), dtype=torch.int64)
+        got = [torch.empty_like(mine) for _ in range(world)]
+        dist.all_gather(got, mine)       # every rank sees the whole plan
+        q.put((rank, [t.tolist() for t in got]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_agree_on_a_plan_that_tiles_the_rows():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_plan_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert out[0] == out[1]
+    rows = sorted(t for rr in out[0] for r0, n in rr for t in (r0, r0 + n))
+    assert rows == [0, 50000, 50000, 100000, 100000, 150000, 150000, 200000]
