@@ -269,6 +269,23 @@ ic_status ic_layer_stack_rows(const char* pattern, const ic_stack_desc* desc,
                               const ic_layer_io* layers, int nlayers, long row0, long rows,
                               int* t_cache, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * The prefill stack over a batch of sequences of different lengths, packed
+ * along the row axis: sequence i is rows [cu_seqlens[i], cu_seqlens[i+1]) of
+ * every row-indexed tensor of `layers` (q_idx, q_scale, w, q, out, lse), of its
+ * keys (k_idx, k_scale, kv, v) and of t_cache [sum L_i, k]. Each sequence runs
+ * the whole routing loop on its own keys at positions 0..L_i - 1, as
+ * ic_layer_stack would with desc->L = L_i.  cu_seqlens: host int64 [nseq + 1],
+ * cu_seqlens[0] = 0, nondecreasing, every L_i <= desc->L (desc->L sizes the
+ * workspace: ic_stack_workspace_size(desc) covers any batch).  The sequences run
+ * one after another on `stream`.  Errors as ic_layer_stack, with the sequence
+ * named.
+ */
+ic_status ic_layer_stack_varlen(const char* pattern, const ic_stack_desc* desc,
+                                const ic_layer_io* layers, int nlayers, const long* cu_seqlens,
+                                int nseq, int* t_cache, void* workspace, size_t ws_bytes,
+                                void* stream);
+
 /* Decode form of the stack (desc->decode must be 1): same routing per layer,
  * one query per sequence; t_cache is [batch, k]. */
 ic_status ic_decode_step(const char* pattern, const ic_stack_desc* desc, const ic_layer_io* layers,

@@ -29,7 +29,7 @@ EXPORTS = ("ic_last_error", "ic_version", "ic_device_status", "ic_trace_begin", 
            "ic_quant_e4m3_rows",
            "ic_indexer_scores", "ic_topk", "ic_sparse_attn", "ic_attn_workspace_size",
            "ic_layer_stack", "ic_decode_step", "ic_stack_workspace_size",
-           "ic_sparse_attn_noalloc", "ic_layer_stack_rows")
+           "ic_sparse_attn_noalloc", "ic_layer_stack_rows", "ic_layer_stack_varlen")
 
 
 class ICError(RuntimeError):
@@ -85,12 +85,15 @@ def lib() -> ctypes.CDLL:
     L.ic_decode_step.argtypes = L.ic_layer_stack.argtypes
     L.ic_layer_stack_rows.argtypes = [ctypes.c_char_p, ctypes.POINTER(ic_stack_desc),
                                       ctypes.POINTER(ic_layer_io), I, Lg, Lg, P, P, S, P]
+    L.ic_layer_stack_varlen.argtypes = [ctypes.c_char_p, ctypes.POINTER(ic_stack_desc),
+                                        ctypes.POINTER(ic_layer_io), I, ctypes.POINTER(Lg), I, P,
+                                        P, S, P]
     L.ic_stack_workspace_size.argtypes = [ctypes.POINTER(ic_stack_desc)]
     L.ic_stack_workspace_size.restype = S
     L.ic_sparse_attn_noalloc.argtypes = [P, P, Lg, P, P, I, I, I, I, I, I, I, I, F, P, P, P]
     for name in ("ic_device_status", "ic_quant_e4m3_rows", "ic_indexer_scores", "ic_topk",
                  "ic_sparse_attn", "ic_layer_stack", "ic_decode_step", "ic_sparse_attn_noalloc",
-                 "ic_layer_stack_rows"):
+                 "ic_layer_stack_rows", "ic_layer_stack_varlen"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -303,6 +306,18 @@ def ic_layer_stack_rows(pattern: str, desc: ic_stack_desc, layers: list[dict], r
     _check(lib().ic_layer_stack_rows(pattern.encode(), ctypes.byref(desc), arr, len(layers),
                                      int(row0), int(rows), _p(t_cache), _p(workspace), ws_bytes,
                                      _stream(stream)))
+
+
+def ic_layer_stack_varlen(pattern: str, desc: ic_stack_desc, layers: list[dict], cu_seqlens,
+                          t_cache, workspace, stream=None):
+    """Prefill stack over sequences packed along the row axis; cu_seqlens = [0, L_0,
+    L_0 + L_1, ...] (host ints).  Every layer tensor holds the packed rows."""
+    cu = (ctypes.c_long * len(cu_seqlens))(*[int(x) for x in cu_seqlens])
+    arr = _layers(layers)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().ic_layer_stack_varlen(pattern.encode(), ctypes.byref(desc), arr, len(layers), cu,
+                                       len(cu_seqlens) - 1, _p(t_cache), _p(workspace), ws_bytes,
+                                       _stream(stream)))
 
 
 def ic_decode_step(pattern: str, desc: ic_stack_desc, layers: list[dict], t_cache, workspace,

@@ -390,6 +390,56 @@ ic_status ic_layer_stack_rows(const char* pattern, const ic_stack_desc* desc,
                    row0, rows);
 }
 
+ic_status ic_layer_stack_varlen(const char* pattern, const ic_stack_desc* desc,
+                                const ic_layer_io* layers, int nlayers, const long* cu_seqlens,
+                                int nseq, int* t_cache, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  if (!desc) return fail(IC_ERR_INVALID_ARG, "stack: desc is NULL");
+  if (!cu_seqlens || nseq < 0) return fail(IC_ERR_INVALID_ARG, "varlen: bad cu_seqlens / nseq");
+  if (cu_seqlens[0] != 0) return fail(IC_ERR_INVALID_ARG, "varlen: cu_seqlens[0] must be 0");
+  for (int i = 0; i < nseq; ++i)
+    if (cu_seqlens[i + 1] < cu_seqlens[i] || cu_seqlens[i + 1] - cu_seqlens[i] > desc->L)
+      return fail(IC_ERR_INVALID_ARG,
+                  "varlen: sequence %d has %ld tokens (must be 0..desc->L = %d)", i,
+                  cu_seqlens[i + 1] - cu_seqlens[i], desc->L);
+  if (nlayers < 1 || nlayers > 4096 || !layers)
+    return fail(IC_ERR_INVALID_ARG, "varlen: bad layers / nlayers");
+  const size_t qrow_b = static_cast<size_t>(desc->H) * desc->D * elem_bytes(desc->idx_dtype);
+  const size_t krow_b = static_cast<size_t>(desc->D) * elem_bytes(desc->idx_dtype);
+  const size_t arow_b = static_cast<size_t>(desc->heads) * desc->dk * elem_bytes(desc->attn_dtype);
+  const size_t kvrow_b = static_cast<size_t>(desc->ld_kv) * elem_bytes(desc->attn_dtype);
+  const size_t vrow_b = static_cast<size_t>(desc->dv) * elem_bytes(desc->attn_dtype);
+  const size_t orow_b = static_cast<size_t>(desc->heads) * desc->dv * elem_bytes(desc->attn_dtype);
+  std::vector<ic_layer_io> sub(nlayers);
+  for (int i = 0; i < nseq; ++i) {
+    const long o = cu_seqlens[i], n = cu_seqlens[i + 1] - cu_seqlens[i];
+    if (n == 0) continue;
+    ic_stack_desc d = *desc;
+    d.L = static_cast<int>(n);
+    auto at = [o](const void* p, size_t row_b) -> void* {
+      return p ? const_cast<uint8_t*>(static_cast<const uint8_t*>(p)) + o * row_b : nullptr;
+    };
+    for (int l = 0; l < nlayers; ++l) {
+      const ic_layer_io& io = layers[l];
+      ic_layer_io& e = sub[l];
+      e.q_idx = at(io.q_idx, qrow_b);
+      e.q_scale = static_cast<const float*>(at(io.q_scale, desc->H * sizeof(float)));
+      e.k_idx = at(io.k_idx, krow_b);
+      e.k_scale = static_cast<const float*>(at(io.k_scale, sizeof(float)));
+      e.w = static_cast<const float*>(at(io.w, desc->H * sizeof(float)));
+      e.q = at(io.q, arow_b);
+      e.kv = at(io.kv, kvrow_b);
+      e.v = at(io.v, vrow_b);
+      e.out = at(io.out, orow_b);
+      e.lse = static_cast<float*>(at(io.lse, desc->heads * sizeof(float)));
+    }
+    ic_status st = run_stack(pattern, &d, sub.data(), nlayers, t_cache + o * desc->k, workspace,
+                             ws_bytes, stream, false);
+    if (st) return fail(st, "varlen: sequence %d: %s", i, ic_last_error());
+  }
+  return IC_OK;
+}
+
 ic_status ic_decode_step(const char* pattern, const ic_stack_desc* desc, const ic_layer_io* layers,
                          int nlayers, int* t_cache, void* workspace, size_t ws_bytes,
                          void* stream) {

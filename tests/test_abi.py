@@ -111,3 +111,14 @@ def test_row_range_stack_rejects_rows_outside_the_sequence(lib):
     assert lib.ic_layer_stack_rows(b"F", ctypes.byref(desc), arr, 1, 4, 8, None, None, 0,
                                    None) == binding.IC_ERR_INVALID_ARG
     assert "NULL" in binding.ic_last_error()
+
+
+def test_varlen_stack_rejects_bad_sequence_offsets(lib):
+    desc = binding.make_desc(L=16, k=4, H=4, D=32, idx_dtype=binding.IC_F32, heads=4, dk=64, dv=64,
+                             attn_dtype=binding.IC_F32, scale=0.125)
+    arr = (binding.ic_layer_io * 1)()
+    for cu in ([1, 4], [0, 8, 4], [0, 17]):
+        c = (ctypes.c_long * len(cu))(*cu)
+        assert lib.ic_layer_stack_varlen(b"F", ctypes.byref(desc), arr, 1, c, len(cu) - 1, None,
+                                         None, 0, None) == binding.IC_ERR_INVALID_ARG
+        assert "varlen" in binding.ic_last_error()

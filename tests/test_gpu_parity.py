@@ -392,6 +392,54 @@ def test_stack_rows_zigzag_pieces_equal_the_whole_stack():
     assert seen == wl.L
 
 
+def test_stack_varlen_batch_matches_the_oracle_per_sequence():
+    """Sequences of 300, 0, 517 and 64 tokens packed along the rows (fp32 config):
+    each one's index set and outputs match the oracle's stack on that sequence alone."""
+    lens = [300, 0, 517, 64]
+    pattern = "F,S,S"
+    seqs = [synth.variant("tiny_stack", L=max(n, 1), pattern=pattern) for n in lens]
+    per = []
+    for i, (wl, n) in enumerate(zip(seqs, lens)):
+        lay = []
+        for l in range(wl.layers):
+            d = synth.indexer_inputs(wl, l, seed=i)
+            d.update(synth.attn_inputs(wl, l, seed=i))
+            lay.append({k: v[:n] for k, v in d.items()})
+        per.append(lay)
+    wl0 = seqs[0]
+    packed = []
+    for l in range(wl0.layers):
+        e = {k: torch.cat([p[l][k] for p in per]).to(DEV) for k in per[0][l]}
+        tot = sum(lens)
+        e["out"] = torch.empty(tot, wl0.Hq, wl0.Dv, device=DEV)
+        e["lse"] = torch.empty(tot, wl0.Hq, device=DEV)
+        packed.append(e)
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    desc = ic.make_desc(L=max(lens), k=wl0.k, H=wl0.H, D=wl0.D, idx_dtype=ic.IC_F32,
+                        heads=wl0.Hq, dk=wl0.Dk, dv=wl0.Dv, attn_dtype=ic.IC_F32, scale=wl0.scale)
+    ws = torch.empty(ic.ic_stack_workspace_size(desc) // 4 + 1, device=DEV)
+    t = torch.full((sum(lens), wl0.k), -7, dtype=torch.int32, device=DEV)
+    ic.ic_layer_stack_varlen(pattern, desc, packed, cu, t, ws)
+    _sync()
+    T = t.cpu().numpy()
+    for i, n in enumerate(lens):
+        if n == 0:
+            continue
+        lay = [{k: v.numpy() for k, v in d.items()} for d in per[i]]
+        ref = oracle.layer_stack(pattern, lay, wl0.k, wl0.scale, keep_scores=True)
+        o0, o1 = cu[i], cu[i + 1]
+        Ti = T[o0:o1]
+        diffs = sum(check_index_row(Ti[r], ref[0]["scores"][r], wl0.k, r + 1, atol=1e-5,
+                                    rtol=1e-5) for r in range(n))
+        assert diffs <= max(1, n // 20)
+        for l in range(wl0.layers):
+            ro, rl = oracle.sparse_attn(lay[l]["q"], lay[l]["kv"], Ti, wl0.scale, v=lay[l]["v"])
+            np.testing.assert_allclose(packed[l]["out"][o0:o1].cpu().numpy(), ro, atol=1e-5,
+                                       rtol=1e-4)
+            np.testing.assert_allclose(packed[l]["lse"][o0:o1].cpu().numpy(), rl, atol=1e-5,
+                                       rtol=1e-5)
+
+
 def test_decode_step_parity():
     """Decode: 6 sequences x 1 token over a 3000-token context, fp8 indexer cache,
     pattern F,S: T per sequence and both layers' outputs against the oracle."""
