@@ -397,16 +397,23 @@ def run_decode(args, dev, peaks, barrier):
             step(pat)
         ic.ic_device_status(stream)
         barrier()
+        # the step time without tracing: an event between launches costs a few
+        # microseconds each and stops consecutive kernels from overlapping
+        ms = _timed(lambda: step(pat), steps, stream)
+        ic.ic_device_status(stream)
+        # then a traced pass of the same steps for the per-stage split (its
+        # stage times add up to the traced step, slightly longer than `ms`)
         cap = 64 * steps
         ic.ic_trace_begin(cap, stream=stream)
-        ms = _timed(lambda: step(pat), steps, stream)
+        ms_traced = _timed(lambda: step(pat), steps, stream)
         n_launch, trace = ic.ic_trace_end(cap)
         ic.ic_device_status(stream)
         hb = bytes_of(pat)
         gbs = hb / (ms * 1e-3) / 1e9
         r = {"pattern": pat, "ms_per_step": ms, "value": B / (ms * 1e-3), "unit": "tokens/s",
              "hbm_bytes_per_step": hb, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
-             "frac_hbm": gbs / peaks["hbm_gbs"], "gpu_launches_per_step": n_launch / steps}
+             "frac_hbm": gbs / peaks["hbm_gbs"], "gpu_launches_per_step": n_launch / steps,
+             "ms_per_step_traced": ms_traced}
         if key is None:
             agg = {}
             for name, kms, work in trace:

@@ -531,6 +531,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const AttnArgs 
     z[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   __syncthreads();
+  grid_dep_wait();  // set-up above touches no global memory
   if (threadIdx.x >= AT_CONSUMERS)
     attn_producer(sm, a);
   else
@@ -544,6 +545,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const AttnArgs 
 // with shuffles; then every thread accumulates its output dims over the pieces.
 __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, int maxp, long tot,
                                     int tq, int G, __nv_bfloat16* out, float* lse) {
+  grid_dep_wait();
   const long qrow = blockIdx.x;
   const int h = blockIdx.y;
   const long c0 = attn_cta_of(qrow * tq, tot, G);
@@ -660,8 +662,9 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
       "cudaFuncSetAttribute(attn)");
   if (st) return st;
   const long grid = p.split ? p.G : (items < num_sms() ? items : num_sms());
-  attn_mla_kernel<<<static_cast<unsigned>(grid), AT_THREADS, smem, stream>>>(a);
-  st = cuda_check(cudaGetLastError(), "attn_mla_kernel launch");
+  st = cuda_check(launch_dep(attn_mla_kernel, dim3(static_cast<unsigned>(grid)), dim3(AT_THREADS),
+                             smem, stream, 1, a),
+                  "attn_mla_kernel launch");
   if (st) return st;
   // algorithmic bytes: each selected latent row gathered once, q read once, out written once
   const double ve = valid_entries >= 0 ? static_cast<double>(valid_entries)
@@ -669,9 +672,9 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
   const double io = static_cast<double>(items) * AT_H * (AT_DK + AT_DV) * 2.0;
   trace_launch(kKindAttnMla, stream, ve * AT_DK * 2.0 + io + 4.0 * static_cast<double>(items) * k);
   if (!p.split) return IC_OK;
-  attn_combine_kernel<<<dim3(static_cast<unsigned>(items), AT_H), 128, 0, stream>>>(
-      a.part_o, a.part_ml, p.maxp, p.tot, p.tq, p.G, a.out, lse);
-  st = cuda_check(cudaGetLastError(), "attn_combine_kernel launch");
+  st = cuda_check(launch_dep(attn_combine_kernel, dim3(static_cast<unsigned>(items), AT_H), dim3(128),
+                             0, stream, 1, a.part_o, a.part_ml, p.maxp, p.tot, p.tq, p.G, a.out, lse),
+                  "attn_combine_kernel launch");
   if (!st) {
     // pieces actually written: every (query, CTA) overlap
     const double pieces = static_cast<double>(p.G) + static_cast<double>(items) - 1.0;

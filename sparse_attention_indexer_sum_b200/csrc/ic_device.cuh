@@ -45,6 +45,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ------------------------------------------------------------------ dependent launch
+// The library launches its kernels with programmatic stream serialization: a
+// kernel may be scheduled while the previous kernel of its stream still runs, so
+// its launch and set-up (barriers, TMEM) overlap the other's tail.
+// grid_dep_wait() returns once every earlier grid of the stream has completed and
+// its writes are visible (at once for a kernel launched without the attribute).
+// Every thread of every kernel calls it, on every path, before its first access
+// to global memory; a grid therefore completes only after its predecessor did.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// No kernel here signals its dependents early (griddepcontrol.launch_dependents):
+// the next grid is scheduled as this grid's CTAs exit.  An early signal at kernel
+// start measured no faster on the decode step.
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

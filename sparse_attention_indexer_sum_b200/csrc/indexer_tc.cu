@@ -202,6 +202,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_wait();  // set-up above touches no global memory
 
   if (nitems > 0) {
     if (warp == 0) {
@@ -411,6 +412,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
 // Writes -inf on the masked keys [pos0 + r + 1, Lk) of every row (the tensor-core
 // kernel only visits key tiles up to its query block's diagonal).  One CTA per row.
 __global__ void fill_masked_kernel(float* scores, long ld, int R, int Lk, long pos0) {
+  grid_dep_wait();
   const long row = blockIdx.x;  // b * R + r
   const long r = row % R;
   for (long s = pos0 + r + 1 + threadIdx.x; s < Lk; s += blockDim.x) scores[row * ld + s] = -INFINITY;
@@ -492,9 +494,9 @@ static ic_status launch_tpl(const void* q, const float* q_scale, const void* k,
                   "cudaFuncSetAttribute(indexer)");
   if (st) return st;
   const long grid = total < num_sms() ? total : num_sms();
-  indexer_tc_kernel<FP8, TPM><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
-      tmK, tmQ, a);
-  st = cuda_check(cudaGetLastError(), "indexer_tc_kernel launch");
+  st = cuda_check(launch_dep(indexer_tc_kernel<FP8, TPM>, dim3(static_cast<unsigned>(grid)),
+                             dim3(C::THREADS), C::SMEM_BYTES, stream, 1, tmK, tmQ, a),
+                  "indexer_tc_kernel launch");
   if (st) return st;
   trace_launch(FP8 ? kKindIndexerE4m3 : kKindIndexerBf16, stream,
                2.0 * 64 * 128 * static_cast<double>(causal_pairs(rows, Lk, pos0)) * batch);
@@ -519,9 +521,9 @@ ic_status launch_indexer_tc(bool fp8, const void* q, const float* q_scale, const
                                       ld, stream);
   if (st || !fill_tail) return st;
   if (pos0 + 1 < Lk) {  // some row has masked keys
-    fill_masked_kernel<<<static_cast<unsigned>(static_cast<long>(batch) * rows), 256, 0, stream>>>(
-        scores, ld, rows, Lk, pos0);
-    st = cuda_check(cudaGetLastError(), "fill_masked_kernel launch");
+    st = cuda_check(launch_dep(fill_masked_kernel, dim3(static_cast<unsigned>(static_cast<long>(batch) * rows)),
+                               dim3(256), 0, stream, 1, scores, ld, rows, Lk, pos0),
+                    "fill_masked_kernel launch");
     if (!st)
       trace_launch(kKindFillMasked, stream,
                    4.0 * (static_cast<double>(rows) * Lk - causal_pairs(rows, Lk, pos0)) * batch);

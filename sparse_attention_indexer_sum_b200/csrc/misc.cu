@@ -14,6 +14,7 @@ namespace ic {
 template <typename T>
 __global__ void quant_e4m3_kernel(const T* __restrict__ x, long rows, int n,
                                   uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  grid_dep_wait();
   const long row = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -40,13 +41,12 @@ ic_status launch_quant_e4m3(const void* x, bool bf16, long rows, int n, uint8_t*
                             float* scales, cudaStream_t stream) {
   if (rows == 0) return IC_OK;
   const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
-  if (bf16)
-    quant_e4m3_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), rows, n, codes, scales);
-  else
-    quant_e4m3_kernel<float><<<blocks, 256, 0, stream>>>(static_cast<const float*>(x), rows, n,
-                                                         codes, scales);
-  ic_status st = cuda_check(cudaGetLastError(), "quant_e4m3_kernel launch");
+  const cudaError_t e =
+      bf16 ? launch_dep(quant_e4m3_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, stream, 1,
+                        static_cast<const __nv_bfloat16*>(x), rows, n, codes, scales)
+           : launch_dep(quant_e4m3_kernel<float>, dim3(blocks), dim3(256), 0, stream, 1,
+                        static_cast<const float*>(x), rows, n, codes, scales);
+  ic_status st = cuda_check(e, "quant_e4m3_kernel launch");
   if (!st)
     trace_launch(kKindQuant, stream,
                  static_cast<double>(rows) * (n * ((bf16 ? 2.0 : 4.0) + 1.0) + 4.0));

@@ -416,6 +416,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
   extern __shared__ uint8_t tk_smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
   const int tid = threadIdx.x;
+  grid_dep_wait();
   // A row is split over the S CTAs of a cluster (S = 1 without clusters): each
   // collects the candidates of its part, CTA 0 merges them and selects.
   const uint32_t S = cluster_nctarank(), crank = cluster_ctarank();
@@ -582,26 +583,9 @@ ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0,
     const long slots = 2L * num_sms();
     while (S < 8 && rows * 2 * S <= slots) S *= 2;
   }
-  if (S == 1) {
-    topk_kernel<<<static_cast<unsigned>(rows), TK_THREADS, smem, stream>>>(scores, ld, n, pos0, k,
-                                                                           idx);
-    st = cuda_check(cudaGetLastError(), "topk_kernel launch");
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(rows * S));
-    cfg.blockDim = dim3(TK_THREADS);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = S;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    st = cuda_check(cudaLaunchKernelEx(&cfg, topk_kernel, scores, ld, n, pos0, k, idx),
-                    "topk_kernel cluster launch");
-  }
+  st = cuda_check(launch_dep(topk_kernel, dim3(static_cast<unsigned>(rows * S)), dim3(TK_THREADS),
+                             smem, stream, static_cast<unsigned>(S), scores, ld, n, pos0, k, idx),
+                  "topk_kernel launch");
   if (st) return st;
   // algorithmic bytes: every candidate score read once, the index rows written once
   const double cand = pos0 < 0 ? static_cast<double>(rows) * n
