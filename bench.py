@@ -399,8 +399,24 @@ def run_decode(args, dev, peaks, barrier):
         barrier()
         # the step time without tracing: an event between launches costs a few
         # microseconds each and stops consecutive kernels from overlapping
-        ms = _timed(lambda: step(pat), steps, stream)
+        ms_eager = _timed(lambda: step(pat), steps, stream)
         ic.ic_device_status(stream)
+        # the same step captured once in a CUDA graph and replayed, as a serving
+        # loop runs it (one host launch per step)
+        graph = ic.decode_step_graph(pat, desc, layers, t_cache, ws)
+        for _ in range(3):
+            graph.replay()
+        ic.ic_device_status(stream)
+        # long enough (~0.5 s) for the 200 ms clock samples to see it
+        n_graph = max(steps, int(500.0 / max(ms_eager, 1e-3)))
+        clocks = ClockSampler("GPU-%s" % torch.cuda.get_device_properties(dev).uuid)
+        clocks.start()
+        time.sleep(0.5)
+        clocks.mark()
+        ms = _timed(graph.replay, n_graph, stream)
+        clk = clocks.stop()
+        ic.ic_device_status(stream)
+        del graph
         # then a traced pass of the same steps for the per-stage split (its
         # stage times add up to the traced step, slightly longer than `ms`)
         cap = 64 * steps
@@ -413,6 +429,8 @@ def run_decode(args, dev, peaks, barrier):
         r = {"pattern": pat, "ms_per_step": ms, "value": B / (ms * 1e-3), "unit": "tokens/s",
              "hbm_bytes_per_step": hb, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
              "frac_hbm": gbs / peaks["hbm_gbs"], "gpu_launches_per_step": n_launch / steps,
+             "timing": "CUDA graph replay of the step, %d steps" % n_graph,
+             "clocks": clk, "ms_per_step_eager": ms_eager,
              "ms_per_step_traced": ms_traced}
         if key is None:
             agg = {}

@@ -327,3 +327,26 @@ def ic_decode_step(pattern: str, desc: ic_stack_desc, layers: list[dict], t_cach
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib().ic_decode_step(pattern.encode(), ctypes.byref(desc), arr, len(layers),
                                 _p(t_cache), _p(workspace), ws_bytes, _stream(stream)))
+
+
+def decode_step_graph(pattern: str, desc: ic_stack_desc, layers: list[dict], t_cache, workspace,
+                      warmup: int = 1) -> torch.cuda.CUDAGraph:
+    """One ic_decode_step captured into a CUDA graph over these buffers.
+
+    ``graph.replay()`` reruns the whole step (its kernels and the programmatic
+    launch edges between them) with one launch from the host, on the current
+    stream.  Every replay reads the same input tensors and writes the same
+    outputs: a caller updates the inputs in place between replays.  The step
+    allocates nothing, so the graph holds no memory of its own."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(warmup):  # first-call set-up (kernel attributes) outside the capture
+            ic_decode_step(pattern, desc, layers, t_cache, workspace, stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    # relaxed: the step's per-launch host calls (kernel attributes, device queries)
+    # are not stream work and need not be refused while capturing
+    with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+        ic_decode_step(pattern, desc, layers, t_cache, workspace)
+    return graph

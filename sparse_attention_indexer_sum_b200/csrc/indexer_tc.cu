@@ -73,7 +73,13 @@ struct IdxCfg {
   static constexpr int SETW = 4 * EPG;             // warps per set
   static constexpr int NEPI = SETW * NSETS;
   static constexpr int TOK_PER_EW = TPM / EPG;     // tokens per epilogue warp
-  static constexpr int THREADS = 64 + 32 * NEPI;
+  // MMA-issuing warps: tile i is issued by warp 1 + i % MMAW.  With N = 64
+  // (one-token blocks) a tile's four or eight MMAs are short, and one thread's
+  // issue loop (waits, MMAs, commits) sets the pace; two threads alternate
+  // tiles.  With N = 256 the tensor pipe itself is the limit.
+  static constexpr int MMAW = (TPM == 1) ? 2 : 1;
+  static constexpr int EPI_W0 = 1 + MMAW;  // first epilogue warp
+  static constexpr int THREADS = 32 * (EPI_W0 + NEPI);
   // TMEM columns an epilogue thread loads at a time: 16, so that the head
   // weights of both its tokens fit in registers beside them
   static constexpr int EPI_COLS = 16;  // matches tmem_ld16
@@ -161,8 +167,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
         mbar_init(accempty_bar(i), C::SETW);
       }
       mbar_init(qfull_bar, 1);
-      mbar_init(qempty_bar, 1);
-      mbar_init(mmadone_bar, 1);
+      mbar_init(qempty_bar, C::MMAW);
+      mbar_init(mmadone_bar, C::MMAW);
       *abort_flag = 0;
       fence_barrier_init();
       fence_proxy_async_smem();
@@ -251,11 +257,21 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
           if (qloads > 0) mbar_wait_drain(qfull_bar, (qloads - 1) & 1);
         }
       }
-    } else if (warp == 1) {
-      // ------------------------------------------------------------ MMA issuer
+    } else if (warp < C::EPI_W0) {
+      // ------------------------------------------------------------ MMA issuer(s)
       if (lane == 0) {
+        const int mw = warp - 1;
         constexpr uint32_t fmt = FP8 ? 0u : 1u;  // e4m3 : bf16
         constexpr uint32_t idesc = idesc_f32acc(fmt, fmt, C::BM, C::N);
+        // Descriptors, built once: one per K step of the resident query block,
+        // and the key ring's base (a K step or stage offset adds its address >> 4
+        // to the start-address field, which cannot carry out: every shared
+        // address is below 256 KB).
+        uint64_t bdesc[C::KSTEPS];
+#pragma unroll
+        for (int kk = 0; kk < C::KSTEPS; ++kk)
+          bdesc[kk] = sdesc_k_sw128(q_base + (kk / 4) * (C::N * 128) + (kk % 4) * 32);
+        const uint64_t adesc0 = sdesc_k_sw128(a_base);
         WorkIt<TPM> it{start[0], start[1], qb_tiles<TPM>(a, start[0])};
         int stage = 0, acc = 0;
         uint32_t ph = 0, aph = 0;
@@ -266,23 +282,23 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
             ++qwaits;
             cur_qb = it.qb;
           }
-          if (!mbar_wait(accempty_bar(acc), aph ^ 1, abort_flag, kErrTimeoutMma)) break;
-          if (!mbar_wait(full_bar(stage), ph, abort_flag, kErrTimeoutMma)) break;
-          tc_fence_after();
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::N);
-          const uint32_t a_st = a_base + stage * C::A_BYTES;
+          if (C::MMAW == 1 || i % C::MMAW == mw) {
+            if (!mbar_wait(accempty_bar(acc), aph ^ 1, abort_flag, kErrTimeoutMma)) break;
+            if (!mbar_wait(full_bar(stage), ph, abort_flag, kErrTimeoutMma)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::N);
+            const uint64_t a_st = adesc0 + static_cast<uint64_t>(stage * (C::A_BYTES >> 4));
 #pragma unroll
-          for (int kk = 0; kk < C::KSTEPS; ++kk) {
-            const uint32_t kblk = kk / 4, koff = (kk % 4) * 32;
-            const uint64_t adesc = sdesc_k_sw128(a_st + kblk * (C::BM * 128) + koff);
-            const uint64_t bdesc = sdesc_k_sw128(q_base + kblk * (C::N * 128) + koff);
-            if constexpr (FP8)
-              tc_mma_f8(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
-            else
-              tc_mma_f16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < C::KSTEPS; ++kk) {
+              const uint64_t adesc = a_st + (((kk / 4) * (C::BM * 128) + (kk % 4) * 32) >> 4);
+              if constexpr (FP8)
+                tc_mma_f8(d_tmem, adesc, bdesc[kk], idesc, kk > 0 ? 1u : 0u);
+              else
+                tc_mma_f16(d_tmem, adesc, bdesc[kk], idesc, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(empty_bar(stage));
+            tc_commit(accfull_bar(acc));
           }
-          tc_commit(empty_bar(stage));
-          tc_commit(accfull_bar(acc));
           WorkIt<TPM> nx = it;
           nx.advance(a);
           if (i + 1 == nitems || nx.qb != it.qb) tc_commit(qempty_bar);
@@ -302,7 +318,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
       }
     } else {
       // ------------------------------------------------------------ epilogue
-      const int e = warp - 2;
+      const int e = warp - C::EPI_W0;
       const int qd = warp & 3;     // TMEM lane quadrant this warp may access
       const int set = e / C::SETW;  // accumulator slots a with a % NSETS == set
       const int member = (e % C::SETW) / 4;  // which tokens of the block this warp reduces

@@ -463,6 +463,47 @@ def test_decode_step_parity():
         assert_attn_close(_np(dl[l]["out"]), ro)
 
 
+def test_decode_step_graph_replay_matches_eager():
+    """The decode step captured in a CUDA graph (programmatic launch edges
+    included) and replayed gives bit-identical T and outputs to eager calls, also
+    after its inputs change in place."""
+    wl = synth.variant("decode_200k", L=5000, batch=5, pattern="F,S,S")
+    layers, _ = _stack_layers(wl, DEV)
+    for d in layers:
+        d["q_idx"], d["q_scale"] = ic.ic_quant_e4m3_rows(d["q_idx"])
+        d["k_idx"], d["k_scale"] = ic.ic_quant_e4m3_rows(d["k_idx"])
+    dl, t_eager = _run_stack(wl, wl.pattern, layers, ic.IC_E4M3, decode=True)
+    out_eager = [d["out"].clone() for d in dl]
+    desc = _desc(wl, ic.IC_E4M3)
+    ws = torch.empty(ic.ic_stack_workspace_size(desc) // 4 + 1, device=DEV)
+    t_cache = torch.full_like(t_eager, -7)
+    for d in dl:
+        d["out"].zero_()
+    g = ic.decode_step_graph(wl.pattern, desc, dl, t_cache, ws, warmup=0)
+    g.replay()
+    _sync()
+    assert torch.equal(t_cache, t_eager)
+    for d, o in zip(dl, out_eager):
+        assert torch.equal(d["out"], o)
+    # new queries written in place: the replay follows them like an eager call
+    for d in dl:
+        d["q"].copy_(torch.flip(d["q"], dims=[0]))
+        d["q_idx"].copy_(torch.flip(d["q_idx"], dims=[0]))
+        d["q_scale"].copy_(torch.flip(d["q_scale"], dims=[0]))
+        d["w"].copy_(torch.flip(d["w"], dims=[0]))
+    g.replay()
+    _sync()
+    t_graph = t_cache.clone()
+    out_graph = [d["out"].clone() for d in dl]
+    ic.ic_decode_step(wl.pattern, desc, dl, t_cache, ws)
+    _sync()
+    assert torch.equal(t_cache, t_graph)
+    for d, o in zip(dl, out_graph):
+        assert torch.equal(d["out"], o)
+    assert not torch.equal(t_graph, t_eager)
+    del g
+
+
 def test_trace_records_every_launch_in_order():
     q, k, w = _idx_inputs(1, 8, 300, seed=3)
     q, k, w = q.to(DEV), k.to(DEV), w.to(DEV)
