@@ -153,8 +153,9 @@ ic_status ic_topk(const float* scores, long rows, int n, long ld, long pos0, int
  * workspace (device, may be NULL): with IC_BF16 and fewer than 4 queries per SM,
  * the (query, 32-key tile) pairs are cut into one equal contiguous range per SM,
  * and the partial results of each query's pieces go through the workspace (see
- * ic_attn_workspace_size) to a merge kernel; with too little workspace there is
- * no split (one CTA per query), never an error.
+ * ic_attn_workspace_size) to a merge kernel; with too little workspace, or a
+ * workspace that is not 16-byte aligned, there is no split (one CTA per query),
+ * never an error.
  */
 ic_status ic_sparse_attn(const void* q, const void* kv, long ld_kv, const void* v, const int* idx,
                          ic_dtype dt, int batch, int rows, int heads, int dk, int dv, int Lkv,

@@ -553,6 +553,17 @@ __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, i
   const long s0 = qrow * maxp;
   __shared__ float wsh[64];
   __shared__ float inv_l;
+  // Each thread owns 4 adjacent output dims.  The first CMB_PRE pieces' partial
+  // outputs are loaded before the weights are known, so their latency overlaps
+  // the (m, l) reduction; later pieces (rare) are loaded as they are used.
+  constexpr int CMB_PRE = 8;
+  const float* po = part_o + (s0 * AT_H + h) * AT_DV;
+  const long pstride = static_cast<long>(AT_H) * AT_DV;
+  const int d = 4 * threadIdx.x;
+  float4 pv[CMB_PRE];
+#pragma unroll
+  for (int i = 0; i < CMB_PRE; ++i)
+    if (i < np) pv[i] = *reinterpret_cast<const float4*>(po + i * pstride + d);
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -580,18 +591,23 @@ __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, i
     }
   }
   __syncthreads();
-  const float* po = part_o + (s0 * AT_H + h) * AT_DV;
-  const long pstride = static_cast<long>(AT_H) * AT_DV;
-  for (int d = threadIdx.x; d < AT_DV; d += blockDim.x) {
-    float a0 = 0.f, a1 = 0.f;
-    int i = 0;
-    for (; i + 1 < np; i += 2) {  // two independent loads in flight per step
-      a0 += wsh[i] * po[i * pstride + d];
-      a1 += wsh[i + 1] * po[(i + 1) * pstride + d];
-    }
-    if (i < np) a0 += wsh[i] * po[i * pstride + d];
-    out[(qrow * AT_H + h) * AT_DV + d] = __float2bfloat16_rn((a0 + a1) * inv_l);
-  }
+  // even pieces accumulate into a0, odd ones into a1
+  float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+  auto madd = [](float4& acc, float w, const float4& u) {
+    acc.x += w * u.x;
+    acc.y += w * u.y;
+    acc.z += w * u.z;
+    acc.w += w * u.w;
+  };
+#pragma unroll
+  for (int i = 0; i < CMB_PRE; ++i)
+    if (i < np) madd((i & 1) ? a1 : a0, wsh[i], pv[i]);
+  for (int i = CMB_PRE; i < np; ++i)
+    madd((i & 1) ? a1 : a0, wsh[i], *reinterpret_cast<const float4*>(po + i * pstride + d));
+  const float il = inv_l;
+  uint32_t* o = reinterpret_cast<uint32_t*>(out + (qrow * AT_H + h) * AT_DV + d);
+  o[0] = pack_bf16((a0.x + a1.x) * il, (a0.y + a1.y) * il);
+  o[1] = pack_bf16((a0.z + a1.z) * il, (a0.w + a1.w) * il);
 }
 
 // Split plan for few queries: G CTAs over the items*tq (query, tile) pairs, each
@@ -635,7 +651,9 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
   if (items == 0) return IC_OK;
   SplitPlan p = split_plan(items, k);
   const size_t need = static_cast<size_t>(items) * p.maxp * AT_H * (AT_DV + 2) * sizeof(float);
-  if (p.split && (ws == nullptr || need > ws_bytes)) p.split = false;  // no room: one CTA per query
+  // no room, or a workspace the merge's 16-byte loads cannot use: one CTA per query
+  if (p.split && (ws == nullptr || need > ws_bytes || reinterpret_cast<uintptr_t>(ws) % 16 != 0))
+    p.split = false;
   AttnArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.kv = static_cast<const __nv_bfloat16*>(kv);
@@ -672,6 +690,7 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
   const double io = static_cast<double>(items) * AT_H * (AT_DK + AT_DV) * 2.0;
   trace_launch(kKindAttnMla, stream, ve * AT_DK * 2.0 + io + 4.0 * static_cast<double>(items) * k);
   if (!p.split) return IC_OK;
+  static_assert(AT_DV == 4 * 128, "combine: 128 threads x 4 dims");
   st = cuda_check(launch_dep(attn_combine_kernel, dim3(static_cast<unsigned>(items), AT_H), dim3(128),
                              0, stream, 1, a.part_o, a.part_ml, p.maxp, p.tot, p.tq, p.G, a.out, lse),
                   "attn_combine_kernel launch");

@@ -455,11 +455,19 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
   } else {
     m = TK_SAMPLE;
     const int run = TK_SAMPLE / 32;  // 128
-    for (int i = tid; i < TK_SAMPLE; i += TK_THREADS) {
+    // every thread's loads go out before any is used
+    constexpr int SPT = TK_SAMPLE / TK_THREADS;
+    static_assert(TK_SAMPLE % TK_THREADS == 0, "whole sample loads per thread");
+    float sv[SPT];
+#pragma unroll
+    for (int u = 0; u < SPT; ++u) {
+      const int i = tid + u * TK_THREADS;
       const int b = i / run, o = i % run;
       const int start = static_cast<int>((static_cast<long>(b) * (nv - run)) / 31) & ~3;
-      samp[i] = score_key(__ldg(x + start + o));
+      sv[u] = __ldg(x + start + o);
     }
+#pragma unroll
+    for (int u = 0; u < SPT; ++u) samp[tid + u * TK_THREADS] = score_key(sv[u]);
     const long jj = (static_cast<long>(k) * 16 * m + 10L * nv - 1) / (10L * nv);
     j = static_cast<int>(jj < 1 ? 1 : (jj > m ? m : jj));
   }
