@@ -540,9 +540,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const AttnArgs 
 }
 
 // Merges the partial results of one query (its pieces in split mode): per head,
-// M = max m_i, L = sum l_i 2^(m_i - M), O = sum O_i 2^(m_i - M) / L.  Warp 0 reads
-// the pieces' (m, l) in parallel (lane i: pieces i and i + 32) and reduces them
-// with shuffles; then every thread accumulates its output dims over the pieces.
+// M = max m_i, L = sum l_i 2^(m_i - M), O = sum O_i 2^(m_i - M) / L.  Each warp
+// reads the pieces' (m, l) in parallel (lane i: pieces i and i + 32) and reduces
+// them with shuffles; every thread accumulates its output dims over the pieces.
 __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, int maxp, long tot,
                                     int tq, int G, __nv_bfloat16* out, float* lse) {
   grid_dep_wait();
@@ -551,8 +551,6 @@ __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, i
   const long c0 = attn_cta_of(qrow * tq, tot, G);
   const int np = static_cast<int>(attn_cta_of((qrow + 1) * tq - 1, tot, G) - c0 + 1);  // <= 64
   const long s0 = qrow * maxp;
-  __shared__ float wsh[64];
-  __shared__ float inv_l;
   // Each thread owns 4 adjacent output dims.  The first CMB_PRE pieces' partial
   // outputs are loaded before the weights are known, so their latency overlaps
   // the (m, l) reduction; later pieces (rare) are loaded as they are used.
@@ -564,8 +562,11 @@ __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, i
 #pragma unroll
   for (int i = 0; i < CMB_PRE; ++i)
     if (i < np) pv[i] = *reinterpret_cast<const float4*>(po + i * pstride + d);
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
+  // Every warp reduces the pieces' (m, l) itself (lane i: pieces i and i + 32), so
+  // no warp waits for another; the values are the same in every warp.
+  const int lane = threadIdx.x & 31;
+  float w0, w1, il;
+  {
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     if (lane < np) {
       m0 = part_ml[((s0 + lane) * AT_H + h) * 2];
@@ -578,19 +579,17 @@ __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, i
     float M = fmaxf(m0, m1);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float w0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M);
-    const float w1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M);
+    w0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M);
+    w1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M);
     float L = l0 * w0 + l1 * w1;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane < np) wsh[lane] = w0;
-    if (lane + 32 < np) wsh[lane + 32] = w1;
-    if (lane == 0) {
-      inv_l = L > 0.f ? 1.f / L : 0.f;
-      if (lse) lse[qrow * AT_H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
-    }
+    il = L > 0.f ? 1.f / L : 0.f;
+    if (threadIdx.x == 0 && lse)
+      lse[qrow * AT_H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
-  __syncthreads();
+  // weight of piece i (held by lane i % 32)
+  auto wt = [&](int i) { return __shfl_sync(0xffffffffu, i < 32 ? w0 : w1, i & 31); };
   // even pieces accumulate into a0, odd ones into a1
   float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
   auto madd = [](float4& acc, float w, const float4& u) {
@@ -601,10 +600,9 @@ __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, i
   };
 #pragma unroll
   for (int i = 0; i < CMB_PRE; ++i)
-    if (i < np) madd((i & 1) ? a1 : a0, wsh[i], pv[i]);
+    if (i < np) madd((i & 1) ? a1 : a0, wt(i), pv[i]);
   for (int i = CMB_PRE; i < np; ++i)
-    madd((i & 1) ? a1 : a0, wsh[i], *reinterpret_cast<const float4*>(po + i * pstride + d));
-  const float il = inv_l;
+    madd((i & 1) ? a1 : a0, wt(i), *reinterpret_cast<const float4*>(po + i * pstride + d));
   uint32_t* o = reinterpret_cast<uint32_t*>(out + (qrow * AT_H + h) * AT_DV + d);
   o[0] = pack_bf16((a0.x + a1.x) * il, (a0.y + a1.y) * il);
   o[1] = pack_bf16((a0.z + a1.z) * il, (a0.w + a1.w) * il);

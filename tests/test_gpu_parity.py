@@ -240,11 +240,15 @@ def test_attn_mla_decode_split_equals_unsplit():
     assert ws.numel() > 1
     o_split = ic.ic_sparse_attn(q, kv, idx, 0.05, workspace=ws)
     o_one = ic.ic_sparse_attn(q, kv, idx, 0.05)
+    # a workspace that is large enough but not 16-byte aligned: no split, exactly
+    # the result without a workspace
+    o_mis = ic.ic_sparse_attn(q, kv, idx, 0.05, workspace=ws[1:])
     _sync()
     ro, _ = oracle.sparse_attn(q.float().cpu().numpy(), kv.float().cpu().numpy(),
                                idx.cpu().numpy(), 0.05, dv=512)
     assert_attn_close(_np(o_split), ro)
     assert_attn_close(_np(o_one), ro)
+    assert torch.equal(o_mis, o_one)
 
 
 @pytest.mark.parametrize("B,R,k,Lkv", [(1, 1, 2048, 5000), (2, 1, 2048, 3000), (3, 1, 1000, 1200),
