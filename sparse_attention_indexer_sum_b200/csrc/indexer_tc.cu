@@ -17,8 +17,9 @@
 // Pipeline (one persistent CTA per SM, warp-specialised):
 //   warp 0      TMA producer: q block (once per query block) + a ring of key tiles
 //   warp 1      MMA issuer: one thread issues tcgen05.mma into a ring of TMEM
-//               accumulators, commits to mbarriers
-//   warps 2..   epilogue: tcgen05.ld -> ReLU -> w-weighted head sum -> causal
+//               accumulators, commits to mbarriers (one-token blocks: warps 1
+//               and 2, alternating key tiles)
+//   the rest    epilogue: tcgen05.ld -> ReLU -> w-weighted head sum -> causal
 //               mask -> fp32 score stores (coalesced, one key per lane)
 // The work is the list of (query block, key tile) pairs of the causal
 // triangle; CTA c takes the c-th equal share of that list, so every SM gets
