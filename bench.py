@@ -47,10 +47,10 @@ from sparse_attention_indexer_sum_b200 import synth  # noqa: E402
 METRIC = "prefill tokens/s (indexer+top-k+sparse attn) at L=200K; % of roofline"
 # DRAM bytes (read + write) per causal (query, key) pair of the bf16 tensor-core
 # indexer, from one ncu capture of the current kernel on 512 query rows at
-# position 100000 (`profile_cases indexer_longrows`: 202.5 MB for 51,331,328
+# position 100000 (`profile_cases indexer_longrows`: 203.9 MB for 51,331,328
 # pairs).  The score writes dominate and grow with the pairs; keys and queries
 # come from L2.  A launch's traffic is this figure times its pairs.
-INDEXER_BF16_DRAM_BYTES_PER_PAIR = 202.5e6 / 51331328
+INDEXER_BF16_DRAM_BYTES_PER_PAIR = 203.9e6 / 51331328
 UNIT = "tokens/s"
 
 
@@ -277,7 +277,7 @@ def run_ours(args, rank, world, local_rank):
                 "unit": "TFLOP/s", "frac": achieved / peak if peak else None, "traffic": traffic,
                 "traffic_source": None if fp8 else
                 "ncu dram__bytes_read.sum + dram__bytes_write.sum of the same kernel on 512 "
-                "rows at position 100000 (3.95 B per causal pair), times the pairs of a launch",
+                "rows at position 100000 (3.97 B per causal pair), times the pairs of a launch",
                 "peak_source": "%s bf16 sustained %.1f TFLOP/s%s" % (
                     peaks["source"], bf16_peak, " x2 (e4m3 nominal ratio)" if fp8 else ""),
                 "work_per_launch": d_work / d_n if d_n else None,
