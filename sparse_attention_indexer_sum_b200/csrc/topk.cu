@@ -329,13 +329,16 @@ __device__ __noinline__ void topk_exact(TopkSmem& sm, const float* __restrict__ 
 }
 
 // The j-th largest of `count` keys held in shared memory (count >= j >= 1), by
-// 12/12/8-bit histogram rounds over the keys.  With bits = 24 it stops after two
-// rounds and returns the lowest key of the j-th key's 24-bit bin (a lower bound:
-// at least j keys are >= it).
+// 12-bit histogram rounds over the keys (the last round takes the bits left).
+// With bits = 24 it stops after two rounds and returns the lowest key of the j-th
+// key's 24-bit bin (a lower bound: at least j keys are >= it).  common_bits > 0
+// says every key shares its top common_bits bits with `common`: the rounds start
+// below them.
 __device__ uint32_t select_kth_smem(TopkSmem& sm, const uint32_t* keys, int count, int j,
-                                    int bits_total = 32) {
-  uint32_t prefix = 0;
-  int pbits = 0;
+                                    int bits_total = 32, int common_bits = 0,
+                                    uint32_t common = 0u) {
+  int pbits = common_bits < bits_total ? common_bits : bits_total;
+  uint32_t prefix = pbits > 0 ? common >> (32 - pbits) : 0u;
   int need = j;
   while (pbits < bits_total) {
     const int bits = (32 - pbits) >= 12 ? 12 : (32 - pbits);
@@ -514,7 +517,19 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
   }
 
   // ---- 3. the exact k-th key T among the candidates
-  const uint32_t T = select_kth_smem(sm, sm.cand_key, C, k);
+  // every candidate lies in [tau, max]: their common leading bits need no round
+  uint32_t kmax = 0u;
+  for (int i = tid; i < C; i += TK_THREADS) kmax = max(kmax, sm.cand_key[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  if ((tid & 31) == 0) sm.scan_tmp[tid >> 5] = static_cast<int>(kmax);
+  __syncthreads();
+  kmax = 0u;
+#pragma unroll
+  for (int w = 0; w < TK_NW; ++w) kmax = max(kmax, static_cast<uint32_t>(sm.scan_tmp[w]));
+  __syncthreads();
+  const int cbits = __clz(static_cast<int>(tau ^ kmax));  // 32 when tau == kmax
+  const uint32_t T = select_kth_smem(sm, sm.cand_key, C, k, 32, cbits, tau);
   int gt_total, eq_total;
   {
     int lg = 0, le = 0;
