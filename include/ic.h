@@ -21,7 +21,14 @@
  *    memory and keeps no state besides a thread-local error message and one
  *    device error word.
  *  - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
- *    stream) and the call returns without synchronising.
+ *    stream) and the call returns without synchronising.  The kernels are
+ *    launched with programmatic dependent launch: each may be scheduled while
+ *    the previous kernel of the stream drains, and each waits for it
+ *    (griddepcontrol.wait) before touching global memory.  None signals its
+ *    dependents early, so stream order is unchanged for whatever the caller
+ *    enqueues before or after.  The calls contain no synchronisation and
+ *    allocate nothing, so a sequence of them can be captured in a CUDA graph
+ *    (ic_decode_step is, in the tests).
  *  - Tensors are dense, row-major, with the layouts given per function.
  *  - Errors are returned as negative ic_status codes; arguments are checked
  *    before anything is launched, so a failed call has launched nothing.
