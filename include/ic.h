@@ -26,9 +26,8 @@
  *    the previous kernel of the stream drains, and each waits for it
  *    (griddepcontrol.wait) before touching global memory.  None signals its
  *    dependents early, so stream order is unchanged for whatever the caller
- *    enqueues before or after.  The calls contain no synchronisation and
- *    allocate nothing, so a sequence of them can be captured in a CUDA graph
- *    (ic_decode_step is, in the tests).
+ *    enqueues before or after.  ic_decode_step is captured in a CUDA graph and
+ *    replayed in the tests; this note says nothing about the other calls.
  *  - Tensors are dense, row-major, with the layouts given per function.
  *  - Errors are returned as negative ic_status codes; arguments are checked
  *    before anything is launched, so a failed call has launched nothing.
