@@ -6,7 +6,7 @@
  * Sources.  "IndexCache: Wie DeepSeek O(NL^2)-Kosten in Sparse Attention um
  * 75% reduziert" (itoverdose.com): the intro (k = 2048 positions per query;
  * attention cost O(Lk)), the second paragraph (the indexer scores all previous
- * tokens), the F/S list and "the first layer is always F", the routing loop of
+ * tokens), the F/S list and the rule that the first layer is F, the routing loop of
  * "Einfache Implementierung, enorme Effizienzgewinne" (I <- Indexer(X);
  * T <- top-k(I); T_cache <- T / T <- T_cache; X <- SparseAttn(X, T)), the
  * T_cache paragraph right after it (one buffer, overwritten by every F layer,
@@ -94,8 +94,8 @@ ic_status ic_trace_begin(void* stream, int capacity);
 long ic_trace_end(float* ms, int* kinds, double* work, int capacity);
 
 /*
- * Per-row e4m3 quantisation (the fp8 variant of the indexer inputs, "per-token
- * fp32 scales"; OCP 8-bit floating point, E4M3).  For each row of n values:
+ * Per-row e4m3 quantisation (the fp8 variant of the indexer inputs, one fp32
+ * scale per token; OCP 8-bit floating point, E4M3).  For each row of n values:
  * scale = amax / 448 (1 for an all-zero row), code = E4M3_rne_satfinite(x / scale),
  * computed in fp32.
  *   x      [rows, n] of x_dtype (IC_BF16 or IC_F32)

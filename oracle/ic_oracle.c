@@ -102,7 +102,7 @@ uint8_t ico_e4m3_encode(double x) {
   return (uint8_t)((neg << 7) | best);
 }
 
-/* Per-row scaling to e4m3 ("per-token fp32 scales"): each row of n values gets
+/* Per-row scaling to e4m3 (one fp32 scale per token): each row of n values gets
  * scale = amax / 448 (1 when the row is all zero); code = E4M3(x / scale).
  * The scale and the division are fp32 operations (IEEE round-to-nearest), the
  * precision the quantised code is decided in. */

@@ -1,6 +1,6 @@
 // misc.cu -- the small kernels of the path:
 //  * per-row e4m3 quantisation of indexer inputs (OCP 8-bit floating point,
-//    E4M3; "per-token fp32 scales" of the fp8 indexer variant);
+//    E4M3, with one fp32 scale per token, as the fp8 indexer variant takes them);
 //  * the indexer on CUDA cores for fp32 inputs (small head counts and dims:
 //    the fp32 workload has 4 heads of dim 32, far too small for tensor tiles).
 #include "ic_device.cuh"
