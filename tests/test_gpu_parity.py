@@ -369,6 +369,33 @@ def test_stack_bf16_row_blocks_and_sharing():
         assert_attn_close(_np(dl[l]["out"][torch.from_numpy(rows).to(DEV)]), ro)
 
 
+def test_stack_e4m3_row_blocks_and_sharing():
+    """The e4m3 indexer inside the prefill stack (F,S,F,S at L=2600, k=2048) with
+    1000-row blocks: each block's per-row query scales are offset with its rows.
+    Sampled rows of T against the oracle on the same e4m3 codes and scales; the
+    attention of both layers that use T on those rows."""
+    wl = synth.variant("stack_32k", L=2600, pattern="F,S,F,S")
+    layers, host = _stack_layers(wl, DEV)
+    for d in layers:
+        d["q_idx"], d["q_scale"] = ic.ic_quant_e4m3_rows(d["q_idx"])
+        d["k_idx"], d["k_scale"] = ic.ic_quant_e4m3_rows(d["k_idx"])
+    ws_bytes = 1000 * wl.L * 4                     # 1000-row blocks: ragged last block
+    dl, t_cache = _run_stack(wl, wl.pattern, layers, ic.IC_E4M3, ws_bytes=ws_bytes)
+    T = t_cache.cpu().numpy()
+    rows = synth.sample_rows(wl.L, wl.k, 40, 1000).numpy()  # includes the block edges
+    d2 = layers[2]
+    ref = oracle.indexer_scores_e4m3(d2["q_idx"].cpu().numpy(), d2["q_scale"].cpu().numpy(),
+                                     d2["k_idx"].cpu().numpy(), d2["k_scale"].cpu().numpy(),
+                                     d2["w"].cpu().numpy(), rows_sel=rows)
+    for j, t in enumerate(rows):
+        check_index_row(T[t], ref[j], wl.k, t + 1)
+    for l in (2, 3):
+        h = host[l]
+        ro, _ = oracle.sparse_attn(h["q"][rows].float().numpy(), h["kv"].float().numpy(), T[rows],
+                                   wl.scale, dv=512)
+        assert_attn_close(_np(dl[l]["out"][torch.from_numpy(rows).to(DEV)]), ro)
+
+
 def test_stack_rows_zigzag_pieces_equal_the_whole_stack():
     """ic_layer_stack_rows over the zig-zag row pieces of 2 ranks (run one after the
     other here) gives the whole stack's index sets bit for bit and its outputs within
