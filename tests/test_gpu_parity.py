@@ -494,6 +494,34 @@ def test_decode_step_parity():
         assert_attn_close(_np(dl[l]["out"]), ro)
 
 
+def test_decode_step_two_full_layers_overwrite_t_cache():
+    """Decode with pattern F,F,S: the second F layer overwrites T_cache, so the final
+    T is layer 1's index set (checked against the oracle's scores of layer 1), and
+    layer 0 attended over layer 0's own set."""
+    wl = synth.variant("decode_200k", L=2500, batch=4, pattern="F,F,S")
+    layers, host = _stack_layers(wl, DEV)
+    for d in layers:
+        d["q_idx"], d["q_scale"] = ic.ic_quant_e4m3_rows(d["q_idx"])
+        d["k_idx"], d["k_scale"] = ic.ic_quant_e4m3_rows(d["k_idx"])
+    dl, t_cache = _run_stack(wl, wl.pattern, layers, ic.IC_E4M3, decode=True)
+    T = t_cache.cpu().numpy()
+    refs = []
+    for l in (0, 1):
+        d = layers[l]
+        refs.append(oracle.indexer_scores_e4m3(d["q_idx"].cpu().numpy(), d["q_scale"].cpu().numpy(),
+                                               d["k_idx"].cpu().numpy(), d["k_scale"].cpu().numpy(),
+                                               d["w"].cpu().numpy(), pos0=wl.L - 1))
+    for b in range(wl.batch):
+        check_index_row(T[b], refs[1][b, 0], wl.k, wl.L)
+    # layer 0's own set, from the oracle's layer-0 scores: its attention used that set
+    T0 = oracle.topk(refs[0][:, 0, :].astype(np.float32), wl.k)
+    for l, Tl in ((0, T0), (1, T), (2, T)):
+        h = host[l]
+        ro, _ = oracle.sparse_attn(h["q"].float().numpy(), h["kv"].float().numpy(), Tl[:, None, :],
+                                   wl.scale, dv=512)
+        assert_attn_close(_np(dl[l]["out"]), ro)
+
+
 def test_decode_step_graph_replay_matches_eager():
     """The decode step captured in a CUDA graph (programmatic launch edges
     included) and replayed gives bit-identical T and outputs to eager calls, also
