@@ -187,16 +187,22 @@ size_t ic_attn_workspace_size(int batch, int rows, int heads, int dv, int k);
  *
  *   batch * rows <= IC_NOALLOC_MAX_QUERIES (64), else IC_ERR_UNSUPPORTED;
  *   v != NULL (the MQA form, which needs no scratch) -> IC_ERR_UNSUPPORTED;
+ *   a split that needs more than IC_NOALLOC_SCRATCH_BYTES -> IC_ERR_WORKSPACE
+ *     (queries * pieces per query <= SMs + 2 * queries: at most 276 of the 512
+ *     slots on a 148-SM B200; only a part with far more SMs could need more);
+ *   a failed device query or address lookup -> IC_ERR_CUDA;
  *   other checks and errors as ic_sparse_attn.
+ * `out` and `lse` are the caller's, as for ic_sparse_attn.
  *
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress with that device current) and caches it; make that
- * first call before any stream capture.  All calls share the one array: calls
- * that overlap on the GPU (other streams, other host threads) race on it and
- * must be serialised by the caller, e.g. by using a single stream.  Each call
- * overwrites every partial it later reads, so leftovers from an earlier call
- * do not matter.  Runs on the calling thread's current device, which must own
- * `stream`.
+ * The first call in a CUDA context looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it under the
+ * context's id; make that first call before any stream capture.  A call made
+ * after a device reset (a new context) looks the address up again.  All calls
+ * share the one array: calls that overlap on the GPU (other streams, other host
+ * threads) race on it and must be serialised by the caller, e.g. by using a
+ * single stream.  Each call overwrites every partial it later reads, so
+ * leftovers from an earlier call do not matter.  Runs on the calling thread's
+ * current device, which must own `stream`.
  */
 #define IC_NOALLOC_MAX_QUERIES 64
 #define IC_NOALLOC_SCRATCH_BYTES (64u * 8u * 16u * 514u * 4u)

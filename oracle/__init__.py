@@ -246,8 +246,9 @@ def sparse_attn(q, kv, idx, scale: float, dv: int | None = None, v=None,
 def parse_pattern(pattern: str) -> list[str]:
     """Layer types from a pattern string such as "F,S,S,S" or "F S S S" or "FSSS".
 
-    The first layer must be F: it fills the index cache ("Die erste Schicht ist
-    stets eine Full-Schicht").  Raises ValueError otherwise.
+    The first layer must be F, since only an F layer fills the index cache that
+    later S layers read ("IndexCache: Wie DeepSeek O(NL^2)-Kosten in Sparse
+    Attention um 75% reduziert", the F/S layer list).  Raises ValueError otherwise.
     """
     if not isinstance(pattern, str):
         raise ValueError("pattern must be a string")

@@ -247,20 +247,28 @@ def ic_sparse_attn(q, kv, idx, scale: float, *, v=None, dv: int | None = None, o
     return out
 
 
-def ic_sparse_attn_noalloc(q, kv, idx, scale: float, *, dv: int = 512, out=None, lse=None,
+def ic_sparse_attn_noalloc(q, kv, idx, scale: float, *, out, dv: int = 512, lse=None,
                            stream=None):
     """Absorbed-MLA sparse attention whose split scratch is the library's fixed device
     array rather than a workspace (for callers that cannot allocate; at most
     IC_NOALLOC_MAX_QUERIES = 64 queries).  q [B?,R,16,576] bf16; kv [B?,Lkv,ld_kv];
-    idx [B?,R,k].  Calls that overlap on the GPU race on the shared array."""
-    _contig(q, idx)
+    idx [B?,R,k] int32.  The caller passes ``out`` [B?,R,16,dv] bf16 (and, if wanted,
+    ``lse`` [B?,R,16] f32), both contiguous: this wrapper allocates nothing either.
+    Calls that overlap on the GPU race on the shared array."""
+    _contig(q, idx, out, lse)
     if kv.stride(-1) != 1:
         raise ValueError("kv rows must be contiguous")
     squeeze = q.dim() == 3
     B = 1 if squeeze else q.shape[0]
     R, heads, dk = q.shape[-3:]
-    if out is None:
-        out = torch.empty(q.shape[:-1] + (dv,), dtype=q.dtype, device=q.device)
+    if idx.dtype != torch.int32 or tuple(idx.shape[:-1]) != tuple(q.shape[:-2]):
+        raise ValueError("idx must be int32 [B?, R, k] matching q")
+    if out is None or out.dtype != q.dtype or tuple(out.shape) != tuple(q.shape[:-1]) + (dv,):
+        raise ValueError("out must be a %s tensor of shape %s" % (
+            q.dtype, tuple(q.shape[:-1]) + (dv,)))
+    if lse is not None and (lse.dtype != torch.float32 or
+                            tuple(lse.shape) != tuple(q.shape[:-1])):
+        raise ValueError("lse must be a float32 tensor of shape %s" % (tuple(q.shape[:-1]),))
     _check(lib().ic_sparse_attn_noalloc(_p(q), _p(kv), kv.stride(-2), None, _p(idx),
                                         dtype_code(q), B, R, heads, dk, dv, kv.shape[-2],
                                         idx.shape[-1], float(scale), _p(out), _p(lse),

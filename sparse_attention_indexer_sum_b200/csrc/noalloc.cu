@@ -6,9 +6,14 @@
 // before its merge kernel combines them: per piece of a query, 16 heads x (512
 // output floats + running max + running sum).  The entry point accepts at most
 // IC_NOALLOC_MAX_QUERIES queries (batch * rows).  The split plan cuts their
-// (query, 32-key tile) pairs into one contiguous range per SM, so a call makes at
-// most SMs + 2 x queries pieces (276 on a 148-SM B200); the array holds
-// IC_NOALLOC_MAX_QUERIES x 8 pieces and a call that would need more is refused.
+// (query, 32-key tile) pairs into G <= SMs equal contiguous ranges, so one query
+// spans at most ceil(G / queries) + 1 pieces, and every query gets that many
+// slots (maxp): queries * maxp <= G + 2 * queries, at most 276 slots on a 148-SM
+// B200.  The array holds IC_NOALLOC_MAX_QUERIES x 8 = 512 slots; the exact need
+// (attn_mla_ws_bytes) is checked on every call and a larger one is refused with
+// IC_ERR_WORKSPACE, which only a part with far more SMs could reach.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "ic_device.cuh"
@@ -27,10 +32,41 @@ static __device__ __align__(256) float g_attn_noalloc_scratch[IC_NOALLOC_SCRATCH
 
 constexpr int kNoallocMaxDevices = 64;
 static std::mutex g_noalloc_mu;
-static void* g_noalloc_ptr[kNoallocMaxDevices];
+struct NoallocSlot {
+  unsigned long long ctx_id;  // context the address belongs to (0 = none yet)
+  void* ptr;
+};
+static NoallocSlot g_noalloc_slot[kNoallocMaxDevices];
 
-// Device address of the scratch array on the calling thread's current device;
-// looked up on the first call for that device and cached.
+// Unique id of the calling thread's current context, or 0 if it has none.  A
+// device reset ends the context and the next one gets a new id, with the module
+// (and so the array) loaded again, possibly at another address.
+static unsigned long long current_ctx_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_cur || !get_id) return 0;
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch array in the calling thread's current context.
+// It is looked up (cudaGetSymbolAddress, with the device current) on the first
+// call in a context and cached with that context's id; a call from a later
+// context (after a device reset, say) looks it up again.
 static ic_status noalloc_scratch(void** out) {
   int dev = -1;
   ic_status st = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
@@ -39,15 +75,18 @@ static ic_status noalloc_scratch(void** out) {
     return fail(IC_ERR_UNSUPPORTED, "sparse_attn_noalloc: device ordinal %d above %d", dev,
                 kNoallocMaxDevices - 1);
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoallocSlot& slot = g_noalloc_slot[dev];
+  const unsigned long long id = current_ctx_id();
+  if (!slot.ptr || id == 0 || id != slot.ctx_id) {
     void* p = nullptr;
     st = cuda_check(cudaGetSymbolAddress(&p, g_attn_noalloc_scratch),
                     "cudaGetSymbolAddress(sparse_attn_noalloc scratch)");
     if (st) return st;
     if (!p) return fail(IC_ERR_CUDA, "sparse_attn_noalloc: scratch symbol has no address");
-    g_noalloc_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx_id = current_ctx_id();  // the lookup above made the context current if needed
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return IC_OK;
 }
 

@@ -21,6 +21,25 @@ def assert_scores_close(got, ref, atol=IDX_ATOL, rtol=IDX_RTOL_BF16, what="score
         what, bad.sum(), bad.size, err.max(), ref[fin][np.argmax(err - lim)])
 
 
+def assert_fp8_scores_close_to_unquantised(got, ref, rtol=IDX_RTOL_FP8):
+    """Scores from e4m3 inputs against the oracle on the unquantised inputs:
+    |got - ref| <= rtol * max(|ref|, rms of the row's finite refs) on finite entries
+    (the row-RMS floor keeps near-zero gated scores from dominating a relative test);
+    -inf exactly where ref is -inf.  Differences are taken on finite entries only."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    fin = np.isfinite(ref)
+    assert (np.isneginf(got) == ~fin).all(), "masked entries differ"
+    sq = np.zeros_like(ref)
+    sq[fin] = ref[fin] ** 2
+    rms = np.sqrt(sq.sum(axis=-1, keepdims=True) / np.maximum(fin.sum(axis=-1, keepdims=True), 1))
+    err = np.zeros_like(ref)
+    err[fin] = np.abs(got[fin] - ref[fin])
+    lim = rtol * np.maximum(np.abs(np.where(fin, ref, 0.0)), rms)
+    assert (err <= lim).all(), float((err - lim).max())
+
+
 def check_index_row(T_row, ref_scores_row, k, valid, atol=IDX_ATOL, rtol=IDX_RTOL_BF16):
     """T_row: the GPU's index set (ascending, -1 padded).  ref_scores_row: the oracle's scores.
 

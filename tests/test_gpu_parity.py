@@ -14,8 +14,8 @@ import torch
 import oracle
 from sparse_attention_indexer_sum_b200 import binding as ic
 from sparse_attention_indexer_sum_b200 import synth
-from tests.paritylib import (IDX_RTOL_FP8, assert_attn_close, assert_scores_close,
-                             check_index_row)
+from tests.paritylib import (assert_attn_close, assert_fp8_scores_close_to_unquantised,
+                             assert_scores_close, check_index_row)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -182,11 +182,7 @@ def test_indexer_fp8_parity(B, R, Lk, pos0):
     assert_scores_close(got, ref_q)
     # (ii) against the unquantised bf16 inputs: rel 5e-2 with a row-RMS floor
     ref = oracle.indexer_scores(q.float().numpy(), k.float().numpy(), w.numpy(), pos0=pos0)
-    fin = np.isfinite(ref)
-    rms = np.sqrt(np.nanmean(np.where(fin, ref, np.nan) ** 2, axis=-1, keepdims=True))
-    err = np.abs(np.where(fin, got - ref, 0))
-    lim = IDX_RTOL_FP8 * np.maximum(np.abs(np.where(fin, ref, 0)), rms)
-    assert (err <= lim).all(), float((err - lim).max())
+    assert_fp8_scores_close_to_unquantised(got, ref)
 
 
 def test_indexer_f32_parity():

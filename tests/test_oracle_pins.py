@@ -221,6 +221,29 @@ def test_indexer_rows_sel_batch_and_pos0():
     np.testing.assert_array_equal(oracle.indexer_scores(q, k2, w, pos0=4)[0], full[0])
 
 
+def test_indexer_scores_at_positions_map_to_causal_rows():
+    # Rows scored one by one at arbitrary positions p_j must equal rows p_j of the
+    # whole causal matrix (the pinned rows_sel path) and the rank-one closed form.
+    g = np.random.default_rng(17)
+    L, H, D = 23, 3, 5
+    u = g.standard_normal(D)
+    u /= np.linalg.norm(u)
+    a = g.standard_normal((L, H))
+    b = g.standard_normal(L) * np.arange(1, L + 1)
+    w = g.uniform(0, 1, (L, H)) * np.arange(1, L + 1)[:, None]
+    q, k = a[:, :, None] * u, b[:, None] * u
+    pos = np.array([22, 0, 7, 8, 21, 3])              # unsorted, first and last rows
+    got = oracle.indexer_scores_at(q[pos], k, w[pos], pos, nthreads=3)
+    np.testing.assert_array_equal(got, oracle.indexer_scores(q, k, w, rows_sel=pos))
+    for j, p in enumerate(pos):
+        assert np.isneginf(got[j, p + 1:]).all()
+        for s in range(p + 1):
+            ref = sum(w[p, h] * max(0.0, a[p, h] * b[s]) for h in range(H))
+            assert abs(got[j, s] - ref) <= 1e-12 * (1 + abs(ref))
+    # an off-by-one in the position mapping would unmask key p + 1 or mask key p
+    assert np.isfinite(got[:, 0]).all()
+
+
 def test_indexer_e4m3_is_definition_on_dequantised_values():
     # integer-valued codes with unit scales: the e4m3 indexer equals exact integer arithmetic
     q_codes = np.zeros((4, 2, 4), dtype=np.uint8)

@@ -33,14 +33,29 @@ def _inputs(B, R, k, Lkv, seed, pad=False):
     return q, kv, torch.from_numpy(idx)
 
 
+SCRATCH_BYTES = 64 * 8 * 16 * 514 * 4  # IC_NOALLOC_SCRATCH_BYTES in include/ic.h
+
+
+@pytest.mark.gpu
+def test_noalloc_scratch_covers_every_accepted_query_count_on_this_device():
+    # the split's scratch need (as the workspace query reports it for this device's
+    # SM count) fits the fixed array for every batch * rows the entry point accepts
+    for n in range(1, MAX_QUERIES + 1):
+        for B, R in ((n, 1), (1, n)):
+            need = ic.ic_attn_workspace_size(B, R, 16, 512, 2048)
+            assert need <= SCRATCH_BYTES, (B, R, need)
+
+
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
     dev = "cuda"
     scale = 1 / math.sqrt(576)
-    # first call: the largest accepted batch (64 decode queries, k = 2048), which
-    # fills the whole array; second call: a ragged, smaller shape with fewer splits,
-    # so the first call's partials are still sitting in the array
+    # first call: the largest accepted batch (64 decode queries, k = 2048, up to 4
+    # pieces each on 148 SMs); second call: 5 queries at k = 2048, the shape with
+    # the most pieces per query (about 30 each), so it reads slots the first call
+    # left holding other partials; third call: a ragged, smaller shape
     for B, R, k, Lkv, seed, pad in ((MAX_QUERIES, 1, 2048, 5000, 11, False),
+                                    (5, 1, 2048, 4000, 13, False),
                                     (3, 5, 1000, 1500, 12, True)):
         q, kv, idx = _inputs(B, R, k, Lkv, seed, pad)
         q, kv, idx = q.to(dev), kv.to(dev), idx.to(dev)
@@ -71,3 +86,11 @@ def test_noalloc_rejects_oversize_and_mqa_before_touching_the_device():
     st = lib.ic_sparse_attn_noalloc(fake, fake, 576, None, fake, ic.IC_BF16, 1, 4, 16, 576, 512,
                                     100, 4096, 1.0, fake, None, None)
     assert st == ic.IC_ERR_UNSUPPORTED  # k above 2048, as for ic_sparse_attn
+    # the Python wrapper allocates nothing either: `out` is required and checked
+    q = torch.zeros(1, 2, 16, 576, dtype=torch.bfloat16)
+    idx = torch.zeros(1, 2, 8, dtype=torch.int32)
+    with pytest.raises(TypeError):
+        ic.ic_sparse_attn_noalloc(q, q[0, 0], idx, 1.0)  # noqa: missing out
+    with pytest.raises(ValueError):
+        ic.ic_sparse_attn_noalloc(q, q[0, 0], idx, 1.0,
+                                  out=torch.zeros(1, 2, 16, 511, dtype=torch.bfloat16))
