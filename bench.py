@@ -51,6 +51,9 @@ METRIC = "prefill tokens/s (indexer+top-k+sparse attn) at L=200K; % of roofline"
 # pairs).  The score writes dominate and grow with the pairs; keys and queries
 # come from L2.  A launch's traffic is this figure times its pairs.
 INDEXER_BF16_DRAM_BYTES_PER_PAIR = 203.9e6 / 51331328
+# The same for the e4m3 indexer (`profile_cases indexer_longrows_e4m3`, same rows and
+# positions: 20.8 MB read + 154.0 MB written for the same 51,331,328 pairs).
+INDEXER_E4M3_DRAM_BYTES_PER_PAIR = 174.76e6 / 51331328
 UNIT = "tokens/s"
 
 
@@ -132,6 +135,56 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------------------------------ fp8 peak
+def measure_fp8_peak(dev, sustain_s: float = 3.0):
+    """Dense e4m3 GEMM throughput on this GPU, the denominator of the e4m3 indexer's
+    roofline: torch._scaled_mm (cuBLASLt) on 8192^3 e4m3 x e4m3 -> bf16 with unit
+    fp32 scales, 2 n^3 flop per call, CUDA events on the current stream.  Burst: the
+    best of 10 timed groups of 5 calls.  Sustained: calls back to back for
+    `sustain_s` seconds under the power cap, with the SM clocks sampled meanwhile.
+    Both accumulation modes are timed and the faster one is the peak."""
+    n = 8192
+    g = torch.Generator(device=dev).manual_seed(0)
+    a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+    one = torch.ones((), device=dev)
+    flop = 2.0 * n ** 3
+    stream = torch.cuda.current_stream(dev)
+    res = {"how": "torch._scaled_mm e4m3 %d^3 -> bf16, unit scales; burst = best of 10 groups "
+                  "of 5 calls, sustained = back to back for %.0f s" % (n, sustain_s)}
+    best = None
+    for fast in (False, True):
+        def mm(fast=fast):
+            return torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one,
+                                    out_dtype=torch.bfloat16, use_fast_accum=fast)
+        try:
+            for _ in range(5):
+                mm()
+            torch.cuda.synchronize(dev)
+        except Exception as e:  # no fp8 GEMM on this torch / GPU
+            res["error_fast_accum_%s" % fast] = str(e).splitlines()[0][:200]
+            continue
+        burst = min(_timed(mm, 5, stream) for _ in range(10))
+        if best is None or burst < best[1]:
+            best = (fast, burst, mm)
+        res["burst_tflops_fast_accum_%s" % str(fast).lower()] = flop / (burst * 1e-3) / 1e12
+    if best is None:
+        return res
+    fast, burst, mm = best
+    calls = max(10, int(sustain_s * 1e3 / burst))
+    clocks = ClockSampler("GPU-%s" % torch.cuda.get_device_properties(dev).uuid)
+    clocks.start()
+    time.sleep(0.3)
+    clocks.mark()
+    ms = _timed(mm, calls, stream)
+    res.update(fp8_tflops=flop / (burst * 1e-3) / 1e12,
+               fp8_tflops_sustained=flop / (ms * 1e-3) / 1e12, use_fast_accum=fast,
+               sustained_calls=calls, clocks=clocks.stop())
+    del a, b
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------------------ ranks
 def reduce_max(x: float, world: int, device) -> float:
     """The largest of every rank's x (one all-reduce; the identity on one rank).
@@ -173,6 +226,90 @@ def make_inputs(wl, device, pattern_all, fp8: bool, seed: int):
 
 def kinds_of(pattern):
     return [c for c in pattern if c in "FS"]
+
+
+def time_stack(step, args, stream, dev, barrier, max_over_ranks):
+    """W warm-up steps; K steps timed untraced between two CUDA events on the launching
+    stream (clocks sampled meanwhile; the max over ranks); then K more steps with an
+    event after every launch, for the per-kernel split.  Returns
+    (ms_per_step, clocks, launches in the traced K steps, trace)."""
+    from sparse_attention_indexer_sum_b200 import binding as ic
+    for _ in range(args.warmup):
+        step()
+    ic.ic_device_status(stream)
+    barrier()
+    clocks = ClockSampler("GPU-%s" % torch.cuda.get_device_properties(dev).uuid)
+    clocks.start()
+    time.sleep(0.5)
+    clocks.mark()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    ic.ic_device_status(stream)
+    cap = max(4096, 256 * args.steps)
+    ic.ic_trace_begin(cap, stream=stream)
+    for _ in range(args.steps):
+        step()
+    n_launch, trace = ic.ic_trace_end(cap)
+    ic.ic_device_status(stream)
+    barrier()
+    return ms, clk, n_launch, trace
+
+
+def stack_roofline(trace, steps, wl, fp8, peaks, fp8_sustained=None):
+    """Per-kernel device time and algorithmic work of a traced pass, and the roofline
+    object of the dominant kernel (the tensor-core indexer)."""
+    agg = {}
+    for name, kms, work in trace:
+        a = agg.setdefault(name, [0, 0.0, 0.0])
+        a[0] += 1
+        a[1] += kms
+        a[2] += work
+    tot_ms = sum(a[1] for a in agg.values())
+    dom = "indexer_tc_e4m3" if fp8 else "indexer_tc_bf16"
+    d_n, d_ms, d_work = agg.get(dom, [0, 0.0, 0.0])
+    bf16_peak = peaks["bf16_sustained"]
+    if fp8 and fp8_sustained:
+        peak = fp8_sustained
+        peak_src = "e4m3 GEMM measured in this run (torch._scaled_mm 8192^3, sustained) %.1f " \
+                   "TFLOP/s" % peak
+    elif fp8:
+        peak = 2.0 * bf16_peak
+        peak_src = "%s bf16 sustained %.1f TFLOP/s x2 (e4m3 nominal ratio; no fp8 GEMM " \
+                   "measurement)" % (peaks["source"], bf16_peak)
+    else:
+        peak = bf16_peak
+        peak_src = "%s bf16 sustained %.1f TFLOP/s" % (peaks["source"], bf16_peak)
+    achieved = d_work / (d_ms * 1e-3) / 1e12 if d_ms > 0 else 0.0
+    stages = {}
+    for name, (n, kms, work) in sorted(agg.items()):
+        st = {"launches_per_step": n / steps, "ms_per_step": kms / steps,
+              "share": kms / tot_ms if tot_ms else 0.0}
+        if name.startswith("indexer_tc"):
+            st.update(bound="tensor", achieved_tflops=work / (kms * 1e-3) / 1e12,
+                      unit="TFLOP/s")
+        else:
+            st.update(bound="hbm", achieved_gbs=work / (kms * 1e-3) / 1e9,
+                      frac_hbm=work / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"], unit="GB/s")
+        stages[name] = st
+    pairs_per_launch = d_work / d_n / (2.0 * wl.H * wl.D) if d_n else 0.0
+    per_pair = INDEXER_E4M3_DRAM_BYTES_PER_PAIR if fp8 else INDEXER_BF16_DRAM_BYTES_PER_PAIR
+    traffic = per_pair * pairs_per_launch if per_pair else None
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak if peak else None, "traffic": traffic,
+                "traffic_source": None if not per_pair else
+                "ncu dram__bytes_read.sum + dram__bytes_write.sum of the same kernel on 512 "
+                "rows at position 100000 (%.2f B per causal pair), times the pairs of a "
+                "launch" % per_pair,
+                "peak_source": peak_src,
+                "work_per_launch": d_work / d_n if d_n else None,
+                "launches": d_n, "ms_per_launch": d_ms / d_n if d_n else None}
+    return stages, roofline
 
 
 def run_ours(args, rank, world, local_rank):
@@ -225,63 +362,11 @@ def run_ours(args, rank, world, local_rank):
     def max_over_ranks(x: float) -> float:
         return reduce_max(x, world, dev)
 
-    for _ in range(args.warmup):
-        step()
-    ic.ic_device_status(stream)
-    barrier()
-    clocks = ClockSampler("GPU-%s" % torch.cuda.get_device_properties(dev).uuid)
-    clocks.start()
-    time.sleep(0.5)
-    clocks.mark()
-    cap = max(4096, 256 * args.steps)
-    ic.ic_trace_begin(cap, stream=stream)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    n_launch, trace = ic.ic_trace_end(cap)
-    barrier()
-    clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    ms = max_over_ranks(ms)
-    ic.ic_device_status(stream)
-
-    # per-kernel device time and algorithmic work over the timed region
-    agg = {}
-    for name, kms, work in trace:
-        a = agg.setdefault(name, [0, 0.0, 0.0])
-        a[0] += 1
-        a[1] += kms
-        a[2] += work
-    tot_ms = sum(a[1] for a in agg.values())
-    dom = "indexer_tc_e4m3" if fp8 else "indexer_tc_bf16"
-    d_n, d_ms, d_work = agg.get(dom, [0, 0.0, 0.0])
-    bf16_peak = peaks["bf16_sustained"]
-    peak = bf16_peak * (2.0 if fp8 else 1.0)   # e4m3 dense peak = 2x bf16 (nominal ratio)
-    achieved = d_work / (d_ms * 1e-3) / 1e12 if d_ms > 0 else 0.0
-    stages = {}
-    for name, (n, kms, work) in sorted(agg.items()):
-        st = {"launches_per_step": n / args.steps, "ms_per_step": kms / args.steps,
-              "share": kms / tot_ms if tot_ms else 0.0}
-        if name.startswith("indexer_tc"):
-            st.update(bound="tensor", achieved_tflops=work / (kms * 1e-3) / 1e12,
-                      unit="TFLOP/s")
-        else:
-            st.update(bound="hbm", achieved_gbs=work / (kms * 1e-3) / 1e9,
-                      frac_hbm=work / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"], unit="GB/s")
-        stages[name] = st
-    pairs_per_launch = d_work / d_n / (2.0 * wl.H * wl.D) if d_n else 0.0
-    traffic = None if fp8 else INDEXER_BF16_DRAM_BYTES_PER_PAIR * pairs_per_launch
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak if peak else None, "traffic": traffic,
-                "traffic_source": None if fp8 else
-                "ncu dram__bytes_read.sum + dram__bytes_write.sum of the same kernel on 512 "
-                "rows at position 100000 (3.97 B per causal pair), times the pairs of a launch",
-                "peak_source": "%s bf16 sustained %.1f TFLOP/s%s" % (
-                    peaks["source"], bf16_peak, " x2 (e4m3 nominal ratio)" if fp8 else ""),
-                "work_per_launch": d_work / d_n if d_n else None,
-                "launches": d_n, "ms_per_launch": d_ms / d_n if d_n else None}
+    fp8_peak = measure_fp8_peak(dev) if rank == 0 and world == 1 else None
+    ms, clk, n_launch, trace = time_stack(step, args, stream, dev, barrier, max_over_ranks)
+    fp8_sus = (fp8_peak or {}).get("fp8_tflops_sustained")
+    stages, roofline = stack_roofline(trace, args.steps, wl, fp8, peaks, fp8_sus)
+    achieved = roofline["achieved"]
     value = wl.L / (ms * 1e-3) if shard else job_throughput(wl.L, world, ms)
     log("rank %d: %.2f ms/step, %.0f tokens/s, indexer %.1f TFLOP/s" % (rank, ms, value, achieved))
 
@@ -300,13 +385,44 @@ def run_ours(args, rank, world, local_rank):
                                    else "single GPU"),
                    "l2": "inputs larger than L2 (no flush needed)"},
         "gpu_launches": n_launch, "roofline": roofline, "stages": stages, "clocks": clk,
+        "timing": "%d steps untraced between CUDA events (value); the per-kernel split and "
+                  "the roofline come from a second pass of %d steps with an event after "
+                  "every launch" % (args.steps, args.steps),
     }
+    if fp8_peak is not None:
+        res["fp8_peak_measured"] = fp8_peak
+
+    if args.e4m3_line and not fp8 and not shard:
+        # the same stack with the e4m3 indexer on the same inputs (quantised per row)
+        lay8 = [dict(d) for d in layers]
+        for l, c in enumerate(kinds_of(pattern)):
+            if c == "F":
+                lay8[l]["q_idx"], lay8[l]["q_scale"] = ic.ic_quant_e4m3_rows(layers[l]["q_idx"])
+                lay8[l]["k_idx"], lay8[l]["k_scale"] = ic.ic_quant_e4m3_rows(layers[l]["k_idx"])
+        desc8 = ic.make_desc(L=wl.L, k=wl.k, H=wl.H, D=wl.D, idx_dtype=ic.IC_E4M3, heads=wl.Hq,
+                             dk=wl.Dk, dv=wl.Dv, attn_dtype=ic.IC_BF16, scale=wl.scale)
+
+        def step8():
+            ic.ic_layer_stack(pattern, desc8, lay8, t_cache, ws, stream=stream)
+        ms8, clk8, n8, trace8 = time_stack(step8, args, stream, dev, barrier, max_over_ranks)
+        stages8, roof8 = stack_roofline(trace8, args.steps, wl, True, peaks, fp8_sus)
+        res["prefill_e4m3"] = {
+            "pattern": pattern, "indexer": "e4m3 per-row scales (q per token and head, k per "
+            "token), fp32 accumulate; attention bf16", "ms_per_step": ms8,
+            "value": job_throughput(wl.L, world, ms8), "unit": UNIT, "gpu_launches": n8,
+            "roofline": roof8, "stages": stages8, "clocks": clk8,
+            "speedup_over_bf16_indexer": ms / ms8}
+        log("e4m3 indexer: %.2f ms/step, indexer %.1f TFLOP/s = %.2f of %s" % (
+            ms8, roof8["achieved"], roof8["frac"] or 0.0, roof8["peak_source"]))
+        del lay8
+        torch.cuda.empty_cache()
 
     if args.compare:
         for _ in range(1):
             step(allf)
         barrier()
         ka = max(2, args.steps // 2)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(ka):
             step(allf)
@@ -755,6 +871,8 @@ def main():
                          "in zig-zag chunks (strong scaling)")
     ap.add_argument("--no-decode", dest="decode", action="store_false",
                     help="skip the decode (64 x 1 token at 200K context) measurement")
+    ap.add_argument("--no-e4m3-line", dest="e4m3_line", action="store_false",
+                    help="skip the same stack with the e4m3 indexer (key prefill_e4m3)")
     ap.add_argument("--no-stack32k", dest="stack32k", action="store_false",
                     help="skip the 8-layer L=32768 stack and its layer-overlap report")
     args = ap.parse_args()

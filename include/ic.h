@@ -142,6 +142,16 @@ ic_status ic_topk(const float* scores, long rows, int n, long ld, long pos0, int
                   void* stream);
 
 /*
+ * ic_topk with an arbitrary candidate count per row: row r's candidates are
+ * columns s < valid_len[r] (clamped to [0, n]).  Rows of different sequences
+ * packed into one call, or rows with their own causal offsets, use this form.
+ *   valid_len [rows] int32, device
+ * Other arguments, the output and the errors as ic_topk.
+ */
+ic_status ic_topk_varlen(const float* scores, long rows, int n, long ld, const int* valid_len,
+                         int k, int* idx, void* stream);
+
+/*
  * Sparse attention of each query over its index set (routing loop:
  * X <- SparseAttn(X, T); MLA paragraph).  For query (b, r), head h, with
  * J = { idx[b, r, j] : idx >= 0 } (-1 entries are skipped):

@@ -27,7 +27,8 @@ IC_F32, IC_BF16, IC_E4M3 = 0, 1, 2
 # names declared in include/ic.h (checked against the header by the tests)
 EXPORTS = ("ic_last_error", "ic_version", "ic_device_status", "ic_trace_begin", "ic_trace_end",
            "ic_quant_e4m3_rows",
-           "ic_indexer_scores", "ic_topk", "ic_sparse_attn", "ic_attn_workspace_size",
+           "ic_indexer_scores", "ic_topk", "ic_topk_varlen", "ic_sparse_attn",
+           "ic_attn_workspace_size",
            "ic_layer_stack", "ic_decode_step", "ic_stack_workspace_size",
            "ic_sparse_attn_noalloc", "ic_layer_stack_rows", "ic_layer_stack_varlen")
 
@@ -77,6 +78,7 @@ def lib() -> ctypes.CDLL:
     L.ic_quant_e4m3_rows.argtypes = [P, I, Lg, I, P, P, P]
     L.ic_indexer_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Lg, P, Lg, P]
     L.ic_topk.argtypes = [P, Lg, I, Lg, Lg, I, P, P]
+    L.ic_topk_varlen.argtypes = [P, Lg, I, Lg, P, I, P, P]
     L.ic_sparse_attn.argtypes = [P, P, Lg, P, P, I, I, I, I, I, I, I, I, F, P, P, P, S, P]
     L.ic_attn_workspace_size.argtypes = [I, I, I, I, I]
     L.ic_attn_workspace_size.restype = S
@@ -92,6 +94,7 @@ def lib() -> ctypes.CDLL:
     L.ic_stack_workspace_size.restype = S
     L.ic_sparse_attn_noalloc.argtypes = [P, P, Lg, P, P, I, I, I, I, I, I, I, I, F, P, P, P]
     for name in ("ic_device_status", "ic_quant_e4m3_rows", "ic_indexer_scores", "ic_topk",
+                 "ic_topk_varlen",
                  "ic_sparse_attn", "ic_layer_stack", "ic_decode_step", "ic_sparse_attn_noalloc",
                  "ic_layer_stack_rows", "ic_layer_stack_varlen"):
         getattr(L, name).restype = I
@@ -215,6 +218,23 @@ def ic_topk(scores, k: int, *, n: int | None = None, pos0: int = -1, idx=None, s
         idx = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
     _check(lib().ic_topk(_p(scores), rows, n, scores.stride(0), int(pos0), int(k), _p(idx),
                          _stream(stream)))
+    return idx
+
+
+def ic_topk_varlen(scores, k: int, valid_len, *, n: int | None = None, idx=None, stream=None):
+    """Exact top-k indices [rows, k] of scores [rows, ld] with row r's candidates the
+    columns s < valid_len[r] (device int32 [rows])."""
+    rows = scores.shape[0]
+    n = scores.shape[1] if n is None else n
+    if scores.stride(1) != 1:
+        raise ValueError("scores rows must be contiguous")
+    if valid_len.dtype != torch.int32 or valid_len.numel() != rows:
+        raise ValueError("valid_len must be int32 [rows]")
+    _contig(valid_len)
+    if idx is None:
+        idx = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
+    _check(lib().ic_topk_varlen(_p(scores), rows, n, scores.stride(0), _p(valid_len), int(k),
+                                _p(idx), _stream(stream)))
     return idx
 
 

@@ -359,6 +359,17 @@ ic_status ic_topk(const float* scores, long rows, int n, long ld, long pos0, int
   return launch_topk(scores, rows, n, ld, pos0, k, idx, static_cast<cudaStream_t>(stream));
 }
 
+ic_status ic_topk_varlen(const float* scores, long rows, int n, long ld, const int* valid_len,
+                         int k, int* idx, void* stream) {
+  if (!scores || !idx || !valid_len) return fail(IC_ERR_INVALID_ARG, "topk_varlen: NULL tensor");
+  if (rows < 0 || n < 0 || ld < n || k < 1 || k > 2048)
+    return fail(IC_ERR_INVALID_ARG, "topk_varlen: bad sizes (rows %ld n %d ld %ld k %d)", rows, n,
+                ld, k);
+  if (rows > 0x7fffffffL) return fail(IC_ERR_UNSUPPORTED, "topk_varlen: too many rows");
+  return launch_topk(scores, rows, n, ld, -1, k, idx, static_cast<cudaStream_t>(stream),
+                     valid_len);
+}
+
 ic_status ic_sparse_attn(const void* q, const void* kv, long ld_kv, const void* v, const int* idx,
                          ic_dtype dt, int batch, int rows, int heads, int dk, int dv, int Lkv,
                          int k, float scale, void* out, float* lse, void* workspace,

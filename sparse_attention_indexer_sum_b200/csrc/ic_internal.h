@@ -70,8 +70,10 @@ ic_status launch_indexer_tc(bool fp8, const void* q, const float* q_scale, const
 ic_status launch_indexer_f32(const float* q, const float* k, const float* w, int batch, int H,
                              int D, int rows, int Lk, long pos0, float* scores, long ld,
                              cudaStream_t stream);
+// valid_len (device int32 [rows], or NULL): row r's candidate count, clamped to
+// [0, n]; NULL means min(n, pos0 + r + 1), or n when pos0 < 0.
 ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0, int k, int* idx,
-                      cudaStream_t stream);
+                      cudaStream_t stream, const int* valid_len = nullptr);
 // valid_entries: number of index entries >= 0 over all rows if the caller knows
 // it (the causal stack does), else -1 (rows * k is assumed for tracing only).
 ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* idx, int batch,

@@ -414,8 +414,9 @@ __device__ __forceinline__ void collect_candidates(TopkSmem& sm, const float* __
 }
 
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restrict__ scores, long ld,
-                                                          int n, long pos0, int k,
-                                                          int* __restrict__ idx) {
+                                                          int n, long pos0,
+                                                          const int* __restrict__ valid_len,
+                                                          int k, int* __restrict__ idx) {
   extern __shared__ uint8_t tk_smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
   const int tid = threadIdx.x;
@@ -424,8 +425,9 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
   // collects the candidates of its part, CTA 0 merges them and selects.
   const uint32_t S = cluster_nctarank(), crank = cluster_ctarank();
   const long row = blockIdx.x / S;
-  long nvl = (pos0 < 0) ? n : pos0 + row + 1;
+  long nvl = valid_len ? static_cast<long>(__ldg(valid_len + row)) : (pos0 < 0) ? n : pos0 + row + 1;
   if (nvl > n) nvl = n;
+  if (nvl < 0) nvl = 0;
   const int nv = static_cast<int>(nvl);
   int* out = idx + row * k;
   if (nv <= k) {
@@ -592,7 +594,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
 }
 
 ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0, int k, int* idx,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, const int* valid_len) {
   if (rows == 0) return IC_OK;
   const int smem = static_cast<int>(sizeof(TopkSmem));
   ic_status st = cuda_check(
@@ -607,12 +609,14 @@ ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0,
     while (S < 8 && rows * 2 * S <= slots) S *= 2;
   }
   st = cuda_check(launch_dep(topk_kernel, dim3(static_cast<unsigned>(rows * S)), dim3(TK_THREADS),
-                             smem, stream, static_cast<unsigned>(S), scores, ld, n, pos0, k, idx),
+                             smem, stream, static_cast<unsigned>(S), scores, ld, n, pos0,
+                             valid_len, k, idx),
                   "topk_kernel launch");
   if (st) return st;
   // algorithmic bytes: every candidate score read once, the index rows written once
-  const double cand = pos0 < 0 ? static_cast<double>(rows) * n
-                               : static_cast<double>(causal_pairs(rows, n, pos0));
+  // (with per-row lengths from the device the host counts every row as n long)
+  const double cand = (pos0 < 0 || valid_len) ? static_cast<double>(rows) * n
+                                              : static_cast<double>(causal_pairs(rows, n, pos0));
   trace_launch(kKindTopk, stream, 4.0 * cand + 4.0 * static_cast<double>(rows) * k);
   return IC_OK;
 }

@@ -1,6 +1,7 @@
 """Small, fixed cases of each hot kernel, for capturing them under a profiler.
 
     python -m sparse_attention_indexer_sum_b200.profile_cases indexer_longrows
+    python -m sparse_attention_indexer_sum_b200.profile_cases indexer_longrows_e4m3
     python -m sparse_attention_indexer_sum_b200.profile_cases attn_tail4k
     python -m sparse_attention_indexer_sum_b200.profile_cases decode_indexer
     python -m sparse_attention_indexer_sum_b200.profile_cases decode_attn
@@ -13,6 +14,8 @@ name captures a warm launch. Every case fits in a few GB of device memory.
   indexer_longrows  512 query rows at causal positions 100000..100511 against
                     100512 keys (bf16, H=64, d=128, w ~ U(0,1)/8): ic_indexer_scores,
                     then ic_topk (k = 2048) on the same rows.
+  indexer_longrows_e4m3  the same rows with e4m3 inputs (per-row scales, quantised
+                    on the GPU): ic_indexer_scores alone.
   attn_tail4k       the last 4096 query rows of the 200000-token prefill workload,
                     with index sets from the indexer + top-k on those rows, then
                     ic_sparse_attn over the full 200000-row latent KV.
@@ -67,6 +70,22 @@ def indexer_longrows():
         ic.ic_indexer_scores(q, k, w, scores=scores, pos0=P0)
         ic.ic_topk(scores, 2048, pos0=P0, idx=idx)
     _rounds(rnd)
+
+
+def indexer_longrows_e4m3():
+    torch.manual_seed(0)
+    dev = "cuda"
+    R, P0 = 512, 100000
+    Lk = P0 + R
+    q = (torch.randn(R, 64, 128, device=dev) / math.sqrt(128)).to(torch.bfloat16)
+    k = (torch.randn(Lk, 128, device=dev) / math.sqrt(128)).to(torch.bfloat16)
+    q8, qs = ic.ic_quant_e4m3_rows(q)
+    k8, ks = ic.ic_quant_e4m3_rows(k)
+    w = torch.rand(R, 64, device=dev) / 8
+    scores = torch.empty(R, Lk, device=dev)
+
+    _rounds(lambda: ic.ic_indexer_scores(q8, k8, w, scores=scores, pos0=P0, q_scale=qs,
+                                         k_scale=ks))
 
 
 def attn_tail4k():
@@ -133,7 +152,8 @@ def decode_attn():
     _rounds(lambda: ic.ic_sparse_attn(q, kv, idx, wl.scale, out=out, workspace=ws))
 
 
-CASES = {"indexer_longrows": indexer_longrows, "attn_tail4k": attn_tail4k,
+CASES = {"indexer_longrows": indexer_longrows, "indexer_longrows_e4m3": indexer_longrows_e4m3,
+         "attn_tail4k": attn_tail4k,
          "decode_indexer": decode_indexer, "decode_attn": decode_attn}
 
 

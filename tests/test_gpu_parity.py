@@ -103,6 +103,23 @@ def test_topk_decode_shape_clusters_and_causal():
     np.testing.assert_array_equal(got, ref)
 
 
+def test_topk_varlen_rows_bit_exact():
+    """Per-row candidate counts from a device array: 0, 1, k-1, k, k+1, the whole
+    row, counts past the row (clamped) and random ones, on random and tied rows."""
+    k, n = 2048, 9000
+    g = torch.Generator().manual_seed(21)
+    s = torch.randn(40, n, generator=g)
+    s[3] = 0.0
+    s[4, ::3] = 1.0
+    lens = [0, 1, k - 1, k, k + 1, n, n + 50, 4321] + \
+        torch.randint(0, n + 1, (32,), generator=g).tolist()
+    vl = torch.tensor(lens, dtype=torch.int32)
+    got = ic.ic_topk_varlen(s.to(DEV), k, vl.to(DEV)).cpu().numpy()
+    _sync()
+    ref = oracle.topk(s.numpy(), k, valid=np.minimum(vl.numpy(), n))
+    np.testing.assert_array_equal(got, ref)
+
+
 @pytest.mark.parametrize("n", [1, 2047, 2048, 2049, 4096])
 def test_topk_sizes_around_k(n):
     k = 2048
