@@ -499,15 +499,19 @@ def run_decode(args, dev, peaks, barrier):
     kk = min(k, L)
     idx_b = B * L * (wl.D + 4)                      # e4m3 key cache + per-token scales
     score_b = B * L * 4 * 2 + B * kk * 4            # scores out and back in, T out
+    t_b = B * kk * 4                                # T out (fused: the scores stay on chip)
     attn_b = B * kk * wl.Dk * 2 + B * wl.Hq * (wl.Dk + wl.Dv) * 2 + B * kk * 4
 
-    def bytes_of(pat):
+    def bytes_of(pat, fused=False):
         f = sum(1 for c in pat if c == "F")
-        return f * (idx_b + score_b) + wl.layers * attn_b
+        return f * (idx_b + (t_b if fused else score_b)) + wl.layers * attn_b
 
     out = {"workload": wl.name, "batch": B, "context": L, "k": k, "pattern": wl.pattern,
-           "indexer": "e4m3 key cache + per-token f32 scales", "kv_cache": "bf16 576-d latent",
-           "l2": "inputs larger than L2 (no flush needed)"}
+           "indexer": "e4m3 key cache + per-token f32 scales",
+           "kv_cache": "bf16 576-d latent", "l2": "inputs larger than L2 (no flush needed)",
+           "algorithmic_bytes": "per F layer the e4m3 key cache and scales read, the scores "
+                                "written and read back, T written; per layer the gathered "
+                                "latent rows, q, out and T read"}
     for pat, key in ((wl.pattern, None), (allf, "all_f")):
         for _ in range(max(3, args.warmup)):
             step(pat)
@@ -564,7 +568,9 @@ def run_decode(args, dev, peaks, barrier):
                 a[2] += work
             st = {}
             for name, (n, kms, work) in sorted(agg.items()):
-                if name.startswith("indexer"):
+                if name.startswith("indexer_topk"):
+                    byt = idx_b * n                      # cache read; candidates stay on chip
+                elif name.startswith("indexer"):
                     byt = (idx_b + B * L * 4) * n        # cache read + scores written
                 elif name == "topk":
                     byt = (B * L * 4 + B * kk * 4) * n
@@ -578,6 +584,26 @@ def run_decode(args, dev, peaks, barrier):
         else:
             out[key] = r
     out["speedup_fsss_over_all_f"] = out["all_f"]["ms_per_step"] / out["ms_per_step"]
+    # the same F,S,S,S step with the indexer and the top-k fused
+    desc_u = ic.make_desc(L=L, k=k, H=wl.H, D=wl.D, idx_dtype=ic.IC_E4M3, heads=wl.Hq, dk=wl.Dk,
+                          dv=wl.Dv, attn_dtype=ic.IC_BF16, scale=wl.scale, batch=B, decode=True,
+                          flags=ic.IC_STACK_FUSED_TOPK)
+    ws_u = torch.empty(ic.ic_stack_workspace_size(desc_u) // 4 + 1, dtype=torch.float32,
+                       device=dev)
+    step_u = lambda: ic.ic_decode_step(wl.pattern, desc_u, layers, t_cache, ws_u,  # noqa: E731
+                                       stream=stream)
+    for _ in range(3):
+        step_u()
+    ic.ic_device_status(stream)
+    ms_u = _timed(step_u, steps, stream)
+    ic.ic_device_status(stream)
+    hb_f = bytes_of(wl.pattern, fused=True)
+    out["fused_topk"] = {"ms_per_step_eager": ms_u, "value": B / (ms_u * 1e-3),
+                         "hbm_bytes_per_step": hb_f,
+                         "frac_hbm": hb_f / (ms_u * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "note": "IC_STACK_FUSED_TOPK: indexer and top-k fused, the scores never "
+                                 "written; eager calls (compare with ms_per_step_eager)"}
+    del ws_u
     log("decode: %.3f ms/step (%.0f tokens/s), %.0f GB/s = %.2f of HBM; all-F %.3f ms" % (
         out["ms_per_step"], out["value"], out["achieved_gbs"], out["frac_hbm"],
         out["all_f"]["ms_per_step"]))

@@ -90,6 +90,9 @@ ic_status ic_device_status(void* stream);
 #define IC_K_ATTN_COMBINE 7
 #define IC_K_ATTN_F32 8
 #define IC_K_QUANT 9
+#define IC_K_TOPK_MERGE 10
+#define IC_K_INDEXER_TOPK_BF16 11
+#define IC_K_INDEXER_TOPK_E4M3 12
 ic_status ic_trace_begin(void* stream, int capacity);
 long ic_trace_end(float* ms, int* kinds, double* work, int capacity);
 
@@ -140,6 +143,30 @@ ic_status ic_indexer_scores(const void* q, const float* q_scale, const void* k,
  */
 ic_status ic_topk(const float* scores, long rows, int n, long ld, long pos0, int k, int* idx,
                   void* stream);
+
+/*
+ * The indexer and the top-k in one pass, for one query per sequence (the decode
+ * shape; routing loop: I <- Indexer(X); T <- top-k(I)).  For sequence b, with
+ * the query at position pos0 and the candidates s <= pos0, s < Lk:
+ *   idx[b, :] = ic_topk of the scores ic_indexer_scores would write for it
+ * -- the same fp32 scores and the same selection rule, so the index sets are
+ * identical -- but the scores are never written to memory.  The indexer's
+ * epilogue keeps, per group of keys, every key that can still be among the k
+ * largest (an exact rising threshold), leaves those candidates in `workspace`,
+ * and a second kernel selects the k largest of each sequence.
+ *   q [batch, 1, H, D], q_scale [batch, 1, H], k [batch, Lk, D], k_scale [batch, Lk],
+ *   w [batch, 1, H]: as ic_indexer_scores with rows = 1; dt = IC_BF16 or IC_E4M3
+ *   (H = 64, D = 128);
+ *   idx [batch, k_top] int32 out: ascending, -1 padded when pos0 + 1 < k_top;
+ *   workspace: device, 16-byte aligned, >= ic_indexer_topk_workspace_size bytes
+ *   (IC_ERR_WORKSPACE otherwise); its contents need no initialisation.
+ * 1 <= k_top <= 2048.  IC_F32 -> IC_ERR_UNSUPPORTED.
+ */
+ic_status ic_indexer_topk(const void* q, const float* q_scale, const void* k,
+                          const float* k_scale, const float* w, ic_dtype dt, int batch, int H,
+                          int D, int Lk, long pos0, int k_top, int* idx, void* workspace,
+                          size_t ws_bytes, void* stream);
+size_t ic_indexer_topk_workspace_size(int batch, int Lk, long pos0);
 
 /*
  * ic_topk with an arbitrary candidate count per row: row r's candidates are
@@ -255,7 +282,13 @@ typedef struct {
   int heads, dk, dv;   /* attention heads, key dim, value dim                    */
   long ld_kv;          /* row stride of kv in elements                           */
   float scale;         /* softmax scale                                          */
+  int flags;           /* IC_STACK_* bits (0 = defaults)                         */
 } ic_stack_desc;
+
+/* Decode with a tensor-core indexer: run the indexer and the top-k fused
+ * (ic_indexer_topk: the scores never leave the chip; the same index sets)
+ * instead of writing batch * L scores to the workspace and running ic_topk. */
+#define IC_STACK_FUSED_TOPK 1
 
 /*
  * The IndexCache layer stack (routing loop of "Einfache Implementierung",
@@ -310,7 +343,9 @@ ic_status ic_layer_stack_varlen(const char* pattern, const ic_stack_desc* desc,
                                 void* stream);
 
 /* Decode form of the stack (desc->decode must be 1): same routing per layer,
- * one query per sequence; t_cache is [batch, k]. */
+ * one query per sequence; t_cache is [batch, k].  With IC_STACK_FUSED_TOPK, F
+ * layers with a bf16 or e4m3 indexer run it fused with the top-k (see
+ * ic_indexer_topk). */
 ic_status ic_decode_step(const char* pattern, const ic_stack_desc* desc, const ic_layer_io* layers,
                          int nlayers, int* t_cache, void* workspace, size_t ws_bytes,
                          void* stream);

@@ -27,7 +27,8 @@ IC_F32, IC_BF16, IC_E4M3 = 0, 1, 2
 # names declared in include/ic.h (checked against the header by the tests)
 EXPORTS = ("ic_last_error", "ic_version", "ic_device_status", "ic_trace_begin", "ic_trace_end",
            "ic_quant_e4m3_rows",
-           "ic_indexer_scores", "ic_topk", "ic_topk_varlen", "ic_sparse_attn",
+           "ic_indexer_scores", "ic_indexer_topk", "ic_indexer_topk_workspace_size", "ic_topk",
+           "ic_topk_varlen", "ic_sparse_attn",
            "ic_attn_workspace_size",
            "ic_layer_stack", "ic_decode_step", "ic_stack_workspace_size",
            "ic_sparse_attn_noalloc", "ic_layer_stack_rows", "ic_layer_stack_varlen")
@@ -51,7 +52,10 @@ class ic_stack_desc(ctypes.Structure):
                 ("k", ctypes.c_int), ("idx_dtype", ctypes.c_int), ("H", ctypes.c_int),
                 ("D", ctypes.c_int), ("attn_dtype", ctypes.c_int), ("heads", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("ld_kv", ctypes.c_long),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("flags", ctypes.c_int)]
+
+
+IC_STACK_FUSED_TOPK = 1
 
 
 _lib = None
@@ -77,6 +81,9 @@ def lib() -> ctypes.CDLL:
     L.ic_trace_end.restype = Lg
     L.ic_quant_e4m3_rows.argtypes = [P, I, Lg, I, P, P, P]
     L.ic_indexer_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Lg, P, Lg, P]
+    L.ic_indexer_topk.argtypes = [P, P, P, P, P, I, I, I, I, I, Lg, I, P, P, S, P]
+    L.ic_indexer_topk_workspace_size.argtypes = [I, I, Lg]
+    L.ic_indexer_topk_workspace_size.restype = S
     L.ic_topk.argtypes = [P, Lg, I, Lg, Lg, I, P, P]
     L.ic_topk_varlen.argtypes = [P, Lg, I, Lg, P, I, P, P]
     L.ic_sparse_attn.argtypes = [P, P, Lg, P, P, I, I, I, I, I, I, I, I, F, P, P, P, S, P]
@@ -94,7 +101,7 @@ def lib() -> ctypes.CDLL:
     L.ic_stack_workspace_size.restype = S
     L.ic_sparse_attn_noalloc.argtypes = [P, P, Lg, P, P, I, I, I, I, I, I, I, I, F, P, P, P]
     for name in ("ic_device_status", "ic_quant_e4m3_rows", "ic_indexer_scores", "ic_topk",
-                 "ic_topk_varlen",
+                 "ic_topk_varlen", "ic_indexer_topk",
                  "ic_sparse_attn", "ic_layer_stack", "ic_decode_step", "ic_sparse_attn_noalloc",
                  "ic_layer_stack_rows", "ic_layer_stack_varlen"):
         getattr(L, name).restype = I
@@ -151,7 +158,8 @@ def ic_device_status(stream=None):
 
 
 KIND_NAMES = {1: "indexer_tc_bf16", 2: "indexer_tc_e4m3", 3: "indexer_f32", 4: "fill_masked",
-              5: "topk", 6: "attn_mla", 7: "attn_combine", 8: "attn_f32", 9: "quant_e4m3"}
+              5: "topk", 6: "attn_mla", 7: "attn_combine", 8: "attn_f32", 9: "quant_e4m3",
+              10: "topk_merge", 11: "indexer_topk_bf16", 12: "indexer_topk_e4m3"}
 
 
 def ic_trace_begin(capacity: int = 4096, stream=None):
@@ -205,6 +213,29 @@ def ic_indexer_scores(q, k, w, scores=None, *, pos0: int = 0, q_scale=None, k_sc
     _check(lib().ic_indexer_scores(_p(q), _p(q_scale), _p(k), _p(k_scale), _p(w), dtype_code(q),
                                    B, H, D, R, Lk, int(pos0), _p(scores), ld, _stream(stream)))
     return scores
+
+
+def ic_indexer_topk_workspace_size(batch: int, Lk: int, pos0: int) -> int:
+    return int(lib().ic_indexer_topk_workspace_size(int(batch), int(Lk), int(pos0)))
+
+
+def ic_indexer_topk(q, k, w, k_top: int, workspace, *, pos0: int, q_scale=None, k_scale=None,
+                    idx=None, stream=None):
+    """Indexer and top-k in one pass for one query per sequence: q [B,1,H,D],
+    k [B,Lk,D], w [B,1,H] (e4m3 codes take q_scale [B,1,H], k_scale [B,Lk]); returns
+    idx [B, k_top] int32.  The scores are never written."""
+    _contig(q, k, w, q_scale, k_scale)
+    if q.dim() != 4 or q.shape[1] != 1:
+        raise ValueError("q must be [B, 1, H, D]")
+    B, _, H, D = q.shape
+    Lk = k.shape[-2]
+    if idx is None:
+        idx = torch.empty((B, k_top), dtype=torch.int32, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().ic_indexer_topk(_p(q), _p(q_scale), _p(k), _p(k_scale), _p(w), dtype_code(q), B,
+                                 H, D, Lk, int(pos0), int(k_top), _p(idx), _p(workspace),
+                                 ws_bytes, _stream(stream)))
+    return idx
 
 
 def ic_topk(scores, k: int, *, n: int | None = None, pos0: int = -1, idx=None, stream=None):
@@ -297,10 +328,10 @@ def ic_sparse_attn_noalloc(q, kv, idx, scale: float, *, out, dv: int = 512, lse=
 
 
 def make_desc(*, L, k, H, D, idx_dtype, heads, dk, dv, attn_dtype, scale, ld_kv=None, batch=1,
-              decode=False) -> ic_stack_desc:
+              decode=False, flags=0) -> ic_stack_desc:
     return ic_stack_desc(L=L, batch=batch, decode=int(bool(decode)), k=k, idx_dtype=idx_dtype, H=H,
                          D=D, attn_dtype=attn_dtype, heads=heads, dk=dk, dv=dv,
-                         ld_kv=dk if ld_kv is None else ld_kv, scale=scale)
+                         ld_kv=dk if ld_kv is None else ld_kv, scale=scale, flags=flags)
 
 
 def ic_stack_workspace_size(desc: ic_stack_desc) -> int:

@@ -209,9 +209,17 @@ static ic_status run_stack(const char* pattern, const ic_stack_desc* d, const ic
   const size_t qrow_b = static_cast<size_t>(d->H) * d->D * elem_bytes(d->idx_dtype);
   const size_t krow_b = static_cast<size_t>(d->D) * elem_bytes(d->idx_dtype);
 
+  // decode with a tensor-core indexer: indexer and top-k fused (no score rows)
+  const bool fused = decode && d->idx_dtype != IC_F32 && (d->flags & IC_STACK_FUSED_TOPK);
+  if (fused) {
+    const size_t need = indexer_topk_fused_ws_bytes(B, d->L, d->L - 1);
+    if (!workspace || ws_bytes < need)
+      return fail(IC_ERR_WORKSPACE, "decode: the fused indexer/top-k needs %zu workspace bytes "
+                  "(got %zu)", need, ws_bytes);
+  }
   // rows of scores per block: prefill streams query rows, decode streams sequences
   const long units = decode ? B : R;
-  const long rb = score_rows(ws_bytes, d->L, units);
+  const long rb = fused ? units : score_rows(ws_bytes, d->L, units);
   if (!workspace || rb < 1)
     return fail(IC_ERR_WORKSPACE, "stack: workspace of %zu bytes holds no score row of %d floats",
                 ws_bytes, d->L);
@@ -219,7 +227,13 @@ static ic_status run_stack(const char* pattern, const ic_stack_desc* d, const ic
 
   for (int l = 0; l < nlayers; ++l) {
     const ic_layer_io& io = layers[l];
-    if (kinds[l] == 'F') {
+    if (kinds[l] == 'F' && fused) {
+      // T_cache <- top-k(Indexer_l(X)) in one pass over the key cache
+      st = launch_indexer_topk_fused(d->idx_dtype == IC_E4M3, io.q_idx, io.q_scale, io.k_idx,
+                                     io.k_scale, io.w, B, d->L, d->L - 1, d->k, t_cache,
+                                     workspace, ws_bytes, stream);
+      if (st) return st;
+    } else if (kinds[l] == 'F') {
       // T_cache <- top-k(Indexer_l(X)), one block of score rows at a time
       for (long u0 = 0; u0 < units; u0 += rb) {
         const long nu = (units - u0 < rb) ? units - u0 : rb;
@@ -267,7 +281,7 @@ extern "C" {
 
 const char* ic_last_error(void) { return t_last_error.c_str(); }
 
-int ic_version(void) { return 100; }
+int ic_version(void) { return 101; }
 
 ic_status ic_device_status(void* stream) {
   ic_status st = cuda_check(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)),
@@ -357,6 +371,28 @@ ic_status ic_topk(const float* scores, long rows, int n, long ld, long pos0, int
     return fail(IC_ERR_INVALID_ARG, "topk: bad sizes (rows %ld n %d ld %ld k %d)", rows, n, ld, k);
   if (rows > 0x7fffffffL) return fail(IC_ERR_UNSUPPORTED, "topk: too many rows");
   return launch_topk(scores, rows, n, ld, pos0, k, idx, static_cast<cudaStream_t>(stream));
+}
+
+ic_status ic_indexer_topk(const void* q, const float* q_scale, const void* k,
+                          const float* k_scale, const float* w, ic_dtype dt, int batch, int H,
+                          int D, int Lk, long pos0, int k_top, int* idx, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  if (dt != IC_BF16 && dt != IC_E4M3)
+    return fail(IC_ERR_UNSUPPORTED, "indexer_topk: needs the tensor-core indexer (bf16 or e4m3)");
+  ic_status st = check_indexer(q, q_scale, k, k_scale, w, dt, batch, H, D, 1, Lk, pos0, nullptr,
+                               Lk, false);
+  if (st) return st;
+  if (!idx) return fail(IC_ERR_INVALID_ARG, "indexer_topk: idx is NULL");
+  if (k_top < 1 || k_top > 2048)
+    return fail(IC_ERR_INVALID_ARG, "indexer_topk: k must be in [1, 2048] (got %d)", k_top);
+  return launch_indexer_topk_fused(dt == IC_E4M3, q, q_scale, k, k_scale, w, batch, Lk, pos0,
+                                   k_top, idx, workspace, ws_bytes,
+                                   static_cast<cudaStream_t>(stream));
+}
+
+size_t ic_indexer_topk_workspace_size(int batch, int Lk, long pos0) {
+  if (batch < 1 || Lk < 1 || pos0 < 0) return 0;
+  return indexer_topk_fused_ws_bytes(batch, Lk, pos0);
 }
 
 ic_status ic_topk_varlen(const float* scores, long rows, int n, long ld, const int* valid_len,
@@ -462,6 +498,8 @@ size_t ic_stack_workspace_size(const ic_stack_desc* d) {
   const long units = d->decode ? d->batch : d->L;
   const long want = d->decode ? units : (units < 4096 ? units : 4096);
   size_t s = static_cast<size_t>(want) * d->L * sizeof(float);
+  if (d->decode && d->idx_dtype != IC_F32 && (d->flags & IC_STACK_FUSED_TOPK))
+    s = indexer_topk_fused_ws_bytes(d->batch, d->L, d->L - 1);
   if (d->decode && d->attn_dtype == IC_BF16) {
     const size_t a = attn_mla_ws_bytes(d->batch, 1, d->k);
     if (a > s) s = a;

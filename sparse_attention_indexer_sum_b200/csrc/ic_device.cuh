@@ -205,6 +205,22 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t a_fmt, uint32_t b_f
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// Order-preserving key of an fp32 score: a > b as floats <=> key(a) > key(b) as
+// unsigned; -0 maps to +0, so the two compare equal.
+__device__ __forceinline__ uint32_t score_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Selection key of (score, index): the score's key in the high word and the
+// complemented index in the low word, so that a larger key means a larger score
+// or, for equal scores, a lower index -- the top-k order, and no two keys of a
+// row are equal.
+__device__ __forceinline__ uint64_t select_key(float score, uint32_t index) {
+  return (static_cast<uint64_t>(score_key(score)) << 32) | static_cast<uint64_t>(~index);
+}
+
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return __shfl_sync(0xffffffffu, threadIdx.x / 32, 0); }
 

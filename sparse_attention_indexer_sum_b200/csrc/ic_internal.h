@@ -53,6 +53,9 @@ enum LaunchKind : int {
   kKindAttnCombine = 7,
   kKindAttnF32 = 8,
   kKindQuant = 9,
+  kKindTopkMerge = 10,
+  kKindIndexerTopkBf16 = 11,
+  kKindIndexerTopkE4m3 = 12,
 };
 // Called after every kernel launch: when tracing is on for this host thread,
 // records an event on `stream` with the launch's kind and algorithmic work
@@ -70,6 +73,17 @@ ic_status launch_indexer_tc(bool fp8, const void* q, const float* q_scale, const
 ic_status launch_indexer_f32(const float* q, const float* k, const float* w, int batch, int H,
                              int D, int rows, int Lk, long pos0, float* scores, long ld,
                              cudaStream_t stream);
+// Fused indexer -> top-k for batch sequences of one query each (at position pos0,
+// keys 0..Lk-1): the indexer kernel keeps each row's candidates in workspace slots
+// (never writing the scores), then topk_merge_kernel writes idx [batch, topk].
+ic_status launch_indexer_topk_fused(bool fp8, const void* q, const float* q_scale, const void* k,
+                                    const float* k_scale, const float* w, int batch, int Lk,
+                                    long pos0, int topk, int* idx, void* ws, size_t ws_bytes,
+                                    cudaStream_t stream);
+size_t indexer_topk_fused_ws_bytes(int batch, int Lk, long pos0);
+ic_status launch_topk_merge(const uint8_t* slots, long rows, long nt, long total, int G, int maxp,
+                            int nsets, size_t slot_bytes, int cb, int nv, int k, int* idx,
+                            cudaStream_t stream);
 // valid_len (device int32 [rows], or NULL): row r's candidate count, clamped to
 // [0, n]; NULL means min(n, pos0 + r + 1), or n when pos0 < 0.
 ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0, int k, int* idx,

@@ -49,9 +49,22 @@ struct IdxTcArgs {
   int qb_per_batch;      // ceil(R / TPM)
   int nqb;               // B * qb_per_batch
   long total_tiles;
+  // Fused top-k (one query per sequence): every (row, CTA piece, epilogue set)
+  // leaves its candidates in a slot of `cslots`; topk_merge_kernel selects.
+  uint8_t* cslots;
+  int maxp;              // CTA pieces per row (slots per row = maxp * NSETS)
+  int topk;              // k of the selection
 };
 
-template <bool FP8, int TPM>
+// Fused top-k slot: a 64-byte header {int count; int pad; uint64 tau} and then
+// `count` selection keys (select_key) of one epilogue set's share of one row's
+// keys in one CTA: every key of that share with selection key >= tau; when tau
+// is not 0, at least k of them.
+constexpr int FUSED_CB = 4096;                         // candidate buffer per set
+constexpr size_t FUSED_SLOT_BYTES = 64 + 8 * FUSED_CB;
+constexpr int FUSED_NSETS = 3;                         // epilogue sets of the TPM = 1 instance
+
+template <bool FP8, int TPM, bool FUSED = false>
 struct IdxCfg {
   static constexpr int H = 64, D = 128;
   static constexpr int BM = 128;                   // keys per tile (MMA M)
@@ -63,7 +76,8 @@ struct IdxCfg {
   static constexpr int KSTEPS = FP8 ? 4 : 8;       // MMAs per tile (K = 32 / 16 each)
   static constexpr int A_BYTES = BM * ROWB;        // one key tile
   static constexpr int Q_BYTES = N * ROWB;         // the query block
-  static constexpr int STAGES = FP8 ? 8 : 4;
+  // the fused top-k's candidate buffers take the shared memory of some ring stages
+  static constexpr int STAGES = FUSED ? (FP8 ? 6 : 2) : (FP8 ? 8 : 4);
   static constexpr int NACC = (TPM == 4) ? 2 : 6;  // TMEM accumulators in the ring
   static constexpr int TMEM_COLS = (NACC * N <= 256) ? 256 : 512;
   static constexpr int EPG = (TPM == 4) ? 2 : 1;   // epilogue warps per TMEM lane quadrant
@@ -79,6 +93,13 @@ struct IdxCfg {
   // issue loop (waits, MMAs, commits) sets the pace; two threads alternate
   // tiles.  With N = 256 the tensor pipe itself is the limit.
   static constexpr int MMAW = (TPM == 1) ? 2 : 1;
+  // Each MMA warp must wait on every phase of the full barriers of the stages it
+  // reads: with STAGES a multiple of MMAW, all uses of a stage fall to the same
+  // warp.  Otherwise a warp waits on parity p two phases apart while the other
+  // warp's phase in between may not have completed yet, and the parity test
+  // passes on the older phase (the ring would run ahead of its data).
+  static_assert(STAGES % MMAW == 0, "every use of a ring stage falls to one MMA warp");
+  static_assert(NACC % MMAW == 0, "every use of an accumulator falls to one MMA warp");
   static constexpr int EPI_W0 = 1 + MMAW;  // first epilogue warp
   static constexpr int THREADS = 32 * (EPI_W0 + NEPI);
   // TMEM columns an epilogue thread loads at a time: 16, so that the head
@@ -90,8 +111,16 @@ struct IdxCfg {
   static constexpr int W_FLOATS = NEPI * TOK_PER_EW * 64;
   static constexpr int OFF_BAR = OFF_W + W_FLOATS * 4;
   static constexpr int NBAR = 2 * STAGES + 2 * NACC + 3;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  // fused top-k: per epilogue set, a buffer of FUSED_CB selection keys, a 256-bin
+  // radix histogram and 64 ints of scratch
+  static constexpr int CB = FUSED ? FUSED_CB : 0;
+  static constexpr int OFF_CBUF = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;
+  static constexpr int OFF_CHIST = OFF_CBUF + NSETS * CB * 8;
+  static constexpr int OFF_CX = OFF_CHIST + (FUSED ? NSETS * 256 * 4 : 0);
+  static constexpr int OFF_MISC = OFF_CX + (FUSED ? NSETS * 64 * 4 : 0);
   static constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;  // + alignment slack
+  static_assert(!FUSED || (TPM == 1 && NSETS == FUSED_NSETS && SETW == 4),
+                "the fused top-k runs in the one-token instance, 3 sets of 4 warps");
   static_assert(A_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0, "swizzle atoms need 1 KB alignment");
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -126,11 +155,219 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
   (void)mbar_wait(bar, parity, &never, kErrTimeoutDrain);
 }
 
-template <bool FP8, int TPM>
-__global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
+// ------------------------------------------------------------------ fused top-k
+// Each epilogue set (4 warps, one thread per key of a tile) keeps, for the row it
+// is working on, a shared-memory buffer of selection keys with a rising
+// threshold tau: a key of the set's tiles enters when its selection key is >=
+// tau; when the buffer fills up, a radix descent finds a new tau with at least k
+// and at most `target` buffered keys >= tau, and the buffer is compacted to
+// those.  Keys below tau have at least k larger keys in the same set's share of
+// the row, so they cannot be among the row's top k: the buffer always holds
+// every candidate.  At the end of the row (or of the CTA's work) the buffer goes
+// to its slot in global memory.
+//
+// The 4 warps of a set meet on a named barrier (one id per set).  Every warp
+// reaches every barrier: the only wait on another role (the accumulator) is
+// bounded, and a warp whose wait gave up raises the set's `dead` flag and still
+// arrives; the set reads the flag right after the barrier and leaves together.
+struct CandSet {
+  uint64_t* buf;   // [FUSED_CB]
+  uint32_t* hist;  // [256]
+  int* x;          // [64]: 0..7 warp sums and 8..15 chosen bin (by round parity), 16..19
+                   // survivor counts, 20..27 per-tile counts, 30 dead flag, 32..47
+                   // per-warp min and max (as 8 uint64)
+  int bar_id;
+  // The warp reconverges first, and the barrier is the non-aligned form, which
+  // counts threads one by one: the set's barriers follow lane-0-only stores.
+  __device__ __forceinline__ void sync() const {
+    __syncwarp();
+    asm volatile("barrier.sync %0, %1;" ::"r"(bar_id), "r"(128) : "memory");
+  }
+  __device__ __forceinline__ uint64_t* mm() const { return reinterpret_cast<uint64_t*>(x + 32); }
+};
+
+// Min and max of the buffered keys over the set (every thread gets them).
+__device__ __forceinline__ void cand_minmax(const CandSet& cs, int cnt, int t, uint64_t& mn,
+                                            uint64_t& mx) {
+  const int lane = t & 31, wid = t >> 5;
+  mn = ~0ull;
+  mx = 0ull;
+  for (int i = t; i < cnt; i += 128) {
+    const uint64_t c = cs.buf[i];
+    mn = c < mn ? c : mn;
+    mx = c > mx ? c : mx;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t a = __shfl_xor_sync(0xffffffffu, mn, o);
+    const uint64_t b = __shfl_xor_sync(0xffffffffu, mx, o);
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
+  }
+  if (lane == 0) {
+    cs.mm()[wid] = mn;
+    cs.mm()[4 + wid] = mx;
+  }
+  cs.sync();
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const uint64_t a = cs.mm()[w], b = cs.mm()[4 + w];
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
+  }
+}
+
+// The new threshold and the compaction.  Every thread of the set calls it with the
+// same cnt and tau (kept in registers, identical in every thread) and t = its
+// index in the set (0..127).  Thread t holds buffer entries t + 128 j (j < 32) in
+// registers for the whole call: the buffer is read once, the radix rounds start
+// below the bits that every buffered key shares (8-bit digits, one shared atomic
+// per distinct bin per warp), and the survivors are written back from registers.
+constexpr int CAND_PER_THREAD = FUSED_CB / 128;
+__device__ __forceinline__ void cand_compact(const CandSet cs, int& cnt_io, uint64_t& tau, int k,
+                                          int target, int t) {
+  const int lane = t & 31, wid = t >> 5;
+  const int cnt = cnt_io;
+  cs.sync();  // this tile's keys are in the buffer
+  uint64_t c[CAND_PER_THREAD];
+  uint64_t mn = ~0ull, mx = 0ull;
+#pragma unroll
+  for (int j = 0; j < CAND_PER_THREAD; ++j) {
+    const int i = t + 128 * j;
+    c[j] = (i < cnt) ? cs.buf[i] : 0ull;
+    if (i < cnt) {
+      mn = c[j] < mn ? c[j] : mn;
+      mx = c[j] > mx ? c[j] : mx;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t a = __shfl_xor_sync(0xffffffffu, mn, o);
+    const uint64_t b = __shfl_xor_sync(0xffffffffu, mx, o);
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
+  }
+  if (lane == 0) {
+    cs.mm()[wid] = mn;
+    cs.mm()[4 + wid] = mx;
+  }
+  cs.hist[t] = 0u;
+  cs.hist[t + 128] = 0u;
+  cs.sync();
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const uint64_t a = cs.mm()[w], b = cs.mm()[4 + w];
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
+  }
+  int pbits = (mn == mx) ? 63 : __clzll(static_cast<long long>(mn ^ mx));
+  uint64_t prefix = pbits == 0 ? 0ull : (mn >> (64 - pbits));
+  int need = k, above = 0;
+  uint64_t tnew;
+  for (int round = 0;; ++round) {
+    const int bits = (64 - pbits) < 8 ? 64 - pbits : 8;
+    const int shift = 64 - pbits - bits;
+    if (round > 0) {  // the first round's bins were cleared above
+      cs.hist[t] = 0u;
+      cs.hist[t + 128] = 0u;
+      cs.sync();
+    }
+#pragma unroll
+    for (int j = 0; j < CAND_PER_THREAD; ++j) {
+      int bin = -1;
+      if (t + 128 * j < cnt && (pbits == 0 || (c[j] >> (64 - pbits)) == prefix))
+        bin = static_cast<int>((c[j] >> shift) & ((1ull << bits) - 1ull));
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cs.hist[bin], __popc(peers));
+    }
+    cs.sync();
+    // thread t owns bins 2t and 2t + 1; count the keys in higher bins
+    const int h1 = static_cast<int>(cs.hist[2 * t + 1]), h0 = static_cast<int>(cs.hist[2 * t]);
+    const int v = h0 + h1;
+    int incl = v;  // sum over lanes >= this lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += y;
+    }
+    if (lane == 0) cs.x[4 * (round & 1) + wid] = incl;
+    cs.sync();
+    int higher = 0;
+    for (int w = wid + 1; w < 4; ++w) higher += cs.x[4 * (round & 1) + w];
+    const int gt1 = higher + incl - v, gt0 = gt1 + h1;
+    int* xb = cs.x + 8 + 4 * (round & 1);  // the chosen bin, by round parity
+    if (gt1 < need && need <= gt1 + h1) {
+      xb[0] = 2 * t + 1;
+      xb[1] = gt1;
+      xb[2] = h1;
+    }
+    if (gt0 < need && need <= gt0 + h0) {
+      xb[0] = 2 * t;
+      xb[1] = gt0;
+      xb[2] = h0;
+    }
+    cs.sync();
+    const uint64_t pre = (prefix << bits) | static_cast<uint64_t>(xb[0]);
+    const int gt = xb[1], inb = xb[2];
+    pbits += bits;
+    if (above + gt + inb <= target || pbits == 64) {  // keys >= the bin's lower edge
+      tnew = pbits == 64 ? pre : pre << (64 - pbits);
+      break;
+    }
+    above += gt;
+    need -= gt;
+    prefix = pre;
+  }
+  // the survivors, written back from registers (every read is done: the barriers
+  // of the rounds come after them)
+  int kept = 0;
+#pragma unroll
+  for (int j = 0; j < CAND_PER_THREAD; ++j) kept += (t + 128 * j < cnt && c[j] >= tnew) ? 1 : 0;
+  int incl = kept;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) cs.x[16 + wid] = incl;
+  cs.sync();
+  int base = incl - kept, total = 0;
+  for (int w = 0; w < 4; ++w) {
+    const int n = cs.x[16 + w];
+    base += (w < wid) ? n : 0;
+    total += n;
+  }
+#pragma unroll
+  for (int j = 0; j < CAND_PER_THREAD; ++j)
+    if (t + 128 * j < cnt && c[j] >= tnew) cs.buf[base++] = c[j];
+  cnt_io = total;
+  if (tnew > tau) tau = tnew;
+  cs.sync();
+}
+
+// Writes the set's buffer to its slot (header: count, tau, largest key) and
+// empties it.
+__device__ __forceinline__ void cand_flush(const CandSet& cs, int& cnt, uint64_t& tau,
+                                           uint8_t* slot, int t) {
+  cs.sync();  // the last tile's keys are in the buffer
+  uint64_t mn, mx;
+  cand_minmax(cs, cnt, t, mn, mx);
+  uint64_t* dst = reinterpret_cast<uint64_t*>(slot + 64);
+  for (int i = t; i < cnt; i += 128) dst[i] = cs.buf[i];
+  if (t == 0) {
+    *reinterpret_cast<int*>(slot) = cnt;
+    *reinterpret_cast<uint64_t*>(slot + 8) = tau;
+    *reinterpret_cast<uint64_t*>(slot + 16) = mx;
+  }
+  cnt = 0;
+  tau = 0;
+}
+
+template <bool FP8, int TPM, bool FUSED>
+__global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmQ, const IdxTcArgs a) {
-  using C = IdxCfg<FP8, TPM>;
+  using C = IdxCfg<FP8, TPM, FUSED>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -170,6 +407,9 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
       mbar_init(qfull_bar, 1);
       mbar_init(qempty_bar, C::MMAW);
       mbar_init(mmadone_bar, C::MMAW);
+      if constexpr (FUSED)
+        for (int j = 0; j < C::NSETS; ++j)
+          reinterpret_cast<int*>(smem + C::OFF_CX)[64 * j + 30] = 0;  // the sets' dead flags
       *abort_flag = 0;
       fence_barrier_init();
       fence_proxy_async_smem();
@@ -335,7 +575,33 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
       for (int t = 0; t < C::TOK_PER_EW; ++t)
 #pragma unroll
         for (int h = 0; h < 64; ++h) wr[t][h] = 0.f;
+      // fused top-k state of this set (identical in its 128 threads)
+      const int swid = e % 4, st = swid * 32 + lane;  // warp and thread index in the set
+      CandSet cs{};
+      int ccnt = 0, tpar = 0, crow = -1;
+      uint64_t ctau = 0;
+      long crow_first = 0;  // first CTA of the current row
+      bool dead = false;
+      if constexpr (FUSED) {
+        cs.buf = reinterpret_cast<uint64_t*>(smem + C::OFF_CBUF) + set * C::CB;
+        cs.hist = reinterpret_cast<uint32_t*>(smem + C::OFF_CHIST) + set * 256;
+        cs.x = reinterpret_cast<int*>(smem + C::OFF_CX) + set * 64;
+        cs.bar_id = 1 + set;
+      }
+      auto slot_of = [&](int row) {
+        const long piece = static_cast<long>(blockIdx.x) - crow_first;
+        return a.cslots + ((static_cast<long>(row) * a.maxp + piece) * C::NSETS + set) *
+                              static_cast<long>(FUSED_SLOT_BYTES);
+      };
       for (long i = 0; i < nitems; ++i) {
+        if constexpr (FUSED) {
+          // every set walks every item, so all of them see each row change
+          if (it.qb != crow) {
+            if (crow >= 0) cand_flush(cs, ccnt, ctau, slot_of(crow), st);
+            crow = it.qb;
+            crow_first = ((g0 + i - it.kt) * gridDim.x + gridDim.x - 1) / a.total_tiles;
+          }
+        }
         if (C::NSETS > 1 && acc % C::NSETS != set) {  // another set's slot
           if (++acc == C::NACC) {
             acc = 0;
@@ -359,10 +625,12 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
             wsl[x] = v;
           }
           __syncwarp();
+          if constexpr (!FUSED) {
 #pragma unroll
-          for (int t = 0; t < C::TOK_PER_EW; ++t)
+            for (int t = 0; t < C::TOK_PER_EW; ++t)
 #pragma unroll
-            for (int h = 0; h < 64; ++h) wr[t][h] = wsl[t * 64 + h];
+              for (int h = 0; h < 64; ++h) wr[t][h] = wsl[t * 64 + h];
+          }
           cur_qb = it.qb;
         }
         // this lane's key; its fp8 scale is fetched before the wait so the load's
@@ -371,9 +639,13 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
         const bool key_ok = s < a.Lk && b < a.B;
         float ks = 1.f;
         if constexpr (FP8) ks = key_ok ? a.k_scale[static_cast<long>(b) * a.Lk + s] : 0.f;
-        if (!mbar_wait(accfull_bar(acc), aph, abort_flag, kErrTimeoutEpilogue)) break;
+        // every lane leaves together, so the warp never splits before tcgen05.ld
+        const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(accfull_bar(acc), aph, abort_flag,
+                                                              kErrTimeoutEpilogue));
+        if (!FUSED && !acc_ok) break;
+        float res[C::TOK_PER_EW] = {};
+        if (acc_ok) {
         tc_fence_after();
-        float res[C::TOK_PER_EW];
 #pragma unroll
         for (int tk = 0; tk < C::TOK_PER_EW; ++tk) {
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
@@ -387,7 +659,11 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
 #pragma unroll
             for (int h4 = 0; h4 < C::EPI_COLS / 4; ++h4) {
               const int h = C::EPI_COLS * part + 4 * h4;
-              const float4 wv = make_float4(wr[tk][h], wr[tk][h + 1], wr[tk][h + 2], wr[tk][h + 3]);
+              // the fused instance reads the weights from the warp's shared copy (one
+              // broadcast load per 4 heads), leaving the registers to the selection
+              const float4 wv =
+                  FUSED ? *reinterpret_cast<const float4*>(wsl + tk * 64 + h)
+                        : make_float4(wr[tk][h], wr[tk][h + 1], wr[tk][h + 2], wr[tk][h + 3]);
               s0 = fmaf(wv.x, fmaxf(v[4 * h4 + 0], 0.f), s0);
               s1 = fmaf(wv.y, fmaxf(v[4 * h4 + 1], 0.f), s1);
               s2 = fmaf(wv.z, fmaxf(v[4 * h4 + 2], 0.f), s2);
@@ -399,7 +675,34 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(accempty_bar(acc));
-        if (key_ok) {
+        }  // acc_ok
+        if constexpr (FUSED) {
+          // one query per sequence: row b, position pos0; the same fp32 score as the
+          // unfused store, as a selection key, offered to the set's buffer
+          const uint64_t ck = select_key(res[0] * ks, static_cast<uint32_t>(s));
+          const bool cand = acc_ok && key_ok && s <= a.pos0 && ck >= ctau;
+          const unsigned m = __ballot_sync(0xffffffffu, cand);
+          if (lane == 0) {
+            cs.x[20 + 4 * tpar + swid] = __popc(m);
+            if (!acc_ok) cs.x[30] = 1;
+          }
+          cs.sync();
+          if (cs.x[30]) {  // a wait of this set gave up: the set leaves together
+            dead = true;
+            break;
+          }
+          int off = 0, tot = 0;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int n = cs.x[20 + 4 * tpar + w];
+            off += (w < swid) ? n : 0;
+            tot += n;
+          }
+          tpar ^= 1;
+          if (cand) cs.buf[ccnt + off + __popc(m & ((1u << lane) - 1u))] = ck;
+          ccnt += tot;
+          if (ccnt > FUSED_CB - 128) cand_compact(cs, ccnt, ctau, a.topk, FUSED_CB - 1280, st);
+        } else if (key_ok) {
 #pragma unroll
           for (int tk = 0; tk < C::TOK_PER_EW; ++tk) {
             const int r = r0 + tk;
@@ -415,6 +718,10 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM>::THREADS, 1)
           aph ^= 1;
         }
         it.advance(a);
+      }
+      if constexpr (FUSED) {
+        // the last row's candidates (after an abort the results are void anyway)
+        if (crow >= 0 && !dead) cand_flush(cs, ccnt, ctau, slot_of(crow), st);
       }
     }
   }
@@ -477,11 +784,12 @@ long long causal_pairs(long R, long Lk, long pos0) {
   return n;
 }
 
-template <bool FP8, int TPM>
+template <bool FP8, int TPM, bool FUSED = false>
 static ic_status launch_tpl(const void* q, const float* q_scale, const void* k,
                             const float* k_scale, const float* w, int batch, int rows, int Lk,
-                            long pos0, float* scores, long ld, cudaStream_t stream) {
-  using C = IdxCfg<FP8, TPM>;
+                            long pos0, float* scores, long ld, cudaStream_t stream,
+                            uint8_t* cslots = nullptr, int maxp = 0, int topk = 0) {
+  using C = IdxCfg<FP8, TPM, FUSED>;
   IdxTcArgs a;
   a.w = w;
   a.q_scale = q_scale;
@@ -494,6 +802,9 @@ static ic_status launch_tpl(const void* q, const float* q_scale, const void* k,
   a.pos0 = pos0;
   a.qb_per_batch = (rows + TPM - 1) / TPM;
   a.nqb = batch * a.qb_per_batch;
+  a.cslots = cslots;
+  a.maxp = maxp;
+  a.topk = topk;
   long total = 0;
   for (int qb = 0; qb < a.qb_per_batch; ++qb) total += qb_tiles<TPM>(a, qb);
   total *= batch;  // every batch has the same triangle
@@ -506,18 +817,72 @@ static ic_status launch_tpl(const void* q, const float* q_scale, const void* k,
   st = make_map(&tmQ, q, FP8, static_cast<uint64_t>(batch) * rows * 64, C::N);
   if (st) return st;
 
-  st = cuda_check(cudaFuncSetAttribute(indexer_tc_kernel<FP8, TPM>,
+  st = cuda_check(cudaFuncSetAttribute(indexer_tc_kernel<FP8, TPM, FUSED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
                   "cudaFuncSetAttribute(indexer)");
   if (st) return st;
   const long grid = total < num_sms() ? total : num_sms();
-  st = cuda_check(launch_dep(indexer_tc_kernel<FP8, TPM>, dim3(static_cast<unsigned>(grid)),
+  st = cuda_check(launch_dep(indexer_tc_kernel<FP8, TPM, FUSED>, dim3(static_cast<unsigned>(grid)),
                              dim3(C::THREADS), C::SMEM_BYTES, stream, 1, tmK, tmQ, a),
                   "indexer_tc_kernel launch");
   if (st) return st;
-  trace_launch(FP8 ? kKindIndexerE4m3 : kKindIndexerBf16, stream,
+  const int kind = FUSED ? (FP8 ? kKindIndexerTopkE4m3 : kKindIndexerTopkBf16)
+                         : (FP8 ? kKindIndexerE4m3 : kKindIndexerBf16);
+  trace_launch(kind, stream,
                2.0 * 64 * 128 * static_cast<double>(causal_pairs(rows, Lk, pos0)) * batch);
   return IC_OK;
+}
+
+// Plan of the fused indexer -> top-k for `batch` sequences of one query each at
+// position pos0 over Lk keys: nt key tiles per row, total = batch * nt tiles cut
+// into G equal contiguous CTA shares (as the kernel cuts them), and the most CTA
+// pieces any row is split into.
+struct FusedPlan {
+  long nt, total;
+  int G, maxp;
+};
+static FusedPlan fused_plan(int batch, int Lk, long pos0) {
+  FusedPlan p{0, 0, 0, 0};
+  const long keys = pos0 + 1 < Lk ? pos0 + 1 : Lk;
+  p.nt = (keys + 127) / 128;
+  p.total = static_cast<long>(batch) * p.nt;
+  if (p.total == 0) return p;
+  const long sms = num_sms();
+  p.G = static_cast<int>(p.total < sms ? p.total : sms);
+  auto cta_of = [&](long t) { return (t * p.G + p.G - 1) / p.total; };
+  for (long b = 0; b < batch; ++b) {
+    const long np = cta_of(b * p.nt + p.nt - 1) - cta_of(b * p.nt) + 1;
+    if (np > p.maxp) p.maxp = static_cast<int>(np);
+  }
+  return p;
+}
+
+size_t indexer_topk_fused_ws_bytes(int batch, int Lk, long pos0) {
+  const FusedPlan p = fused_plan(batch, Lk, pos0);
+  return static_cast<size_t>(batch) * p.maxp * FUSED_NSETS * FUSED_SLOT_BYTES;
+}
+
+ic_status launch_indexer_topk_fused(bool fp8, const void* q, const float* q_scale, const void* k,
+                                    const float* k_scale, const float* w, int batch, int Lk,
+                                    long pos0, int topk, int* idx, void* ws, size_t ws_bytes,
+                                    cudaStream_t stream) {
+  const FusedPlan p = fused_plan(batch, Lk, pos0);
+  const long nv = pos0 + 1 < Lk ? pos0 + 1 : Lk;
+  uint8_t* slots = static_cast<uint8_t*>(ws);
+  if (nv > topk) {  // otherwise every candidate is selected: the merge alone writes T
+    const size_t need = static_cast<size_t>(batch) * p.maxp * FUSED_NSETS * FUSED_SLOT_BYTES;
+    if (!ws || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % 16 != 0)
+      return fail(IC_ERR_WORKSPACE,
+                  "indexer_topk: needs a 16-byte aligned workspace of %zu bytes (got %zu)", need,
+                  ws_bytes);
+    ic_status st = fp8 ? launch_tpl<true, 1, true>(q, q_scale, k, k_scale, w, batch, 1, Lk, pos0,
+                                                   nullptr, Lk, stream, slots, p.maxp, topk)
+                       : launch_tpl<false, 1, true>(q, q_scale, k, k_scale, w, batch, 1, Lk,
+                                                    pos0, nullptr, Lk, stream, slots, p.maxp, topk);
+    if (st) return st;
+  }
+  return launch_topk_merge(slots, batch, p.nt, p.total, p.G, p.maxp, FUSED_NSETS,
+                           FUSED_SLOT_BYTES, FUSED_CB, static_cast<int>(nv), topk, idx, stream);
 }
 
 ic_status launch_indexer_tc(bool fp8, const void* q, const float* q_scale, const void* k,

@@ -55,13 +55,6 @@ struct TopkSmem {
   int counter, ties;
 };
 
-// Order-preserving key: a > b as floats  <=>  key(a) > key(b) as unsigned; -0 -> +0.
-__device__ __forceinline__ uint32_t score_key(float x) {
-  uint32_t u = __float_as_uint(x);
-  if (u == 0x80000000u) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 // Exclusive block-wide prefix sum of v; *total receives the sum over the block.
 __device__ __forceinline__ int block_excl_scan(int v, int* tmp, int* total) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -91,7 +84,13 @@ __device__ __forceinline__ int block_excl_scan(int v, int* tmp, int* total) {
 
 // Finds the bin B (of nbins) with count(bins > B) < need <= count(bins >= B).
 // Writes B to sm.bcast[0] and count(bins > B) to sm.bcast[1].
-__device__ __forceinline__ void find_bin(TopkSmem& sm, int nbins, int need) {
+// (If no bin qualifies -- inconsistent counts -- bin 0 and 0 are reported.)
+template <typename Smem>
+__device__ __forceinline__ void find_bin(Smem& sm, int nbins, int need) {
+  if (threadIdx.x == 0) {
+    sm.bcast[0] = 0;
+    sm.bcast[1] = 0;
+  }
   const int per = nbins / TK_THREADS;  // 8 (4096 bins) or 0 (256 bins)
   int local = 0;
   int b_lo = 0, b_hi = 0;
@@ -591,6 +590,266 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
       }
     }
   }
+}
+
+// ------------------------------------------------------------------ fused top-k merge
+// The second half of the fused indexer -> top-k (indexer_tc.cu, one query per
+// sequence): every (row, CTA piece, epilogue set) left a slot holding every key
+// of its share of the row whose selection key (score key << 32 | ~index) is >=
+// the slot's tau, and, when tau != 0, at least k of them.  So the row's k largest
+// selection keys are all in the slots and all >= the largest tau.  One CTA per
+// row gathers the slot keys >= that tau into shared memory (narrowing the bound
+// by radix digits over the slots if too many pass), finds the exact k-th largest
+// selection key by 12-bit radix rounds, and writes the k selected indices in
+// ascending order (bitonic sort).  Selection keys are unique within a row, so
+// exactly k keys are >= the k-th: ties need no separate handling.
+constexpr int TM_CAP = 8192;  // selection keys gathered into shared memory
+
+struct MergeSmem {
+  uint64_t cand[TM_CAP];
+  int hist[TK_NBINS];
+  int sel[TK_MAXK];
+  int scnt[512];        // keys per slot (clamped)
+  int soff[513];        // prefix of scnt
+  int scan_tmp[TK_NW];
+  int bcast[4];
+  int counter;
+  unsigned long long tau, kmax;
+};
+
+// One radix round over keys offered by `each` (which calls its argument with
+// (ok, key) for every key, in warp-uniform rounds): counts the keys >= lo whose
+// top pbits bits equal prefix into sm.hist by their next `bits` bits, one shared
+// atomic per distinct bin per warp.
+template <typename Each>
+__device__ __forceinline__ void merge_hist(MergeSmem& sm, Each&& each, uint64_t lo,
+                                           uint64_t prefix, int pbits, int bits) {
+  const int lane = threadIdx.x & 31;
+  const int shift = 64 - pbits - bits;
+  const uint64_t mask = (1ull << bits) - 1ull;
+  for (int b = threadIdx.x; b < (1 << bits); b += TK_THREADS) sm.hist[b] = 0;
+  __syncthreads();
+  each([&](bool ok, uint64_t c) {
+    int bin = -1;
+    if (ok && c >= lo && (pbits == 0 || (c >> (64 - pbits)) == prefix))
+      bin = static_cast<int>((c >> shift) & mask);
+    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+    if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], __popc(peers));
+  });
+  __syncthreads();
+}
+
+// Calls f(ok, key) for every key of the row's slots, 8 loads in flight per thread.
+// The loop runs the same number of rounds in every thread (f may use warp votes):
+// past the last key, f gets ok = false.
+template <typename F>
+__device__ __forceinline__ void for_slot_keys(const MergeSmem& sm, const uint8_t* base, int nslot,
+                                              long slot_bytes, F&& f) {
+  const int tot = sm.soff[nslot];
+  for (int f0 = 0; f0 < tot; f0 += 8 * TK_THREADS) {
+    uint64_t c[8];
+    bool ok[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int fi = f0 + u * TK_THREADS + static_cast<int>(threadIdx.x);
+      ok[u] = fi < tot;
+      c[u] = 0;
+      if (ok[u]) {
+        int j = 0;  // slot of flat index fi (few slots: linear search)
+        while (sm.soff[j + 1] <= fi) ++j;
+        c[u] = __ldg(reinterpret_cast<const unsigned long long*>(base + j * slot_bytes + 64) +
+                     (fi - sm.soff[j]));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) f(ok[u], c[u]);
+  }
+}
+
+__global__ void __launch_bounds__(TK_THREADS) topk_merge_kernel(
+    const uint8_t* __restrict__ slots, long nt, long total, int G, int maxp, int nsets,
+    long slot_bytes, int cb, int nv, int k, int* __restrict__ idx) {
+  extern __shared__ __align__(16) uint8_t tm_smem_raw[];
+  MergeSmem& sm = *reinterpret_cast<MergeSmem*>(tm_smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31;
+  grid_dep_wait();
+  const long row = blockIdx.x;
+  int* out = idx + row * k;
+  if (nv <= k) {  // every candidate is selected
+    for (int j = tid; j < k; j += TK_THREADS) out[j] = (j < nv) ? j : -1;
+    return;
+  }
+  const long first = (row * nt * G + G - 1) / total;
+  const long last = ((row * nt + nt - 1) * G + G - 1) / total;
+  int nslot = static_cast<int>(last - first + 1) * nsets;
+  if (nslot > 512) nslot = 512;  // cannot happen for a plan of <= 170 pieces per row
+  const uint8_t* base = slots + row * static_cast<long>(maxp) * nsets * slot_bytes;
+  if (tid == 0) {
+    sm.tau = 0ull;
+    sm.kmax = 0ull;
+  }
+  for (int j = tid; j < nslot; j += TK_THREADS) {
+    int c = *reinterpret_cast<const int*>(base + j * slot_bytes);
+    sm.scnt[j] = c < 0 ? 0 : (c > cb ? cb : c);
+  }
+  __syncthreads();
+  for (int j = tid; j < nslot; j += TK_THREADS) {
+    atomicMax(&sm.tau, *reinterpret_cast<const unsigned long long*>(base + j * slot_bytes + 8));
+    if (sm.scnt[j] > 0)
+      atomicMax(&sm.kmax, *reinterpret_cast<const unsigned long long*>(base + j * slot_bytes + 16));
+  }
+  if (tid == 0) {
+    int acc = 0;
+    for (int j = 0; j < nslot; ++j) {
+      sm.soff[j] = acc;
+      acc += sm.scnt[j];
+    }
+    sm.soff[nslot] = acc;
+  }
+  __syncthreads();
+  uint64_t tau = sm.tau;
+
+  // gather every slot key >= tau (the count may pass TM_CAP: then nothing is usable)
+  auto gather = [&](uint64_t t) {
+    if (tid == 0) sm.counter = 0;
+    __syncthreads();
+    for_slot_keys(sm, base, nslot, slot_bytes, [&](bool ok, uint64_t c) {
+      const bool take = ok && c >= t;
+      const unsigned m = __ballot_sync(0xffffffffu, take);
+      if (m) {
+        int p = 0;
+        if (lane == 0) p = atomicAdd(&sm.counter, __popc(m));
+        p = __shfl_sync(0xffffffffu, p, 0) + __popc(m & ((1u << lane) - 1u));
+        if (take && p < TM_CAP) sm.cand[p] = c;
+      }
+    });
+    __syncthreads();
+    return sm.counter;
+  };
+  // Each slot's tau bounds only its own share, so many more than k keys of the row
+  // pass the largest tau (about 17 k at the decode shape).  If the slots hold more
+  // keys than fit, first narrow the bound by 12-bit digits over the slot keys >= tau
+  // until the keys >= the k-th key's bin fit (usually one round), then gather.
+  // every candidate lies in [tau, kmax]: the leading bits these share need no round
+  const uint64_t kmax = sm.kmax;
+  auto common = [&](uint64_t lo, int& pbits, uint64_t& prefix) {
+    pbits = (lo >= kmax) ? 63 : __clzll(static_cast<long long>(lo ^ kmax));
+    prefix = pbits == 0 ? 0ull : (lo >> (64 - pbits));
+  };
+  auto slot_each = [&](auto&& f) { for_slot_keys(sm, base, nslot, slot_bytes, f); };
+  int C = 0;
+  if (sm.soff[nslot] <= TM_CAP) {
+    C = gather(tau);
+  } else {
+    uint64_t prefix;
+    int pbits, need = k, above = 0;
+    common(tau, pbits, prefix);
+    for (;;) {
+      const int bits = (64 - pbits) >= 12 ? 12 : 64 - pbits;
+      merge_hist(sm, slot_each, tau, prefix, pbits, bits);
+      find_bin(sm, 1 << bits, need);
+      const int B = min(max(sm.bcast[0], 0), (1 << bits) - 1), gt = sm.bcast[1];
+      const int inb = sm.hist[B];
+      prefix = (prefix << bits) | static_cast<uint64_t>(B);
+      pbits += bits;
+      __syncthreads();
+      if (above + gt + inb <= TM_CAP || pbits == 64) {
+        const uint64_t edge = pbits == 64 ? prefix : prefix << (64 - pbits);
+        if (edge > tau) tau = edge;
+        break;
+      }
+      above += gt;
+      need -= gt;
+    }
+    C = gather(tau);
+    if (C > TM_CAP) {  // cannot happen: the descent stops once the keys >= tau fit
+      if (tid == 0) record_error(kErrTopkOverflow);
+      C = TM_CAP;
+    }
+  }
+
+  // the exact k-th largest selection key T among the gathered keys (all in [tau, kmax])
+  auto cand_each = [&](auto&& f) {
+    for (int i0 = 0; i0 < C; i0 += TK_THREADS) {
+      const int i = i0 + tid;
+      f(i < C, i < C ? sm.cand[i] : 0ull);
+    }
+  };
+  uint64_t prefix;
+  int pbits, need = k;
+  common(tau, pbits, prefix);
+  uint64_t T;
+  for (;;) {
+    const int bits = (64 - pbits) >= 12 ? 12 : 64 - pbits;
+    merge_hist(sm, cand_each, 0ull, prefix, pbits, bits);
+    find_bin(sm, 1 << bits, need);
+    const int B = min(max(sm.bcast[0], 0), (1 << bits) - 1), gt = sm.bcast[1];
+    const int inb = sm.hist[B];
+    prefix = (prefix << bits) | static_cast<uint64_t>(B);
+    pbits += bits;
+    __syncthreads();
+    if (gt + inb == need || pbits == 64) {  // every key of bin B is selected
+      T = pbits == 64 ? prefix : prefix << (64 - pbits);
+      break;
+    }
+    need -= gt;
+  }
+
+  // the k keys >= T, their indices sorted ascending
+  int P = 1;
+  while (P < k) P <<= 1;
+  for (int j = tid; j < P; j += TK_THREADS) sm.sel[j] = 0x7fffffff;
+  if (tid == 0) sm.counter = 0;
+  __syncthreads();
+  for (int i0 = 0; i0 < C; i0 += TK_THREADS) {
+    const int i = i0 + tid;
+    const uint64_t c = i < C ? sm.cand[i] : 0ull;
+    const bool take = i < C && c >= T;
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (m) {
+      int p = 0;
+      if (lane == 0) p = atomicAdd(&sm.counter, __popc(m));
+      p = __shfl_sync(0xffffffffu, p, 0) + __popc(m & ((1u << lane) - 1u));
+      if (take && p < TK_MAXK) sm.sel[p] = static_cast<int>(~static_cast<uint32_t>(c));
+    }
+  }
+  __syncthreads();
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < P / 2; i += TK_THREADS) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const int x = sm.sel[lo], y = sm.sel[hi];
+        if ((x > y) == ((lo & size) == 0)) {
+          sm.sel[lo] = y;
+          sm.sel[hi] = x;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int got = sm.counter < k ? sm.counter : k;
+  if (sm.counter != k && tid == 0) record_error(kErrTopkOverflow);  // cannot happen
+  for (int j = tid; j < k; j += TK_THREADS) out[j] = (j < got) ? sm.sel[j] : -1;
+}
+
+ic_status launch_topk_merge(const uint8_t* slots, long rows, long nt, long total, int G, int maxp,
+                            int nsets, size_t slot_bytes, int cb, int nv, int k, int* idx,
+                            cudaStream_t stream) {
+  if (rows == 0) return IC_OK;
+  const int smem = static_cast<int>(sizeof(MergeSmem));
+  ic_status st = cuda_check(
+      cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+      "cudaFuncSetAttribute(topk_merge)");
+  if (st) return st;
+  st = cuda_check(launch_dep(topk_merge_kernel, dim3(static_cast<unsigned>(rows)),
+                             dim3(TK_THREADS), smem, stream, 1, slots, nt, total, G, maxp, nsets,
+                             static_cast<long>(slot_bytes), cb, nv, k, idx),
+                  "topk_merge_kernel launch");
+  if (st) return st;
+  // algorithmic bytes: the index rows written (the candidates it reads depend on the data)
+  trace_launch(kKindTopkMerge, stream, 4.0 * static_cast<double>(rows) * k);
+  return IC_OK;
 }
 
 ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0, int k, int* idx,

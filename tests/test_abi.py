@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_empty_error(lib):
-    assert binding.ic_version() == 100
+    assert binding.ic_version() == 101
     assert isinstance(binding.ic_last_error(), str)
 
 
@@ -122,3 +122,26 @@ def test_varlen_stack_rejects_bad_sequence_offsets(lib):
         assert lib.ic_layer_stack_varlen(b"F", ctypes.byref(desc), arr, 1, c, len(cu) - 1, None,
                                          None, 0, None) == binding.IC_ERR_INVALID_ARG
         assert "varlen" in binding.ic_last_error()
+
+
+def test_indexer_topk_rejects_before_launch(lib):
+    fake = ctypes.c_void_p(256)  # never dereferenced: the checks fail first
+    # fp32 has no fused path
+    st = lib.ic_indexer_topk(fake, None, fake, None, fake, binding.IC_F32, 2, 4, 32, 100, 99, 8,
+                             fake, fake, 1 << 20, None)
+    assert st == binding.IC_ERR_UNSUPPORTED
+    # k outside [1, 2048]
+    st = lib.ic_indexer_topk(fake, None, fake, None, fake, binding.IC_BF16, 2, 64, 128, 100, 99,
+                             4096, fake, fake, 1 << 20, None)
+    assert st == binding.IC_ERR_INVALID_ARG
+    # e4m3 without scales
+    st = lib.ic_indexer_topk(fake, None, fake, None, fake, binding.IC_E4M3, 2, 64, 128, 100, 99,
+                             16, fake, fake, 1 << 20, None)
+    assert st == binding.IC_ERR_INVALID_ARG
+    assert binding.ic_indexer_topk_workspace_size(0, 100, 99) == 0
+
+
+def test_topk_varlen_rejects_before_launch(lib):
+    fake = ctypes.c_void_p(256)
+    assert lib.ic_topk_varlen(fake, 4, 100, 100, None, 8, fake, None) == binding.IC_ERR_INVALID_ARG
+    assert lib.ic_topk_varlen(fake, 4, 100, 50, fake, 8, fake, None) == binding.IC_ERR_INVALID_ARG

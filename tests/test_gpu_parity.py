@@ -576,6 +576,105 @@ def test_decode_step_graph_replay_matches_eager():
     del g
 
 
+# ------------------------------------------------------------------ fused indexer -> top-k
+def _fused_vs_unfused(q, k, w, pos0, k_top, q_scale=None, k_scale=None):
+    B, Lk = k.shape[0], k.shape[1]
+    ws = torch.empty(ic.ic_indexer_topk_workspace_size(B, Lk, pos0) // 4 + 4, device=DEV)
+    got = ic.ic_indexer_topk(q, k, w, k_top, ws, pos0=pos0, q_scale=q_scale, k_scale=k_scale)
+    scores = ic.ic_indexer_scores(q, k, w, pos0=pos0, q_scale=q_scale, k_scale=k_scale)
+    ref = ic.ic_topk(scores.view(B, Lk), k_top, pos0=pos0)
+    _sync()
+    assert torch.equal(got, ref)
+    return got, scores
+
+
+@pytest.mark.parametrize("fp8", [False, True], ids=["bf16", "e4m3"])
+@pytest.mark.parametrize("B,Lk,pos0,k_top", [(6, 5000, 4999, 2048), (64, 30000, 29999, 2048),
+                                             (3, 20000, 11000, 2048), (2, 1500, 1499, 2048),
+                                             (5, 9000, 8999, 100), (1, 60000, 59999, 1),
+                                             (4, 2100, 2047, 2048)])
+def test_indexer_topk_fused_equals_scores_then_topk(fp8, B, Lk, pos0, k_top):
+    """The fused indexer -> top-k selects exactly what ic_topk selects on the scores
+    ic_indexer_scores writes for the same inputs (one query per sequence): many CTA
+    pieces per row (B = 1..6), several rows per CTA (B = 64), masked keys past pos0,
+    rows with fewer candidates than k, k = 1 and k = 100."""
+    q, k, w = _idx_inputs(B, 1, Lk, seed=B * 7 + Lk)
+    q, k, w = q.to(DEV), k.to(DEV), w.to(DEV)
+    qs = ks = None
+    if fp8:
+        q, qs = ic.ic_quant_e4m3_rows(q)
+        k, ks = ic.ic_quant_e4m3_rows(k)
+    got, scores = _fused_vs_unfused(q, k, w, pos0, k_top, qs, ks)
+    # and the oracle's top-k on those scores, as for ic_topk
+    ref = oracle.topk(scores.view(B, Lk).cpu().numpy(), k_top,
+                      valid=np.full(B, min(Lk, pos0 + 1), np.int32))
+    np.testing.assert_array_equal(got.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("fp8", [False, True], ids=["bf16", "e4m3"])
+def test_indexer_topk_fused_repeatable(fp8):
+    """Ten calls in a row on a shape with several compactions per epilogue set and
+    rows split over CTAs: every call selects exactly what ic_topk selects."""
+    B, Lk = 64, 30000
+    q, k, w = _idx_inputs(B, 1, Lk, seed=99)
+    q, k, w = q.to(DEV), k.to(DEV), w.to(DEV)
+    qs = ks = None
+    if fp8:
+        q, qs = ic.ic_quant_e4m3_rows(q)
+        k, ks = ic.ic_quant_e4m3_rows(k)
+    scores = ic.ic_indexer_scores(q, k, w, pos0=Lk - 1, q_scale=qs, k_scale=ks)
+    ref = ic.ic_topk(scores.view(B, Lk), 2048, pos0=Lk - 1)
+    ws = torch.empty(ic.ic_indexer_topk_workspace_size(B, Lk, Lk - 1) // 4 + 4, device=DEV)
+    for _ in range(10):
+        ws.fill_(float("nan"))   # leftovers must not matter
+        got = ic.ic_indexer_topk(q, k, w, 2048, ws, pos0=Lk - 1, q_scale=qs, k_scale=ks)
+        _sync()
+        assert torch.equal(got, ref)
+
+
+def test_indexer_topk_fused_ties():
+    """Tied scores: all zero (queries 0), every head dead (negated queries over keys
+    with positive dots) and four distinct values; the lowest indices win."""
+    B, Lk = 4, 40000
+    g = torch.Generator().manual_seed(5)
+    k = torch.rand(B, Lk, 128, generator=g).to(torch.bfloat16).to(DEV)      # k >= 0
+    w = torch.rand(B, 1, 64, generator=g).to(DEV)
+    q0 = torch.zeros(B, 1, 64, 128, dtype=torch.bfloat16, device=DEV)
+    qneg = (-torch.rand(B, 1, 64, 128, generator=g)).to(torch.bfloat16).to(DEV)
+    for q in (q0, qneg):
+        got, _ = _fused_vs_unfused(q, k, w, Lk - 1, 2048)
+        assert torch.equal(got, torch.arange(2048, device=DEV, dtype=torch.int32).expand(B, -1))
+    # four distinct scores: keys are one of four vectors along one direction
+    u = torch.zeros(128)
+    u[0] = 1.0
+    kk = (torch.randint(0, 4, (B, Lk, 1), generator=g).float() * u).to(torch.bfloat16).to(DEV)
+    qq = torch.zeros(B, 1, 64, 128)
+    qq[..., 0] = 1.0
+    _fused_vs_unfused(qq.to(torch.bfloat16).to(DEV), kk, w, Lk - 1, 2048)
+
+
+def test_decode_step_fused_equals_unfused_top_k():
+    """ic_decode_step writes the scores and runs ic_topk by default; with
+    IC_STACK_FUSED_TOPK it fuses the indexer and the top-k.  Same T and outputs, bit
+    for bit."""
+    wl = synth.variant("decode_200k", L=7000, batch=9, pattern="F,S,F")
+    layers, _ = _stack_layers(wl, DEV)
+    for d in layers:
+        d["q_idx"], d["q_scale"] = ic.ic_quant_e4m3_rows(d["q_idx"])
+        d["k_idx"], d["k_scale"] = ic.ic_quant_e4m3_rows(d["k_idx"])
+    dl, t_fused = _run_stack(wl, wl.pattern, layers, ic.IC_E4M3, decode=True)
+    outs = [d["out"].clone() for d in dl]
+    desc = _desc(wl, ic.IC_E4M3)
+    desc.flags = ic.IC_STACK_FUSED_TOPK
+    ws = torch.empty(ic.ic_stack_workspace_size(desc) // 4 + 1, device=DEV)
+    t_unf = torch.full_like(t_fused, -7)
+    ic.ic_decode_step(wl.pattern, desc, dl, t_unf, ws)
+    _sync()
+    assert torch.equal(t_fused, t_unf)
+    for d, o in zip(dl, outs):
+        assert torch.equal(d["out"], o)
+
+
 def test_trace_records_every_launch_in_order():
     q, k, w = _idx_inputs(1, 8, 300, seed=3)
     q, k, w = q.to(DEV), k.to(DEV), w.to(DEV)
