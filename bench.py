@@ -604,6 +604,40 @@ def run_decode(args, dev, peaks, barrier):
                          "note": "IC_STACK_FUSED_TOPK: indexer and top-k fused, the scores never "
                                  "written; eager calls (compare with ms_per_step_eager)"}
     del ws_u
+    # the same F,S,S,S step over fp8 latent caches (ic_pack_kv_e4m3 rows of 656 bytes)
+    for d in layers:
+        d["kv"] = ic.ic_pack_kv_e4m3(d["kv"])
+        torch.cuda.empty_cache()
+    desc8 = ic.make_desc(L=L, k=k, H=wl.H, D=wl.D, idx_dtype=ic.IC_E4M3, heads=wl.Hq, dk=wl.Dk,
+                         dv=wl.Dv, attn_dtype=ic.IC_E4M3, scale=wl.scale, batch=B, decode=True,
+                         ld_kv=ic.KV8_ROW_BYTES)
+    ws8 = torch.empty(ic.ic_stack_workspace_size(desc8) // 4 + 1, dtype=torch.float32, device=dev)
+    step8 = lambda: ic.ic_decode_step(wl.pattern, desc8, layers, t_cache, ws8,  # noqa: E731
+                                      stream=stream)
+    for _ in range(3):
+        step8()
+    ic.ic_device_status(stream)
+    ms8 = _timed(step8, steps, stream)
+    ic.ic_device_status(stream)
+    ic.ic_trace_begin(64 * steps, stream=stream)
+    _timed(step8, steps, stream)
+    _, tr8 = ic.ic_trace_end(64 * steps)
+    ic.ic_device_status(stream)
+    attn8 = [ms for name, ms, _ in tr8 if name == "attn_mla_kv8"]
+    attn8_b = B * kk * ic.KV8_ROW_BYTES + B * wl.Hq * (wl.Dk + wl.Dv) * 2 + B * kk * 4
+    hb8 = sum(1 for c in wl.pattern if c == "F") * (idx_b + score_b) + wl.layers * attn8_b
+    out["fp8_kv"] = {
+        "pattern": wl.pattern, "kv_cache": "fp8 latent rows: 512 e4m3 (four 128-dim groups with "
+        "fp32 scales) + 64 bf16 rope = 656 B", "ms_per_step_eager": ms8,
+        "value": B / (ms8 * 1e-3), "unit": "tokens/s", "hbm_bytes_per_step": hb8,
+        "frac_hbm": hb8 / (ms8 * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "attn_ms_per_launch": sum(attn8) / max(1, len(attn8)),
+        "attn_frac_hbm": (attn8_b / (sum(attn8) / max(1, len(attn8)) * 1e-3) / 1e9 /
+                          peaks["hbm_gbs"]) if attn8 else None,
+        "speedup_over_bf16_kv_eager": out["ms_per_step_eager"] / ms8}
+    del ws8
+    log("decode fp8 kv: %.3f ms/step eager (bf16 cache %.3f ms eager)" % (
+        ms8, out["ms_per_step_eager"]))
     log("decode: %.3f ms/step (%.0f tokens/s), %.0f GB/s = %.2f of HBM; all-F %.3f ms" % (
         out["ms_per_step"], out["value"], out["achieved_gbs"], out["frac_hbm"],
         out["all_f"]["ms_per_step"]))

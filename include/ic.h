@@ -93,6 +93,8 @@ ic_status ic_device_status(void* stream);
 #define IC_K_TOPK_MERGE 10
 #define IC_K_INDEXER_TOPK_BF16 11
 #define IC_K_INDEXER_TOPK_E4M3 12
+#define IC_K_ATTN_MLA_KV8 13
+#define IC_K_PACK_KV 14
 ic_status ic_trace_begin(void* stream, int capacity);
 long ic_trace_end(float* ms, int* kinds, double* work, int capacity);
 
@@ -179,6 +181,22 @@ ic_status ic_topk_varlen(const float* scores, long rows, int n, long ld, const i
                          int k, int* idx, void* stream);
 
 /*
+ * The fp8 latent-KV cache (a serving-side variant of the MLA cache: the same
+ * latent rows, about 57% of the bytes to gather).  Row r of kv [rows, ld_kv]
+ * bf16 (576 dims: 512 latent + 64 rope) becomes 656 bytes at out + r * ld_out:
+ *   bytes   0..511  the 512 latent dims as OCP E4M3 codes, in four groups of 128;
+ *                   group g: scale_g = amax_g / 448 (1 if all zero),
+ *                   code = E4M3_rne_satfinite(x / scale_g), in fp32 (the same
+ *                   arithmetic as ic_quant_e4m3_rows on each 128-dim group)
+ *   bytes 512..527  scale_0..scale_3, fp32
+ *   bytes 528..655  the 64 rope dims, bf16, unchanged
+ * ld_kv >= 576 (elements, a multiple of 8); ld_out >= 656 (bytes, a multiple of
+ * 16); both tensors 16-byte aligned.
+ */
+ic_status ic_pack_kv_e4m3(const void* kv, long rows, long ld_kv, uint8_t* out, long ld_out,
+                          void* stream);
+
+/*
  * Sparse attention of each query over its index set (routing loop:
  * X <- SparseAttn(X, T); MLA paragraph).  For query (b, r), head h, with
  * J = { idx[b, r, j] : idx >= 0 } (-1 entries are skipped):
@@ -187,7 +205,12 @@ ic_status ic_topk_varlen(const float* scores, long rows, int n, long ld, const i
  *   lse[b, r, h]    = log sum_j exp(z_j)      (natural log; -inf if J is empty)
  * Two forms:
  *   v == NULL  absorbed MLA: V = kv[..., :dv] (the first dv latent dims);
- *              dt = IC_BF16, dk = 576, dv = 512, heads = 16, k <= 2048; out bf16.
+ *              dk = 576, dv = 512, heads = 16, k <= 2048; q and out bf16;
+ *              dt = IC_BF16: kv rows are bf16, ld_kv in elements (a multiple of 8);
+ *              dt = IC_E4M3: kv rows are fp8 cache rows (ic_pack_kv_e4m3), ld_kv in
+ *              bytes (>= 656, a multiple of 16); each gathered row is dequantised
+ *              in shared memory (code * its group's scale, rounded to bf16; rope
+ *              as stored) before the same bf16 products.
  *   v != NULL  MQA with separate values v [batch, Lkv, dv]; dt = IC_F32,
  *              dk, dv <= 256, heads <= 64; out f32.
  *   q   [batch, rows, heads, dk]; kv [batch, Lkv, ld_kv] (ld_kv >= dk, elements);
@@ -278,7 +301,8 @@ typedef struct {
   int k;               /* top-k (<= 2048)                                        */
   ic_dtype idx_dtype;  /* IC_BF16, IC_E4M3 (H=64, D=128) or IC_F32              */
   int H, D;            /* indexer heads and head dim                             */
-  ic_dtype attn_dtype; /* IC_BF16 (absorbed MLA) or IC_F32 (MQA)                 */
+  ic_dtype attn_dtype; /* IC_BF16 / IC_E4M3 (absorbed MLA over a bf16 / fp8 cache,
+                          ld_kv in elements / bytes) or IC_F32 (MQA)            */
   int heads, dk, dv;   /* attention heads, key dim, value dim                    */
   long ld_kv;          /* row stride of kv in elements                           */
   float scale;         /* softmax scale                                          */

@@ -242,6 +242,43 @@ def sparse_attn(q, kv, idx, scale: float, dv: int | None = None, v=None,
     return out, lse
 
 
+# ----------------------------------------------------------------------------- fp8 latent KV
+KV_GROUP = 128     # latent dims per e4m3 scale group
+KV_LATENT = 512    # e4m3 latent dims of a 576-d row; the other 64 (rope) stay bf16
+
+
+def kv_pack_e4m3(kv):
+    """The fp8 latent-KV cache of bf16-valued rows kv [..., 576] (float arrays).
+
+    The 512 latent dims are quantised in four groups of 128 with the per-row
+    quantiser (scale = amax / 448 per group, code = E4M3(x / scale)); the 64
+    rope dims are kept as they are.  Returns (codes uint8 [..., 512],
+    scales f32 [..., 4], rope f32 [..., 64])."""
+    kv = np.asarray(kv, dtype=np.float32)
+    assert kv.shape[-1] == KV_LATENT + 64
+    lead = kv.shape[:-1]
+    lat = np.ascontiguousarray(kv[..., :KV_LATENT]).reshape(lead + (KV_LATENT // KV_GROUP, KV_GROUP))
+    codes, scales = quant_rows_e4m3(lat)
+    return codes.reshape(lead + (KV_LATENT,)), scales, np.ascontiguousarray(kv[..., KV_LATENT:])
+
+
+def kv_dequant_e4m3(codes, scales, rope):
+    """fp64 rows [..., 576] of an fp8 latent-KV cache: code value * its group's scale
+    for the 512 latent dims, then the 64 rope dims."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    lead = codes.shape[:-1]
+    g = codes.reshape(lead + (KV_LATENT // KV_GROUP, KV_GROUP))
+    lat = dequant_rows_e4m3(g, scales).reshape(lead + (KV_LATENT,))
+    return np.concatenate([lat, np.asarray(rope, dtype=np.float64)], axis=-1)
+
+
+def sparse_attn_kv_e4m3(q, codes, scales, rope, idx, scale: float, nthreads: int | None = None):
+    """Absorbed-MLA sparse attention over an fp8 latent-KV cache: the same definition
+    as sparse_attn on the dequantised rows (values = their first 512 dims)."""
+    kv = kv_dequant_e4m3(codes, scales, rope)
+    return sparse_attn(q, kv, idx, scale, dv=KV_LATENT, nthreads=nthreads)
+
+
 # ----------------------------------------------------------------------------- F/S stack
 def parse_pattern(pattern: str) -> list[str]:
     """Layer types from a pattern string such as "F,S,S,S" or "F S S S" or "FSSS".

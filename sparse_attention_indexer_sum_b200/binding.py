@@ -26,7 +26,7 @@ IC_F32, IC_BF16, IC_E4M3 = 0, 1, 2
 
 # names declared in include/ic.h (checked against the header by the tests)
 EXPORTS = ("ic_last_error", "ic_version", "ic_device_status", "ic_trace_begin", "ic_trace_end",
-           "ic_quant_e4m3_rows",
+           "ic_quant_e4m3_rows", "ic_pack_kv_e4m3",
            "ic_indexer_scores", "ic_indexer_topk", "ic_indexer_topk_workspace_size", "ic_topk",
            "ic_topk_varlen", "ic_sparse_attn",
            "ic_attn_workspace_size",
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
     L.ic_trace_end.argtypes = [P, P, P, I]
     L.ic_trace_end.restype = Lg
     L.ic_quant_e4m3_rows.argtypes = [P, I, Lg, I, P, P, P]
+    L.ic_pack_kv_e4m3.argtypes = [P, Lg, Lg, P, Lg, P]
     L.ic_indexer_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Lg, P, Lg, P]
     L.ic_indexer_topk.argtypes = [P, P, P, P, P, I, I, I, I, I, Lg, I, P, P, S, P]
     L.ic_indexer_topk_workspace_size.argtypes = [I, I, Lg]
@@ -100,7 +101,8 @@ def lib() -> ctypes.CDLL:
     L.ic_stack_workspace_size.argtypes = [ctypes.POINTER(ic_stack_desc)]
     L.ic_stack_workspace_size.restype = S
     L.ic_sparse_attn_noalloc.argtypes = [P, P, Lg, P, P, I, I, I, I, I, I, I, I, F, P, P, P]
-    for name in ("ic_device_status", "ic_quant_e4m3_rows", "ic_indexer_scores", "ic_topk",
+    for name in ("ic_device_status", "ic_quant_e4m3_rows", "ic_pack_kv_e4m3", "ic_indexer_scores",
+                 "ic_topk",
                  "ic_topk_varlen", "ic_indexer_topk",
                  "ic_sparse_attn", "ic_layer_stack", "ic_decode_step", "ic_sparse_attn_noalloc",
                  "ic_layer_stack_rows", "ic_layer_stack_varlen"):
@@ -159,7 +161,8 @@ def ic_device_status(stream=None):
 
 KIND_NAMES = {1: "indexer_tc_bf16", 2: "indexer_tc_e4m3", 3: "indexer_f32", 4: "fill_masked",
               5: "topk", 6: "attn_mla", 7: "attn_combine", 8: "attn_f32", 9: "quant_e4m3",
-              10: "topk_merge", 11: "indexer_topk_bf16", 12: "indexer_topk_e4m3"}
+              10: "topk_merge", 11: "indexer_topk_bf16", 12: "indexer_topk_e4m3",
+              13: "attn_mla_kv8", 14: "pack_kv_e4m3"}
 
 
 def ic_trace_begin(capacity: int = 4096, stream=None):
@@ -195,6 +198,22 @@ def ic_quant_e4m3_rows(x: torch.Tensor, codes=None, scales=None, stream=None):
     _check(lib().ic_quant_e4m3_rows(_p(x), dtype_code(x), rows, n, _p(codes), _p(scales),
                                     _stream(stream)))
     return codes, scales
+
+
+KV8_ROW_BYTES = 656
+
+
+def ic_pack_kv_e4m3(kv: torch.Tensor, out=None, stream=None):
+    """fp8 latent-KV cache rows [..., 656] uint8 of bf16 latent rows kv [..., 576]
+    (512 e4m3 codes in four 128-dim groups, 4 fp32 group scales, 64 bf16 rope dims)."""
+    if kv.dtype != torch.bfloat16 or kv.shape[-1] != 576 or kv.stride(-1) != 1:
+        raise ValueError("kv must be bf16 [..., 576] with contiguous rows")
+    rows = kv.numel() // 576
+    if out is None:
+        out = torch.empty(kv.shape[:-1] + (KV8_ROW_BYTES,), dtype=torch.uint8, device=kv.device)
+    _contig(kv, out)
+    _check(lib().ic_pack_kv_e4m3(_p(kv), rows, 576, _p(out), out.shape[-1], _stream(stream)))
+    return out
 
 
 def ic_indexer_scores(q, k, w, scores=None, *, pos0: int = 0, q_scale=None, k_scale=None,
@@ -276,7 +295,8 @@ def ic_attn_workspace_size(batch: int, rows: int, heads: int, dv: int, k: int) -
 def ic_sparse_attn(q, kv, idx, scale: float, *, v=None, dv: int | None = None, out=None, lse=None,
                    workspace=None, stream=None):
     """Sparse attention.  q [B?,R,heads,dk]; kv [B?,Lkv,ld_kv]; idx [B?,R,k];
-    v [B?,Lkv,dv] for the MQA form (fp32), else absorbed MLA over kv[..., :dv] (bf16)."""
+    v [B?,Lkv,dv] for the MQA form (fp32), else absorbed MLA over kv[..., :dv]: a bf16
+    cache, or an fp8 cache (uint8 rows of ic_pack_kv_e4m3) with q and out bf16."""
     _contig(q, idx, v)
     if kv.stride(-1) != 1:
         raise ValueError("kv rows must be contiguous")
@@ -292,7 +312,8 @@ def ic_sparse_attn(q, kv, idx, scale: float, *, v=None, dv: int | None = None, o
     if out is None:
         out = torch.empty(q.shape[:-1] + (dv,), dtype=q.dtype, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().ic_sparse_attn(_p(q), _p(kv), kv.stride(-2), _p(v), _p(idx), dtype_code(q), B, R,
+    dt = IC_E4M3 if (v is None and kv.dtype == torch.uint8) else dtype_code(q)
+    _check(lib().ic_sparse_attn(_p(q), _p(kv), kv.stride(-2), _p(v), _p(idx), dt, B, R,
                                 heads, dk, dv, Lkv, kk, float(scale), _p(out), _p(lse),
                                 _p(workspace), ws_bytes, _stream(stream)))
     return out

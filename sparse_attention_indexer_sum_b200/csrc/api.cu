@@ -126,12 +126,14 @@ static ic_status check_attn(const void* q, const void* kv, long ld_kv, const voi
   if (batch < 1 || rows < 0 || Lkv < 1 || k < 1 || ld_kv < dk)
     return fail(IC_ERR_INVALID_ARG, "attn: bad sizes");
   if (!v) {
-    if (dt != IC_BF16 || heads != 16 || dk != 576 || dv != 512)
+    if ((dt != IC_BF16 && dt != IC_E4M3) || heads != 16 || dk != 576 || dv != 512)
       return fail(IC_ERR_UNSUPPORTED,
-                  "attn: absorbed MLA needs bf16, 16 heads, dk 576, dv 512 (got %d, %d, %d, %d)",
-                  static_cast<int>(dt), heads, dk, dv);
-    if (!aligned(q, 16) || !aligned(kv, 16) || (ld_kv % 8) != 0)
-      return fail(IC_ERR_INVALID_ARG, "attn: q/kv rows must be 16-byte aligned");
+                  "attn: absorbed MLA needs a bf16 or e4m3 cache, 16 heads, dk 576, dv 512 "
+                  "(got %d, %d, %d, %d)", static_cast<int>(dt), heads, dk, dv);
+    if (!aligned(q, 16) || !aligned(kv, 16) ||
+        (dt == IC_BF16 ? (ld_kv % 8) != 0 : (ld_kv < KV8_ROW_BYTES || (ld_kv % 16) != 0)))
+      return fail(IC_ERR_INVALID_ARG,
+                  "attn: q/kv rows must be 16-byte aligned (e4m3 cache: ld_kv >= 656 bytes)");
     if (k > 2048) return fail(IC_ERR_UNSUPPORTED, "attn: absorbed MLA needs k <= 2048");
   } else {
     if (dt != IC_F32 || heads < 1 || heads > 64 || dk < 1 || dk > 256 || dv < 1 || dv > 256)
@@ -142,12 +144,12 @@ static ic_status check_attn(const void* q, const void* kv, long ld_kv, const voi
 }
 
 static ic_status run_attn(const void* q, const void* kv, long ld_kv, const void* v,
-                          const int* idx, int batch, int rows, int heads, int dk, int dv, int Lkv,
-                          int k, float scale, void* out, float* lse, void* ws, size_t ws_bytes,
-                          long long valid_entries, cudaStream_t stream) {
+                          const int* idx, ic_dtype dt, int batch, int rows, int heads, int dk,
+                          int dv, int Lkv, int k, float scale, void* out, float* lse, void* ws,
+                          size_t ws_bytes, long long valid_entries, cudaStream_t stream) {
   if (!v)
     return launch_attn_mla(q, kv, ld_kv, idx, batch, rows, Lkv, k, scale, out, lse, ws, ws_bytes,
-                           valid_entries, stream);
+                           valid_entries, stream, dt == IC_E4M3);
   return launch_attn_f32(static_cast<const float*>(q), static_cast<const float*>(kv), ld_kv,
                          static_cast<const float*>(v), idx, batch, rows, heads, dk, dv, Lkv, k,
                          scale, static_cast<float*>(out), lse, stream);
@@ -266,8 +268,8 @@ static ic_status run_stack(const char* pattern, const ic_stack_desc* d, const ic
     // out_l <- SparseAttn_l(T_cache); the score workspace is free again here
     const long long valid = decode ? static_cast<long long>(B) * (d->k < d->L ? d->k : d->L)
                                    : causal_pairs(R, d->k, row0);
-    st = run_attn(io.q, io.kv, d->ld_kv, io.v, t_cache, B, R, d->heads, d->dk, d->dv, d->L, d->k,
-                  d->scale, io.out, io.lse, workspace, ws_bytes, valid, stream);
+    st = run_attn(io.q, io.kv, d->ld_kv, io.v, t_cache, d->attn_dtype, B, R, d->heads, d->dk,
+                  d->dv, d->L, d->k, d->scale, io.out, io.lse, workspace, ws_bytes, valid, stream);
     if (st) return st;
   }
   return IC_OK;
@@ -353,6 +355,17 @@ ic_status ic_quant_e4m3_rows(const void* x, ic_dtype x_dtype, long rows, int n, 
                            static_cast<cudaStream_t>(stream));
 }
 
+ic_status ic_pack_kv_e4m3(const void* kv, long rows, long ld_kv, uint8_t* out, long ld_out,
+                          void* stream) {
+  if (!kv || !out) return fail(IC_ERR_INVALID_ARG, "pack_kv: NULL tensor");
+  if (rows < 0 || ld_kv < 576 || (ld_kv % 8) != 0 || ld_out < KV8_ROW_BYTES || (ld_out % 16) != 0)
+    return fail(IC_ERR_INVALID_ARG,
+                "pack_kv: need ld_kv >= 576 (a multiple of 8) and ld_out >= 656 (of 16)");
+  if (!aligned(kv, 16) || !aligned(out, 16))
+    return fail(IC_ERR_INVALID_ARG, "pack_kv: rows must be 16-byte aligned");
+  return launch_pack_kv_e4m3(kv, rows, ld_kv, out, ld_out, static_cast<cudaStream_t>(stream));
+}
+
 ic_status ic_indexer_scores(const void* q, const float* q_scale, const void* k,
                             const float* k_scale, const float* w, ic_dtype dt, int batch, int H,
                             int D, int rows, int Lk, long pos0, float* scores, long ld,
@@ -412,7 +425,7 @@ ic_status ic_sparse_attn(const void* q, const void* kv, long ld_kv, const void* 
                          size_t ws_bytes, void* stream) {
   ic_status st = check_attn(q, kv, ld_kv, v, idx, dt, batch, rows, heads, dk, dv, Lkv, k, out);
   if (st) return st;
-  return run_attn(q, kv, ld_kv, v, idx, batch, rows, heads, dk, dv, Lkv, k, scale, out, lse,
+  return run_attn(q, kv, ld_kv, v, idx, dt, batch, rows, heads, dk, dv, Lkv, k, scale, out, lse,
                   workspace, ws_bytes, -1, static_cast<cudaStream_t>(stream));
 }
 
@@ -453,10 +466,13 @@ ic_status ic_layer_stack_varlen(const char* pattern, const ic_stack_desc* desc,
     return fail(IC_ERR_INVALID_ARG, "varlen: bad layers / nlayers");
   const size_t qrow_b = static_cast<size_t>(desc->H) * desc->D * elem_bytes(desc->idx_dtype);
   const size_t krow_b = static_cast<size_t>(desc->D) * elem_bytes(desc->idx_dtype);
-  const size_t arow_b = static_cast<size_t>(desc->heads) * desc->dk * elem_bytes(desc->attn_dtype);
+  // q, v and out are fp32 (MQA) or bf16 (MLA, also over an e4m3 cache, whose ld_kv is
+  // in bytes)
+  const size_t qe = desc->attn_dtype == IC_F32 ? 4 : 2;
+  const size_t arow_b = static_cast<size_t>(desc->heads) * desc->dk * qe;
   const size_t kvrow_b = static_cast<size_t>(desc->ld_kv) * elem_bytes(desc->attn_dtype);
-  const size_t vrow_b = static_cast<size_t>(desc->dv) * elem_bytes(desc->attn_dtype);
-  const size_t orow_b = static_cast<size_t>(desc->heads) * desc->dv * elem_bytes(desc->attn_dtype);
+  const size_t vrow_b = static_cast<size_t>(desc->dv) * qe;
+  const size_t orow_b = static_cast<size_t>(desc->heads) * desc->dv * qe;
   std::vector<ic_layer_io> sub(nlayers);
   for (int i = 0; i < nseq; ++i) {
     const long o = cu_seqlens[i], n = cu_seqlens[i + 1] - cu_seqlens[i];
@@ -500,7 +516,7 @@ size_t ic_stack_workspace_size(const ic_stack_desc* d) {
   size_t s = static_cast<size_t>(want) * d->L * sizeof(float);
   if (d->decode && d->idx_dtype != IC_F32 && (d->flags & IC_STACK_FUSED_TOPK))
     s = indexer_topk_fused_ws_bytes(d->batch, d->L, d->L - 1);
-  if (d->decode && d->attn_dtype == IC_BF16) {
+  if (d->decode && d->attn_dtype != IC_F32) {
     const size_t a = attn_mla_ws_bytes(d->batch, 1, d->k);
     if (a > s) s = a;
   }

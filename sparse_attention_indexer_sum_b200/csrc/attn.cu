@@ -43,6 +43,7 @@ constexpr int AT_CONSUMERS = 256;           // 8 consumer warps
 constexpr int AT_PRODUCERS = 4;             // producer warps; each issues 8 of a tile's 32 rows
 constexpr int AT_THREADS = AT_CONSUMERS + 32 * AT_PRODUCERS;
 constexpr int AT_ROWB = AT_DK * 2 + 16;     // padded shared row: 1168 B
+static_assert(AT_ROWB - KV8_ROW_BYTES == 512, "an fp8 row lands behind its 512 bf16 latent dims");
 constexpr uint32_t AT_ROW_BYTES = AT_DK * 2;  // 1152 B gathered per row
 
 constexpr int AT_SROW = 40;  // padded partial-score row (floats): conflict-free 64-bit access
@@ -63,6 +64,7 @@ struct AttnSmem {
   uint64_t qfull, qempty;
   uint64_t ifull[2];
   uint64_t pitem;   // producers meet here at every item start
+  uint64_t rawf[AT_STAGES];  // fp8 cache: a stage's raw rows have landed
   int abort;
 };
 
@@ -86,7 +88,56 @@ struct AttnArgs {
   float* lse;               // [B, R, 16] or null (not split)
   float* part_o;            // [items * maxp, 16, 512] (split)
   float* part_ml;           // [items * maxp, 16, 2]   (split)
+  // fp8 latent cache (kv8): rows of 656 bytes (512 e4m3 codes, 4 fp32 group scales,
+  // 64 bf16 rope dims) at kv8p + row * ld_kv8 bytes; dequantised in shared memory
+  // to the bf16 row layout the consumers read
+  int kv8;
+  const uint8_t* kv8p;
+  long ld_kv8;
 };
+
+// Dequantises the fp8 rows of one tile stage that belong to producer warp pw (rows
+// 8pw..8pw+7 with their bit set in `valid`) in place: a raw row (656 bytes at slot
+// offset 512) becomes the 576 bf16 values of the row at offset 0, latent code *
+// its group's scale rounded to bf16, rope copied.  Lane l owns latent dims
+// 16l..16l+15 of every row (and rope bytes 16l..16l+15 for l < 8).  All eight
+// rows are loaded before any store, so the overlapping expansion is safe and the
+// rows' loads overlap; rows without a copy are left as they are (finite values
+// of an earlier tile).
+__device__ __forceinline__ void attn_dequant_rows(uint8_t* stage_rows, unsigned valid, int pw) {
+  const int lane = threadIdx.x & 31;
+  uint8_t* rows = stage_rows + 8 * pw * AT_ROWB;
+  const unsigned mine = (valid >> (8 * pw)) & 0xFFu;
+  uint4 codes[8], rope[8];
+  float sc[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const uint8_t* row = rows + r * AT_ROWB;
+    codes[r] = *reinterpret_cast<const uint4*>(row + 512 + 16 * lane);
+    sc[r] = *reinterpret_cast<const float*>(row + 1024 + 4 * (lane / 8));
+    rope[r] = lane < 8 ? *reinterpret_cast<const uint4*>(row + 1040 + 16 * lane)
+                       : make_uint4(0, 0, 0, 0);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (!((mine >> r) & 1u)) continue;
+    uint8_t* row = rows + r * AT_ROWB;
+    const __nv_fp8x2_storage_t* cp = reinterpret_cast<const __nv_fp8x2_storage_t*>(&codes[r]);
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // two codes -> two exact halves -> scaled, rounded to bf16
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(cp[i], __NV_E4M3);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+      __nv_bfloat162 v = __floats2bfloat162_rn(f.x * sc[r], f.y * sc[r]);
+      o[i] = *reinterpret_cast<uint32_t*>(&v);
+    }
+    *reinterpret_cast<uint4*>(row + 32 * lane) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(row + 32 * lane + 16) = make_uint4(o[4], o[5], o[6], o[7]);
+    if (lane < 8) *reinterpret_cast<uint4*>(row + 1024 + 16 * lane) = rope[r];
+  }
+  __syncwarp();
+}
 
 // CTA holding (query, tile) pair t of the split list: the largest c with
 // floor(c * tot / G) <= t.
@@ -204,6 +255,22 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
   int ib = 0;
   long nitem = 0;
   const long nj = attn_nitems(a);
+  // fp8 cache: the stage, phase and valid rows of the tile whose raw rows are the
+  // next to dequantise (one tile behind the copies, so that they overlap)
+  int pend_stage = -1;
+  uint32_t pend_ph = 0;
+  unsigned pend_valid = 0u;
+  auto dequant_pending = [&]() -> bool {
+    if (pend_stage < 0) return true;
+    if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.rawf[pend_stage]), pend_ph, abort,
+                                           kErrTimeoutProducer)))
+      return false;
+    attn_dequant_rows(&sm.kv[pend_stage][0][0], pend_valid, pw);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&sm.full[pend_stage]));
+    pend_stage = -1;
+    return true;
+  };
   if (pw == 0 && nj > 0) {
     attn_load_indices(sm, a, 0, 0, bulk);
     ipending[0] = bulk;
@@ -213,6 +280,7 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
     const int cnt = x.end - x.beg;
     const long b = x.qrow / a.R;
     const __nv_bfloat16* kvb = a.kv + b * static_cast<long>(a.Lkv) * a.ld_kv;
+    const uint8_t* kvb8 = a.kv8p + b * static_cast<long>(a.Lkv) * a.ld_kv8;
     // every producer is done with the previous item (and its index list)
     if (lane == 0) mbar_arrive(smem_u32(&sm.pitem));
     if (!mbar_wait(smem_u32(&sm.pitem), static_cast<uint32_t>(nitem & 1), abort, kErrTimeoutProducer))
@@ -265,12 +333,32 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
         sm.vmask[stage] = valid;
         sm.last[stage] = (t == nt - 1);
       }
-      const uint32_t fb = smem_u32(&sm.full[stage]);
-      if (lane == 0) mbar_arrive_expect_tx(fb, __popc(valid & (0xFFu << (8 * pw))) * AT_ROW_BYTES);
-      __syncwarp();
-      if (mine && s >= 0)
-        bulk_g2s(kv0 + (stage * AT_BK + lane) * AT_ROWB, kvb + static_cast<long>(s) * a.ld_kv,
-                 AT_ROW_BYTES, fb);
+      if (a.kv8) {
+        // the raw fp8 row lands in the slot's last 656 bytes; the warp dequantises
+        // its rows of the previous tile while these copies are in flight
+        const uint32_t rb = smem_u32(&sm.rawf[stage]);
+        if (lane == 0)
+          mbar_arrive_expect_tx(rb, __popc(valid & (0xFFu << (8 * pw))) * KV8_ROW_BYTES);
+        __syncwarp();
+        if (mine && s >= 0)
+          bulk_g2s(kv0 + (stage * AT_BK + lane) * AT_ROWB + (AT_ROWB - KV8_ROW_BYTES),
+                   kvb8 + static_cast<long>(s) * a.ld_kv8, KV8_ROW_BYTES, rb);
+        if (!dequant_pending()) {
+          ok = false;
+          break;
+        }
+        pend_stage = stage;
+        pend_ph = ph;
+        pend_valid = valid;
+      } else {
+        const uint32_t fb = smem_u32(&sm.full[stage]);
+        if (lane == 0)
+          mbar_arrive_expect_tx(fb, __popc(valid & (0xFFu << (8 * pw))) * AT_ROW_BYTES);
+        __syncwarp();
+        if (mine && s >= 0)
+          bulk_g2s(kv0 + (stage * AT_BK + lane) * AT_ROWB, kvb + static_cast<long>(s) * a.ld_kv,
+                   AT_ROW_BYTES, fb);
+      }
       ++issued;
       if (++stage == AT_STAGES) {
         stage = 0;
@@ -279,13 +367,14 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
     }
     if (!ok) break;
   }
+  if (a.kv8 && !*abort) (void)dequant_pending();  // the last tile
   if (*abort) {
     // let every copy still in flight land before the CTA exits
     volatile int never = 0;
     const long n = issued < AT_STAGES ? issued : AT_STAGES;
     for (long j = issued - n; j < issued; ++j)
-      (void)mbar_wait(smem_u32(&sm.full[j % AT_STAGES]), static_cast<uint32_t>((j / AT_STAGES) & 1),
-                      &never, kErrTimeoutDrain);
+      (void)mbar_wait(smem_u32(a.kv8 ? &sm.rawf[j % AT_STAGES] : &sm.full[j % AT_STAGES]),
+                      static_cast<uint32_t>((j / AT_STAGES) & 1), &never, kErrTimeoutDrain);
     if (qloads > 0) (void)mbar_wait(smem_u32(&sm.qfull), (qloads - 1) & 1, &never, kErrTimeoutDrain);
     for (int b2 = 0; b2 < 2; ++b2)
       if (ipending[b2]) (void)mbar_wait(smem_u32(&sm.ifull[b2]), iph[b2], &never, kErrTimeoutDrain);
@@ -521,6 +610,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const AttnArgs 
     mbar_init(smem_u32(&sm.ifull[0]), 1);
     mbar_init(smem_u32(&sm.ifull[1]), 1);
     mbar_init(smem_u32(&sm.pitem), AT_PRODUCERS);
+    for (int st = 0; st < AT_STAGES; ++st) mbar_init(smem_u32(&sm.rawf[st]), AT_PRODUCERS);
     sm.abort = 0;
     fence_barrier_init();
   }
@@ -644,7 +734,8 @@ size_t attn_mla_ws_bytes(int batch, int rows, int k) {
 
 ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* idx, int batch,
                           int rows, int Lkv, int k, float scale, void* out, float* lse, void* ws,
-                          size_t ws_bytes, long long valid_entries, cudaStream_t stream) {
+                          size_t ws_bytes, long long valid_entries, cudaStream_t stream,
+                          bool kv8) {
   const long items = static_cast<long>(batch) * rows;
   if (items == 0) return IC_OK;
   SplitPlan p = split_plan(items, k);
@@ -654,8 +745,11 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
     p.split = false;
   AttnArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
-  a.kv = static_cast<const __nv_bfloat16*>(kv);
-  a.ld_kv = ld_kv;
+  a.kv = kv8 ? nullptr : static_cast<const __nv_bfloat16*>(kv);
+  a.ld_kv = kv8 ? 0 : ld_kv;
+  a.kv8 = kv8 ? 1 : 0;
+  a.kv8p = kv8 ? static_cast<const uint8_t*>(kv) : nullptr;
+  a.ld_kv8 = kv8 ? ld_kv : 0;
   a.idx = idx;
   a.B = batch;
   a.R = rows;
@@ -686,7 +780,8 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
   const double ve = valid_entries >= 0 ? static_cast<double>(valid_entries)
                                        : static_cast<double>(items) * k;
   const double io = static_cast<double>(items) * AT_H * (AT_DK + AT_DV) * 2.0;
-  trace_launch(kKindAttnMla, stream, ve * AT_DK * 2.0 + io + 4.0 * static_cast<double>(items) * k);
+  trace_launch(kv8 ? kKindAttnMlaKv8 : kKindAttnMla, stream,
+               ve * (kv8 ? KV8_ROW_BYTES : AT_DK * 2.0) + io + 4.0 * static_cast<double>(items) * k);
   if (!p.split) return IC_OK;
   static_assert(AT_DV == 4 * 128, "combine: 128 threads x 4 dims");
   st = cuda_check(launch_dep(attn_combine_kernel, dim3(static_cast<unsigned>(items), AT_H), dim3(128),

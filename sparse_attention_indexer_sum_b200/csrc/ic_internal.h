@@ -56,6 +56,8 @@ enum LaunchKind : int {
   kKindTopkMerge = 10,
   kKindIndexerTopkBf16 = 11,
   kKindIndexerTopkE4m3 = 12,
+  kKindAttnMlaKv8 = 13,
+  kKindPackKv = 14,
 };
 // Called after every kernel launch: when tracing is on for this host thread,
 // records an event on `stream` with the launch's kind and algorithmic work
@@ -90,9 +92,12 @@ ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0,
                       cudaStream_t stream, const int* valid_len = nullptr);
 // valid_entries: number of index entries >= 0 over all rows if the caller knows
 // it (the causal stack does), else -1 (rows * k is assumed for tracing only).
+// kv8: kv holds fp8 latent rows (KV8_ROW_BYTES, ld_kv in bytes), else bf16 rows
+// (ld_kv in elements).
 ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* idx, int batch,
                           int rows, int Lkv, int k, float scale, void* out, float* lse,
-                          void* ws, size_t ws_bytes, long long valid_entries, cudaStream_t stream);
+                          void* ws, size_t ws_bytes, long long valid_entries, cudaStream_t stream,
+                          bool kv8 = false);
 size_t attn_mla_ws_bytes(int batch, int rows, int k);
 ic_status launch_attn_f32(const float* q, const float* kv, long ld_kv, const float* v,
                           const int* idx, int batch, int rows, int heads, int dk, int dv,
@@ -100,5 +105,10 @@ ic_status launch_attn_f32(const float* q, const float* kv, long ld_kv, const flo
                           cudaStream_t stream);
 ic_status launch_quant_e4m3(const void* x, bool bf16, long rows, int n, uint8_t* codes,
                             float* scales, cudaStream_t stream);
+// fp8 latent-KV cache rows (656 bytes: 512 e4m3 codes, 4 fp32 group scales, 64 bf16
+// rope dims) of bf16 latent rows [rows, ld_kv >= 576].
+constexpr int KV8_ROW_BYTES = 656;
+ic_status launch_pack_kv_e4m3(const void* kv, long rows, long ld_kv, uint8_t* out, long ld_out,
+                              cudaStream_t stream);
 
 }  // namespace ic

@@ -56,13 +56,14 @@ struct IdxTcArgs {
   int topk;              // k of the selection
 };
 
-// Fused top-k slot: a 64-byte header {int count; int pad; uint64 tau} and then
-// `count` selection keys (select_key) of one epilogue set's share of one row's
-// keys in one CTA: every key of that share with selection key >= tau; when tau
-// is not 0, at least k of them.
-constexpr int FUSED_CB = 4096;                         // candidate buffer per set
+// Fused top-k slot: a 64-byte header {int count; int pad; uint64 tau; uint64 max}
+// and then `count` selection keys (select_key) of one row's keys in one CTA:
+// every key of that share with selection key >= tau; when tau is not 0, at least
+// k of them; max is the largest.
+constexpr int FUSED_CB = 8192;                         // candidate buffer of a CTA
 constexpr size_t FUSED_SLOT_BYTES = 64 + 8 * FUSED_CB;
-constexpr int FUSED_NSETS = 3;                         // epilogue sets of the TPM = 1 instance
+constexpr int FUSED_NSTG = 24;                         // staged tiles of scores
+constexpr int FUSED_SELW = 4;                          // selector warps
 
 template <bool FP8, int TPM, bool FUSED = false>
 struct IdxCfg {
@@ -76,8 +77,9 @@ struct IdxCfg {
   static constexpr int KSTEPS = FP8 ? 4 : 8;       // MMAs per tile (K = 32 / 16 each)
   static constexpr int A_BYTES = BM * ROWB;        // one key tile
   static constexpr int Q_BYTES = N * ROWB;         // the query block
-  // the fused top-k's candidate buffers take the shared memory of some ring stages
-  static constexpr int STAGES = FUSED ? (FP8 ? 6 : 2) : (FP8 ? 8 : 4);
+  // the fused top-k's staging ring and candidate buffer take the shared memory
+  // of some key ring stages
+  static constexpr int STAGES = FP8 ? 8 : 4;
   static constexpr int NACC = (TPM == 4) ? 2 : 6;  // TMEM accumulators in the ring
   static constexpr int TMEM_COLS = (NACC * N <= 256) ? 256 : 512;
   static constexpr int EPG = (TPM == 4) ? 2 : 1;   // epilogue warps per TMEM lane quadrant
@@ -101,7 +103,13 @@ struct IdxCfg {
   static_assert(STAGES % MMAW == 0, "every use of a ring stage falls to one MMA warp");
   static_assert(NACC % MMAW == 0, "every use of an accumulator falls to one MMA warp");
   static constexpr int EPI_W0 = 1 + MMAW;  // first epilogue warp
-  static constexpr int THREADS = 32 * (EPI_W0 + NEPI);
+  // fused top-k: selector warps after the epilogue warps consume the tiles'
+  // scores from a staging ring of NSTG tiles (a multiple of NSETS, so that every
+  // use of a staging slot falls to the same epilogue set)
+  static constexpr int NSEL = FUSED ? FUSED_SELW : 0;
+  static constexpr int SEL_W0 = EPI_W0 + NEPI;
+  static constexpr int NSTG = FUSED ? FUSED_NSTG : 0;
+  static constexpr int THREADS = 32 * (EPI_W0 + NEPI + NSEL);
   // TMEM columns an epilogue thread loads at a time: 16, so that the head
   // weights of both its tokens fit in registers beside them
   static constexpr int EPI_COLS = 16;  // matches tmem_ld16
@@ -110,17 +118,18 @@ struct IdxCfg {
   static constexpr int OFF_W = OFF_Q + Q_BYTES;
   static constexpr int W_FLOATS = NEPI * TOK_PER_EW * 64;
   static constexpr int OFF_BAR = OFF_W + W_FLOATS * 4;
-  static constexpr int NBAR = 2 * STAGES + 2 * NACC + 3;
-  // fused top-k: per epilogue set, a buffer of FUSED_CB selection keys, a 256-bin
-  // radix histogram and 64 ints of scratch
+  static constexpr int NBAR = 2 * STAGES + 2 * NACC + 3 + 2 * NSTG + (FUSED ? 2 : 0);
+  // fused top-k: the staging ring (NSTG x 128 fp32 scores), the candidate buffer
+  // of FUSED_CB selection keys, a 256-bin radix histogram and 64 ints of scratch
   static constexpr int CB = FUSED ? FUSED_CB : 0;
-  static constexpr int OFF_CBUF = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;
-  static constexpr int OFF_CHIST = OFF_CBUF + NSETS * CB * 8;
-  static constexpr int OFF_CX = OFF_CHIST + (FUSED ? NSETS * 256 * 4 : 0);
-  static constexpr int OFF_MISC = OFF_CX + (FUSED ? NSETS * 64 * 4 : 0);
+  static constexpr int OFF_STG = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;
+  static constexpr int OFF_CBUF = OFF_STG + NSTG * BM * 4;
+  static constexpr int OFF_CHIST = OFF_CBUF + CB * 8;
+  static constexpr int OFF_CX = OFF_CHIST + (FUSED ? 256 * 4 : 0);
+  static constexpr int OFF_MISC = OFF_CX + (FUSED ? 96 * 4 : 0);
   static constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;  // + alignment slack
-  static_assert(!FUSED || (TPM == 1 && NSETS == FUSED_NSETS && SETW == 4),
-                "the fused top-k runs in the one-token instance, 3 sets of 4 warps");
+  static_assert(!FUSED || (TPM == 1 && NSTG % NSETS == 0 && SETW == 4),
+                "the fused top-k runs in the one-token instance");
   static_assert(A_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0, "swizzle atoms need 1 KB alignment");
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -156,38 +165,44 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------------ fused top-k
-// Each epilogue set (4 warps, one thread per key of a tile) keeps, for the row it
-// is working on, a shared-memory buffer of selection keys with a rising
-// threshold tau: a key of the set's tiles enters when its selection key is >=
-// tau; when the buffer fills up, a radix descent finds a new tau with at least k
-// and at most `target` buffered keys >= tau, and the buffer is compacted to
-// those.  Keys below tau have at least k larger keys in the same set's share of
-// the row, so they cannot be among the row's top k: the buffer always holds
-// every candidate.  At the end of the row (or of the CTA's work) the buffer goes
-// to its slot in global memory.
+// The epilogue warps leave each tile's 128 scores in a staging ring; 4 selector
+// warps (one thread per key of a tile) walk the tiles in order and keep, for the
+// row they are working on, a shared-memory buffer of selection keys with a
+// rising threshold tau: a key enters when its selection key is >= tau; when the
+// buffer fills up, a radix descent finds a new tau with at least k and at most
+// `target` buffered keys >= tau, and the buffer is compacted to those.  Keys
+// below tau have at least k larger keys in the same CTA's share of the row, so
+// they cannot be among the row's top k: the buffer always holds every
+// candidate.  At the end of the row (or of the CTA's work) the buffer goes to its
+// slot in global memory.  Selection runs beside the tensor-core pipeline: a
+// compaction only delays the selectors, which the staging ring absorbs.
 //
-// The 4 warps of a set meet on a named barrier (one id per set).  Every warp
-// reaches every barrier: the only wait on another role (the accumulator) is
-// bounded, and a warp whose wait gave up raises the set's `dead` flag and still
-// arrives; the set reads the flag right after the barrier and leaves together.
+// The selectors meet on named barrier 1.  Every selector warp reaches every
+// barrier: the only wait on another role (a staged tile) is bounded, and a warp
+// whose wait gave up raises the `dead` flag and still arrives; the selectors read
+// the flag right after the barrier and leave together.
 struct CandSet {
   uint64_t* buf;   // [FUSED_CB]
   uint32_t* hist;  // [256]
-  int* x;          // [64]: 0..7 warp sums and 8..15 chosen bin (by round parity), 16..19
-                   // survivor counts, 20..27 per-tile counts, 30 dead flag, 32..47
-                   // per-warp min and max (as 8 uint64)
-  int bar_id;
-  // The warp reconverges first, and the barrier is the non-aligned form, which
-  // counts threads one by one: the set's barriers follow lane-0-only stores.
-  __device__ __forceinline__ void sync() const {
+  int* x;          // [96]: 0..7 warp sums and 8..15 chosen bin (by round parity),
+                   // 16..23 per-round counts, 48..63 per-warp min and max (8 uint64),
+                   // 64.. the streamer's request (op, count, target, tau as uint64)
+  uint32_t bar;    // group barrier (mbarrier, 4 arrivals: lane 0 of each selector warp)
+  uint32_t phase;  // its phase parity, the same in every selector thread
+  volatile int* abort;
+  // Bounded: false if the CTA aborted (the group's results are void then).
+  __device__ __forceinline__ bool sync() {
     __syncwarp();
-    asm volatile("barrier.sync %0, %1;" ::"r"(bar_id), "r"(128) : "memory");
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_poll(bar, phase, abort, kErrTimeoutEpilogue));
+    phase ^= 1u;
+    return ok;
   }
-  __device__ __forceinline__ uint64_t* mm() const { return reinterpret_cast<uint64_t*>(x + 32); }
+  __device__ __forceinline__ uint64_t* mm() const { return reinterpret_cast<uint64_t*>(x + 48); }
 };
 
-// Min and max of the buffered keys over the set (every thread gets them).
-__device__ __forceinline__ void cand_minmax(const CandSet& cs, int cnt, int t, uint64_t& mn,
+// Min and max of the buffered keys (every thread gets them).
+__device__ __forceinline__ bool cand_minmax(CandSet& cs, int cnt, int t, uint64_t& mn,
                                             uint64_t& mx) {
   const int lane = t & 31, wid = t >> 5;
   mn = ~0ull;
@@ -208,58 +223,29 @@ __device__ __forceinline__ void cand_minmax(const CandSet& cs, int cnt, int t, u
     cs.mm()[wid] = mn;
     cs.mm()[4 + wid] = mx;
   }
-  cs.sync();
+  if (!cs.sync()) return false;
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     const uint64_t a = cs.mm()[w], b = cs.mm()[4 + w];
     mn = a < mn ? a : mn;
     mx = b > mx ? b : mx;
   }
+  return true;
 }
 
-// The new threshold and the compaction.  Every thread of the set calls it with the
+// The new threshold and the compaction.  Every selector thread calls it with the
 // same cnt and tau (kept in registers, identical in every thread) and t = its
-// index in the set (0..127).  Thread t holds buffer entries t + 128 j (j < 32) in
-// registers for the whole call: the buffer is read once, the radix rounds start
-// below the bits that every buffered key shares (8-bit digits, one shared atomic
-// per distinct bin per warp), and the survivors are written back from registers.
-constexpr int CAND_PER_THREAD = FUSED_CB / 128;
-__device__ __forceinline__ void cand_compact(const CandSet cs, int& cnt_io, uint64_t& tau, int k,
+// index (0..127).  The radix rounds start below the bits that every buffered key
+// shares, with 8-bit digits, and count with one shared atomic per distinct bin
+// per warp; the survivors are moved down in place, 128 entries per round (a
+// round's reads precede its writes, which land below the next round's reads).
+__device__ __noinline__ bool cand_compact(CandSet& cs, int& cnt_io, uint64_t& tau, int k,
                                           int target, int t) {
   const int lane = t & 31, wid = t >> 5;
   const int cnt = cnt_io;
-  cs.sync();  // this tile's keys are in the buffer
-  uint64_t c[CAND_PER_THREAD];
-  uint64_t mn = ~0ull, mx = 0ull;
-#pragma unroll
-  for (int j = 0; j < CAND_PER_THREAD; ++j) {
-    const int i = t + 128 * j;
-    c[j] = (i < cnt) ? cs.buf[i] : 0ull;
-    if (i < cnt) {
-      mn = c[j] < mn ? c[j] : mn;
-      mx = c[j] > mx ? c[j] : mx;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const uint64_t a = __shfl_xor_sync(0xffffffffu, mn, o);
-    const uint64_t b = __shfl_xor_sync(0xffffffffu, mx, o);
-    mn = a < mn ? a : mn;
-    mx = b > mx ? b : mx;
-  }
-  if (lane == 0) {
-    cs.mm()[wid] = mn;
-    cs.mm()[4 + wid] = mx;
-  }
-  cs.hist[t] = 0u;
-  cs.hist[t + 128] = 0u;
-  cs.sync();
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    const uint64_t a = cs.mm()[w], b = cs.mm()[4 + w];
-    mn = a < mn ? a : mn;
-    mx = b > mx ? b : mx;
-  }
+  if (!cs.sync()) return false;  // the streamer's keys are in the buffer
+  uint64_t mn, mx;
+  if (!cand_minmax(cs, cnt, t, mn, mx)) return false;
   int pbits = (mn == mx) ? 63 : __clzll(static_cast<long long>(mn ^ mx));
   uint64_t prefix = pbits == 0 ? 0ull : (mn >> (64 - pbits));
   int need = k, above = 0;
@@ -267,20 +253,21 @@ __device__ __forceinline__ void cand_compact(const CandSet cs, int& cnt_io, uint
   for (int round = 0;; ++round) {
     const int bits = (64 - pbits) < 8 ? 64 - pbits : 8;
     const int shift = 64 - pbits - bits;
-    if (round > 0) {  // the first round's bins were cleared above
-      cs.hist[t] = 0u;
-      cs.hist[t + 128] = 0u;
-      cs.sync();
-    }
-#pragma unroll
-    for (int j = 0; j < CAND_PER_THREAD; ++j) {
+    cs.hist[t] = 0u;
+    cs.hist[t + 128] = 0u;
+    if (!cs.sync()) return false;
+    for (int base = 0; base < cnt; base += 128) {
+      const int i = base + t;
       int bin = -1;
-      if (t + 128 * j < cnt && (pbits == 0 || (c[j] >> (64 - pbits)) == prefix))
-        bin = static_cast<int>((c[j] >> shift) & ((1ull << bits) - 1ull));
+      if (i < cnt) {
+        const uint64_t c = cs.buf[i];
+        if (pbits == 0 || (c >> (64 - pbits)) == prefix)
+          bin = static_cast<int>((c >> shift) & ((1ull << bits) - 1ull));
+      }
       const unsigned peers = __match_any_sync(0xffffffffu, bin);
       if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cs.hist[bin], __popc(peers));
     }
-    cs.sync();
+    if (!cs.sync()) return false;
     // thread t owns bins 2t and 2t + 1; count the keys in higher bins
     const int h1 = static_cast<int>(cs.hist[2 * t + 1]), h0 = static_cast<int>(cs.hist[2 * t]);
     const int v = h0 + h1;
@@ -291,7 +278,7 @@ __device__ __forceinline__ void cand_compact(const CandSet cs, int& cnt_io, uint
       if (lane + o < 32) incl += y;
     }
     if (lane == 0) cs.x[4 * (round & 1) + wid] = incl;
-    cs.sync();
+    if (!cs.sync()) return false;
     int higher = 0;
     for (int w = wid + 1; w < 4; ++w) higher += cs.x[4 * (round & 1) + w];
     const int gt1 = higher + incl - v, gt0 = gt1 + h1;
@@ -306,8 +293,8 @@ __device__ __forceinline__ void cand_compact(const CandSet cs, int& cnt_io, uint
       xb[1] = gt0;
       xb[2] = h0;
     }
-    cs.sync();
-    const uint64_t pre = (prefix << bits) | static_cast<uint64_t>(xb[0]);
+    if (!cs.sync()) return false;
+    const uint64_t pre = (prefix << bits) | static_cast<uint64_t>(xb[0] & 255);
     const int gt = xb[1], inb = xb[2];
     pbits += bits;
     if (above + gt + inb <= target || pbits == 64) {  // keys >= the bin's lower edge
@@ -318,49 +305,31 @@ __device__ __forceinline__ void cand_compact(const CandSet cs, int& cnt_io, uint
     need -= gt;
     prefix = pre;
   }
-  // the survivors, written back from registers (every read is done: the barriers
-  // of the rounds come after them)
-  int kept = 0;
-#pragma unroll
-  for (int j = 0; j < CAND_PER_THREAD; ++j) kept += (t + 128 * j < cnt && c[j] >= tnew) ? 1 : 0;
-  int incl = kept;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+  int wpos = 0;
+  for (int base = 0, par = 0; base < cnt; base += 128, par ^= 1) {
+    const int i = base + t;
+    uint64_t c = 0;
+    bool keep = false;
+    if (i < cnt) {
+      c = cs.buf[i];
+      keep = c >= tnew;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) cs.x[16 + 4 * par + wid] = __popc(m);
+    if (!cs.sync()) return false;
+    int off = 0, tot = 0;
+    for (int w = 0; w < 4; ++w) {
+      const int n = cs.x[16 + 4 * par + w];
+      off += (w < wid) ? n : 0;
+      tot += n;
+    }
+    const int dst = wpos + off + __popc(m & ((1u << lane) - 1u));
+    if (keep && dst < FUSED_CB) cs.buf[dst] = c;
+    wpos += tot;
   }
-  if (lane == 31) cs.x[16 + wid] = incl;
-  cs.sync();
-  int base = incl - kept, total = 0;
-  for (int w = 0; w < 4; ++w) {
-    const int n = cs.x[16 + w];
-    base += (w < wid) ? n : 0;
-    total += n;
-  }
-#pragma unroll
-  for (int j = 0; j < CAND_PER_THREAD; ++j)
-    if (t + 128 * j < cnt && c[j] >= tnew) cs.buf[base++] = c[j];
-  cnt_io = total;
+  cnt_io = wpos < FUSED_CB ? wpos : FUSED_CB;
   if (tnew > tau) tau = tnew;
-  cs.sync();
-}
-
-// Writes the set's buffer to its slot (header: count, tau, largest key) and
-// empties it.
-__device__ __forceinline__ void cand_flush(const CandSet& cs, int& cnt, uint64_t& tau,
-                                           uint8_t* slot, int t) {
-  cs.sync();  // the last tile's keys are in the buffer
-  uint64_t mn, mx;
-  cand_minmax(cs, cnt, t, mn, mx);
-  uint64_t* dst = reinterpret_cast<uint64_t*>(slot + 64);
-  for (int i = t; i < cnt; i += 128) dst[i] = cs.buf[i];
-  if (t == 0) {
-    *reinterpret_cast<int*>(slot) = cnt;
-    *reinterpret_cast<uint64_t*>(slot + 8) = tau;
-    *reinterpret_cast<uint64_t*>(slot + 16) = mx;
-  }
-  cnt = 0;
-  tau = 0;
+  return cs.sync();
 }
 
 template <bool FP8, int TPM, bool FUSED>
@@ -382,6 +351,13 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
   const uint32_t qfull_bar = bar0 + 8u * (2 * C::STAGES + 2 * C::NACC);
   const uint32_t qempty_bar = qfull_bar + 8;
   const uint32_t mmadone_bar = qfull_bar + 16;
+  // fused top-k: staging slot s holds a tile's scores (full: 4 epilogue warps
+  // arrive; empty: the selector warps arrive)
+  auto stgfull_bar = [&](int s) { return mmadone_bar + 8u * (1 + s); };
+  auto stgempty_bar = [&](int s) { return mmadone_bar + 8u * (1 + C::NSTG + s); };
+  // the streaming selector's requests to its helpers, and the selector group barrier
+  const uint32_t selreq_bar = mmadone_bar + 8u * (1 + 2 * C::NSTG);
+  const uint32_t selgrp_bar = selreq_bar + 8;
 
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -407,9 +383,15 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
       mbar_init(qfull_bar, 1);
       mbar_init(qempty_bar, C::MMAW);
       mbar_init(mmadone_bar, C::MMAW);
-      if constexpr (FUSED)
-        for (int j = 0; j < C::NSETS; ++j)
-          reinterpret_cast<int*>(smem + C::OFF_CX)[64 * j + 30] = 0;  // the sets' dead flags
+      if constexpr (FUSED) {
+        for (int j = 0; j < C::NSTG; ++j) {
+          mbar_init(stgfull_bar(j), C::SETW);
+          mbar_init(stgempty_bar(j), 1);
+        }
+        mbar_init(selreq_bar, 1);
+        mbar_init(selgrp_bar, C::NSEL);
+        for (int j = 0; j < 96; ++j) reinterpret_cast<int*>(smem + C::OFF_CX)[j] = 0;
+      }
       *abort_flag = 0;
       fence_barrier_init();
       fence_proxy_async_smem();
@@ -557,7 +539,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
         tc_commit(mmadone_bar);
         mbar_wait_drain(mmadone_bar, 0);
       }
-    } else {
+    } else if (warp < C::SEL_W0) {
       // ------------------------------------------------------------ epilogue
       const int e = warp - C::EPI_W0;
       const int qd = warp & 3;     // TMEM lane quadrant this warp may access
@@ -575,33 +557,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
       for (int t = 0; t < C::TOK_PER_EW; ++t)
 #pragma unroll
         for (int h = 0; h < 64; ++h) wr[t][h] = 0.f;
-      // fused top-k state of this set (identical in its 128 threads)
-      const int swid = e % 4, st = swid * 32 + lane;  // warp and thread index in the set
-      CandSet cs{};
-      int ccnt = 0, tpar = 0, crow = -1;
-      uint64_t ctau = 0;
-      long crow_first = 0;  // first CTA of the current row
-      bool dead = false;
-      if constexpr (FUSED) {
-        cs.buf = reinterpret_cast<uint64_t*>(smem + C::OFF_CBUF) + set * C::CB;
-        cs.hist = reinterpret_cast<uint32_t*>(smem + C::OFF_CHIST) + set * 256;
-        cs.x = reinterpret_cast<int*>(smem + C::OFF_CX) + set * 64;
-        cs.bar_id = 1 + set;
-      }
-      auto slot_of = [&](int row) {
-        const long piece = static_cast<long>(blockIdx.x) - crow_first;
-        return a.cslots + ((static_cast<long>(row) * a.maxp + piece) * C::NSETS + set) *
-                              static_cast<long>(FUSED_SLOT_BYTES);
-      };
+      float* stg = reinterpret_cast<float*>(smem + C::OFF_STG);  // fused: staged scores
       for (long i = 0; i < nitems; ++i) {
-        if constexpr (FUSED) {
-          // every set walks every item, so all of them see each row change
-          if (it.qb != crow) {
-            if (crow >= 0) cand_flush(cs, ccnt, ctau, slot_of(crow), st);
-            crow = it.qb;
-            crow_first = ((g0 + i - it.kt) * gridDim.x + gridDim.x - 1) / a.total_tiles;
-          }
-        }
         if (C::NSETS > 1 && acc % C::NSETS != set) {  // another set's slot
           if (++acc == C::NACC) {
             acc = 0;
@@ -642,9 +599,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
         // every lane leaves together, so the warp never splits before tcgen05.ld
         const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(accfull_bar(acc), aph, abort_flag,
                                                               kErrTimeoutEpilogue));
-        if (!FUSED && !acc_ok) break;
-        float res[C::TOK_PER_EW] = {};
-        if (acc_ok) {
+        if (!acc_ok) break;
+        float res[C::TOK_PER_EW];
         tc_fence_after();
 #pragma unroll
         for (int tk = 0; tk < C::TOK_PER_EW; ++tk) {
@@ -675,33 +631,17 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(accempty_bar(acc));
-        }  // acc_ok
         if constexpr (FUSED) {
-          // one query per sequence: row b, position pos0; the same fp32 score as the
-          // unfused store, as a selection key, offered to the set's buffer
-          const uint64_t ck = select_key(res[0] * ks, static_cast<uint32_t>(s));
-          const bool cand = acc_ok && key_ok && s <= a.pos0 && ck >= ctau;
-          const unsigned m = __ballot_sync(0xffffffffu, cand);
-          if (lane == 0) {
-            cs.x[20 + 4 * tpar + swid] = __popc(m);
-            if (!acc_ok) cs.x[30] = 1;
-          }
-          cs.sync();
-          if (cs.x[30]) {  // a wait of this set gave up: the set leaves together
-            dead = true;
+          // the tile's scores (the same fp32 values the unfused store writes) go to
+          // staging slot i % NSTG, which only this set uses, for the selectors
+          const int sl = static_cast<int>(i % C::NSTG);
+          const uint32_t use = static_cast<uint32_t>(i / C::NSTG);
+          if (!__all_sync(0xffffffffu, mbar_wait(stgempty_bar(sl), (use & 1u) ^ 1u, abort_flag,
+                                                 kErrTimeoutEpilogue)))
             break;
-          }
-          int off = 0, tot = 0;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int n = cs.x[20 + 4 * tpar + w];
-            off += (w < swid) ? n : 0;
-            tot += n;
-          }
-          tpar ^= 1;
-          if (cand) cs.buf[ccnt + off + __popc(m & ((1u << lane) - 1u))] = ck;
-          ccnt += tot;
-          if (ccnt > FUSED_CB - 128) cand_compact(cs, ccnt, ctau, a.topk, FUSED_CB - 1280, st);
+          stg[sl * C::BM + qd * 32 + lane] = res[0] * ks;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(stgfull_bar(sl));
         } else if (key_ok) {
 #pragma unroll
           for (int tk = 0; tk < C::TOK_PER_EW; ++tk) {
@@ -719,9 +659,127 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
         }
         it.advance(a);
       }
+    } else {
+      // ------------------------------------------------------------ selectors (fused)
+      // The first selector warp streams: it takes every tile's 128 scores from the
+      // staging ring (4 keys per lane) and appends the candidates to the buffer,
+      // warp-synchronously.  The other three sleep until it asks them to compact the
+      // buffer with it (or to leave).
       if constexpr (FUSED) {
-        // the last row's candidates (after an abort the results are void anyway)
-        if (crow >= 0 && !dead) cand_flush(cs, ccnt, ctau, slot_of(crow), st);
+        const int wid = warp - C::SEL_W0, t = wid * 32 + lane;
+        CandSet cs{reinterpret_cast<uint64_t*>(smem + C::OFF_CBUF),
+                   reinterpret_cast<uint32_t*>(smem + C::OFF_CHIST),
+                   reinterpret_cast<int*>(smem + C::OFF_CX), selgrp_bar, 0u, abort_flag};
+        int* req = cs.x + 64;  // op (1 compact, 2 leave), count, target; tau at req + 4
+        if (wid == 0) {
+          const float* stg = reinterpret_cast<const float*>(smem + C::OFF_STG);
+          WorkIt<TPM> it{start[0], start[1], qb_tiles<TPM>(a, start[0])};
+          int ccnt = 0, crow = -1;
+          uint64_t ctau = 0;
+          long crow_first = 0;  // first CTA of the current row
+          bool ok = true;
+          auto compact = [&](int target) {  // with the helpers
+            if (!ok) return;
+            if (lane == 0) {
+              req[0] = 1;
+              req[1] = ccnt;
+              req[2] = target;
+              *reinterpret_cast<uint64_t*>(req + 4) = ctau;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(selreq_bar);
+            ok = cand_compact(cs, ccnt, ctau, a.topk, target, t);
+          };
+          // the buffer to the row's slot (header: count, tau, largest key), emptied;
+          // more than 2k keys are first compacted to at most k + 256
+          auto flush = [&](int row) {
+            if (ccnt > 2 * a.topk) compact(a.topk + 256);
+            if (!ok) return;
+            const long piece = static_cast<long>(blockIdx.x) - crow_first;
+            uint8_t* slot = a.cslots + (static_cast<long>(row) * a.maxp + piece) *
+                                           static_cast<long>(FUSED_SLOT_BYTES);
+            uint64_t* dst = reinterpret_cast<uint64_t*>(slot + 64);
+            uint64_t mx = 0;
+            for (int j = lane; j < ccnt; j += 32) {
+              const uint64_t c = cs.buf[j];
+              dst[j] = c;
+              mx = c > mx ? c : mx;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              const uint64_t y = __shfl_xor_sync(0xffffffffu, mx, o);
+              mx = y > mx ? y : mx;
+            }
+            if (lane == 0) {
+              *reinterpret_cast<int*>(slot) = ccnt;
+              *reinterpret_cast<uint64_t*>(slot + 8) = ctau;
+              *reinterpret_cast<uint64_t*>(slot + 16) = mx;
+            }
+            __syncwarp();
+            ccnt = 0;
+            ctau = 0;
+          };
+          for (long i = 0; i < nitems && ok; ++i) {
+            if (it.qb != crow) {
+              if (crow >= 0) flush(crow);
+              crow = it.qb;
+              crow_first = ((g0 + i - it.kt) * gridDim.x + gridDim.x - 1) / a.total_tiles;
+            }
+            const int sl = static_cast<int>(i % C::NSTG);
+            const uint32_t use = static_cast<uint32_t>(i / C::NSTG);
+            if (!__all_sync(0xffffffffu, mbar_wait_poll(stgfull_bar(sl), use & 1u, abort_flag,
+                                                        kErrTimeoutEpilogue))) {
+              ok = false;
+              break;
+            }
+            const float4 v = *reinterpret_cast<const float4*>(stg + sl * C::BM + 4 * lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stgempty_bar(sl));
+            // keys 4 lane .. 4 lane + 3 of the tile: one query per sequence, at pos0
+            const float sv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int s = it.kt * C::BM + 4 * lane + e;
+              const uint64_t ck = select_key(sv[e], static_cast<uint32_t>(s));
+              const bool cand = s < a.Lk && s <= a.pos0 && ck >= ctau;
+              const unsigned m = __ballot_sync(0xffffffffu, cand);
+              if (cand) cs.buf[ccnt + __popc(m & ((1u << lane) - 1u))] = ck;
+              ccnt += __popc(m);
+            }
+            if (ccnt > FUSED_CB - C::BM) compact(3 * FUSED_CB / 8);
+            it.advance(a);
+          }
+          if (crow >= 0 && ok) flush(crow);
+          // the helpers leave
+          __syncwarp();
+          if (lane == 0) {
+            req[0] = 2;
+            mbar_arrive(selreq_bar);
+          }
+        } else {
+          uint32_t rph = 0;
+          for (;;) {
+            // wait for a request: bounded by a long limit (the streamer always ends
+            // with one), or the CTA's abort
+            bool got = mbar_try_wait(selreq_bar, rph);
+            const uint64_t t0 = globaltimer();
+            while (!got) {
+              if (*abort_flag) break;
+              if (globaltimer() - t0 > 30ull * IC_WAIT_NS) {
+                *abort_flag = 1;
+                record_error(kErrTimeoutEpilogue);
+                break;
+              }
+              got = mbar_try_wait(selreq_bar, rph);
+            }
+            if (!__all_sync(0xffffffffu, got)) break;
+            rph ^= 1u;
+            if (req[0] != 1) break;
+            int cnt = req[1];
+            uint64_t tau = *reinterpret_cast<const uint64_t*>(req + 4);
+            if (!cand_compact(cs, cnt, tau, a.topk, req[2], t)) break;
+          }
+        }
       }
     }
   }
@@ -859,7 +917,7 @@ static FusedPlan fused_plan(int batch, int Lk, long pos0) {
 
 size_t indexer_topk_fused_ws_bytes(int batch, int Lk, long pos0) {
   const FusedPlan p = fused_plan(batch, Lk, pos0);
-  return static_cast<size_t>(batch) * p.maxp * FUSED_NSETS * FUSED_SLOT_BYTES;
+  return static_cast<size_t>(batch) * p.maxp * FUSED_SLOT_BYTES;
 }
 
 ic_status launch_indexer_topk_fused(bool fp8, const void* q, const float* q_scale, const void* k,
@@ -870,7 +928,7 @@ ic_status launch_indexer_topk_fused(bool fp8, const void* q, const float* q_scal
   const long nv = pos0 + 1 < Lk ? pos0 + 1 : Lk;
   uint8_t* slots = static_cast<uint8_t*>(ws);
   if (nv > topk) {  // otherwise every candidate is selected: the merge alone writes T
-    const size_t need = static_cast<size_t>(batch) * p.maxp * FUSED_NSETS * FUSED_SLOT_BYTES;
+    const size_t need = static_cast<size_t>(batch) * p.maxp * FUSED_SLOT_BYTES;
     if (!ws || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % 16 != 0)
       return fail(IC_ERR_WORKSPACE,
                   "indexer_topk: needs a 16-byte aligned workspace of %zu bytes (got %zu)", need,
@@ -881,8 +939,8 @@ ic_status launch_indexer_topk_fused(bool fp8, const void* q, const float* q_scal
                                                     pos0, nullptr, Lk, stream, slots, p.maxp, topk);
     if (st) return st;
   }
-  return launch_topk_merge(slots, batch, p.nt, p.total, p.G, p.maxp, FUSED_NSETS,
-                           FUSED_SLOT_BYTES, FUSED_CB, static_cast<int>(nv), topk, idx, stream);
+  return launch_topk_merge(slots, batch, p.nt, p.total, p.G, p.maxp, 1, FUSED_SLOT_BYTES,
+                           FUSED_CB, static_cast<int>(nv), topk, idx, stream);
 }
 
 ic_status launch_indexer_tc(bool fp8, const void* q, const float* q_scale, const void* k,

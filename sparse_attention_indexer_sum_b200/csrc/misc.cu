@@ -53,6 +53,65 @@ ic_status launch_quant_e4m3(const void* x, bool bf16, long rows, int n, uint8_t*
   return st;
 }
 
+// The fp8 latent-KV cache row of a 576-dim bf16 latent row (656 bytes): the 512
+// latent dims as e4m3 codes in four groups of 128, each group quantised as a row
+// of quant_e4m3_kernel (scale = amax / 448, 1 for an all-zero group; code =
+// e4m3_rn_satfinite(x / scale)); the four fp32 scales; the 64 rope dims in bf16.
+// One warp per row: lane l quantises latent dims 16l..16l+15 (group l / 8).
+__global__ void pack_kv_e4m3_kernel(const __nv_bfloat16* __restrict__ kv, long rows, long ld_kv,
+                                    uint8_t* __restrict__ out, long ld_out) {
+  grid_dep_wait();
+  const long row = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const __nv_bfloat16* x = kv + row * ld_kv;
+  uint8_t* o = out + row * ld_out;
+  float v[16];
+  const uint4 a = *reinterpret_cast<const uint4*>(x + 16 * lane);
+  const uint4 b = *reinterpret_cast<const uint4*>(x + 16 * lane + 8);
+  const __nv_bfloat16* pa = reinterpret_cast<const __nv_bfloat16*>(&a);
+  const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(&b);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[i] = __bfloat162float(pa[i]);
+    v[8 + i] = __bfloat162float(pb[i]);
+    amax = fmaxf(amax, fmaxf(fabsf(v[i]), fabsf(v[8 + i])));
+  }
+#pragma unroll
+  for (int off = 4; off > 0; off >>= 1)  // the 8 lanes of the group
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  uint32_t c[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      word |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(v[4 * w + j], scale),
+                                                           __NV_SATFINITE, __NV_E4M3))
+              << (8 * j);
+    c[w] = word;
+  }
+  *reinterpret_cast<uint4*>(o + 16 * lane) = make_uint4(c[0], c[1], c[2], c[3]);
+  if ((lane & 7) == 0) *reinterpret_cast<float*>(o + 512 + 4 * (lane / 8)) = scale;
+  if (lane < 8)  // rope: dims 512..575, 16 bytes per lane
+    *reinterpret_cast<uint4*>(o + 528 + 16 * lane) =
+        *reinterpret_cast<const uint4*>(x + 512 + 8 * lane);
+}
+
+ic_status launch_pack_kv_e4m3(const void* kv, long rows, long ld_kv, uint8_t* out, long ld_out,
+                              cudaStream_t stream) {
+  if (rows == 0) return IC_OK;
+  const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  ic_status st = cuda_check(launch_dep(pack_kv_e4m3_kernel, dim3(blocks), dim3(256), 0, stream, 1,
+                                       static_cast<const __nv_bfloat16*>(kv), rows, ld_kv, out,
+                                       ld_out),
+                            "pack_kv_e4m3_kernel launch");
+  if (!st) trace_launch(kKindPackKv, stream, static_cast<double>(rows) * (576.0 * 2 + 656.0));
+  return st;
+}
+
 // I[b,r,s] = sum_h w[b,r,h] * max(0, q[b,r,h,:] . k[b,s,:]) on CUDA cores.
 // Grid (batch * rows, ceil(Lk / 128)); one key per thread, the query row in smem.
 __global__ void indexer_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,

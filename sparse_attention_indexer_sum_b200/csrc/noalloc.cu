@@ -123,7 +123,8 @@ ic_status ic_sparse_attn_noalloc(const void* q, const void* kv, long ld_kv, cons
   // Every split item writes its whole partial before the merge reads it, so the
   // previous call's contents need no clearing.
   return launch_attn_mla(q, kv, ld_kv, idx, batch, rows, Lkv, k, scale, out, lse, scratch,
-                         IC_NOALLOC_SCRATCH_BYTES, -1, static_cast<cudaStream_t>(stream));
+                         IC_NOALLOC_SCRATCH_BYTES, -1, static_cast<cudaStream_t>(stream),
+                         dt == IC_E4M3);
 }
 
 }  // extern "C"

@@ -145,3 +145,13 @@ def test_topk_varlen_rejects_before_launch(lib):
     fake = ctypes.c_void_p(256)
     assert lib.ic_topk_varlen(fake, 4, 100, 100, None, 8, fake, None) == binding.IC_ERR_INVALID_ARG
     assert lib.ic_topk_varlen(fake, 4, 100, 50, fake, 8, fake, None) == binding.IC_ERR_INVALID_ARG
+
+
+def test_pack_kv_and_fp8_attention_reject_before_launch(lib):
+    fake = ctypes.c_void_p(256)
+    assert lib.ic_pack_kv_e4m3(fake, 4, 570, fake, 656, None) == binding.IC_ERR_INVALID_ARG
+    assert lib.ic_pack_kv_e4m3(fake, 4, 576, fake, 650, None) == binding.IC_ERR_INVALID_ARG
+    # an fp8 cache needs rows of at least 656 bytes, a multiple of 16
+    st = lib.ic_sparse_attn(fake, fake, 576, None, fake, binding.IC_E4M3, 1, 4, 16, 576, 512, 100,
+                            64, 1.0, fake, None, None, 0, None)
+    assert st == binding.IC_ERR_INVALID_ARG

@@ -243,6 +243,56 @@ def test_attn_mla_parity(B, R, k, Lkv):
     np.testing.assert_allclose(lse.cpu().numpy(), rl, atol=2e-3, rtol=1e-3)
 
 
+def test_pack_kv_e4m3_bit_exact():
+    g = torch.Generator().manual_seed(31)
+    kv = torch.randn(333, 576, generator=g) * torch.rand(333, 1, generator=g) * 4
+    kv[7] = 0
+    kv[9, 128:256] = 0            # one all-zero group: scale 1, codes 0
+    kv[11, :128] *= 1e-4          # a tiny group next to large ones
+    kvb = kv.to(torch.bfloat16)
+    packed = ic.ic_pack_kv_e4m3(kvb.to(DEV))
+    _sync()
+    P = packed.cpu().numpy()
+    codes, scales, rope = oracle.kv_pack_e4m3(kvb.float().numpy())
+    np.testing.assert_array_equal(P[:, :512], codes)
+    np.testing.assert_array_equal(P[:, 512:528].view(np.float32), scales)
+    np.testing.assert_array_equal(P[:, 528:].view(np.uint16),
+                                  kvb[:, 512:].view(torch.int16).numpy().view(np.uint16))
+
+
+def _unpack_kv8(P):
+    P = np.ascontiguousarray(P)
+    codes = P[..., :512]
+    scales = np.ascontiguousarray(P[..., 512:528]).view(np.float32)
+    rope = torch.from_numpy(np.ascontiguousarray(P[..., 528:]).view(np.int16)).view(
+        torch.bfloat16).float().numpy()
+    return codes, scales, rope
+
+
+@pytest.mark.parametrize("B,R,k,Lkv", [(1, 37, 2048, 3000), (6, 1, 2048, 4000), (2, 7, 37, 90),
+                                       (64, 1, 2048, 2100)])
+def test_attn_mla_kv8_parity(B, R, k, Lkv):
+    """Absorbed MLA over the fp8 cache (split and unsplit forms, ragged lists, a hole)
+    against the oracle on the dequantised cache rows."""
+    g = torch.Generator().manual_seed(B * 17 + R)
+    q = torch.randn(B, R, 16, 576, generator=g).to(torch.bfloat16)
+    kv = torch.randn(B, Lkv, 576, generator=g).to(torch.bfloat16)
+    pads = [k - (r * 37) % max(1, k // 2) for r in range(R)]
+    idx = _rand_idx(B, R, k, Lkv, seed=R + 5, pad_from=pads)
+    idx[:, 0, 5 % k] = -1
+    packed = ic.ic_pack_kv_e4m3(kv.to(DEV))
+    scale = 1 / math.sqrt(576)
+    ws = torch.empty(ic.ic_attn_workspace_size(B, R, 16, 512, k) // 4 + 1, device=DEV)
+    lse = torch.empty(B, R, 16, device=DEV)
+    out = ic.ic_sparse_attn(q.to(DEV), packed, torch.from_numpy(idx).to(DEV), scale, lse=lse,
+                            workspace=ws)
+    _sync()
+    codes, scales, rope = _unpack_kv8(packed.cpu().numpy())
+    ro, rl = oracle.sparse_attn_kv_e4m3(q.float().numpy(), codes, scales, rope, idx, scale)
+    assert_attn_close(_np(out), ro)
+    np.testing.assert_allclose(lse.cpu().numpy(), rl, atol=2e-3, rtol=1e-3)
+
+
 def test_attn_mla_decode_split_equals_unsplit():
     B, k, Lkv = 6, 2048, 4000
     g = torch.Generator().manual_seed(3)
@@ -505,6 +555,44 @@ def test_decode_step_parity():
         ro, _ = oracle.sparse_attn(h["q"].float().numpy(), h["kv"].float().numpy(), T[:, None, :],
                                    wl.scale, dv=512)
         assert_attn_close(_np(dl[l]["out"]), ro)
+
+
+def test_decode_step_fp8_kv_cache():
+    """Decode over an fp8 latent cache (e4m3 indexer cache too), pattern F,S,S: T
+    against the oracle's scores, every layer's output against the oracle on the
+    dequantised cache rows."""
+    wl = synth.variant("decode_200k", L=4500, batch=5, pattern="F,S,S")
+    layers, host = _stack_layers(wl, DEV)
+    for d in layers:
+        d["q_idx"], d["q_scale"] = ic.ic_quant_e4m3_rows(d["q_idx"])
+        d["k_idx"], d["k_scale"] = ic.ic_quant_e4m3_rows(d["k_idx"])
+        d["kv"] = ic.ic_pack_kv_e4m3(d["kv"])
+    desc = ic.make_desc(L=wl.L, k=wl.k, H=wl.H, D=wl.D, idx_dtype=ic.IC_E4M3, heads=wl.Hq,
+                        dk=wl.Dk, dv=wl.Dv, attn_dtype=ic.IC_E4M3, scale=wl.scale,
+                        ld_kv=ic.KV8_ROW_BYTES, batch=wl.batch, decode=True)
+    dl = []
+    for d in layers:
+        e = dict(d)
+        e["out"] = torch.empty(wl.batch, 1, wl.Hq, wl.Dv, dtype=torch.bfloat16, device=DEV)
+        e["lse"] = torch.empty(wl.batch, 1, wl.Hq, device=DEV)
+        dl.append(e)
+    t_cache = torch.full((wl.batch, wl.k), -7, dtype=torch.int32, device=DEV)
+    ws = torch.empty(ic.ic_stack_workspace_size(desc) // 4 + 1, device=DEV)
+    ic.ic_decode_step(wl.pattern, desc, dl, t_cache, ws)
+    _sync()
+    T = t_cache.cpu().numpy()
+    d0 = layers[0]
+    ref = oracle.indexer_scores_e4m3(d0["q_idx"].cpu().numpy(), d0["q_scale"].cpu().numpy(),
+                                     d0["k_idx"].cpu().numpy(), d0["k_scale"].cpu().numpy(),
+                                     d0["w"].cpu().numpy(), pos0=wl.L - 1)
+    for b in range(wl.batch):
+        check_index_row(T[b], ref[b, 0], wl.k, wl.L)
+    for l in range(3):
+        codes, scales, rope = _unpack_kv8(dl[l]["kv"].cpu().numpy())
+        ro, rl = oracle.sparse_attn_kv_e4m3(host[l]["q"].float().numpy(), codes, scales, rope,
+                                            T[:, None, :], wl.scale)
+        assert_attn_close(_np(dl[l]["out"]), ro)
+        np.testing.assert_allclose(dl[l]["lse"].cpu().numpy(), rl, atol=2e-3, rtol=1e-3)
 
 
 def test_decode_step_two_full_layers_overwrite_t_cache():

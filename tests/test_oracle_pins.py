@@ -359,6 +359,66 @@ def test_attn_golden_hand_worked():
     np.testing.assert_allclose(out[0, 0], [e / (1 + 2 * e), 1 / (1 + 2 * e)], rtol=1e-15)
 
 
+def test_kv_e4m3_pack_groups_and_rope():
+    # each 128-dim latent group has its own scale (amax / 448), so a group of small
+    # values keeps its precision next to a group of large ones; rope is untouched
+    g = np.random.default_rng(21)
+    kv = g.standard_normal((5, 576)).astype(np.float32)
+    kv[:, 128:256] *= 1e-3
+    kv[2, 256:384] = 0.0
+    codes, scales, rope = oracle.kv_pack_e4m3(kv)
+    assert codes.shape == (5, 512) and scales.shape == (5, 4) and rope.shape == (5, 64)
+    for gi in range(4):
+        amax = np.abs(kv[:, 128 * gi:128 * (gi + 1)]).max(axis=1)
+        want = np.where(amax > 0, (amax / np.float32(448)).astype(np.float32), 1.0)
+        np.testing.assert_array_equal(scales[:, gi], want.astype(np.float32))
+    np.testing.assert_array_equal(rope, kv[:, 512:])
+    deq = oracle.kv_dequant_e4m3(codes, scales, rope)
+    # 3 mantissa bits: relative error at most 2^-4 of the group's amax-scaled grid
+    for gi in range(4):
+        sl = slice(128 * gi, 128 * (gi + 1))
+        err = np.abs(deq[:, sl] - kv[:, sl])
+        assert (err <= np.abs(kv[:, sl]) * 2.0 ** -4 + scales[:, gi:gi + 1] * 2.0 ** -9).all()
+    np.testing.assert_array_equal(deq[:, 512:], kv[:, 512:])
+    assert (deq[2, 256:384] == 0).all()
+
+
+def test_kv_e4m3_attention_hand_worked():
+    # the hand-worked example of attn_tiny.txt, carried by an fp8 cache: latent dims
+    # 0..2 hold the example's rows (exact e4m3 values with unit scales), the rest 0
+    d = _read_attn_fixture()
+    rows = np.zeros((4, 576), dtype=np.float64)
+    rows[:, :3] = np.array(d["kv"])
+    codes = np.zeros((4, 512), dtype=np.uint8)
+    for r in range(4):
+        for c in range(3):
+            codes[r, c] = oracle.e4m3_encode(rows[r, c])
+    scales = np.ones((4, 4), dtype=np.float32)
+    rope = np.zeros((4, 64), dtype=np.float32)
+    q = np.zeros((1, 1, 576))
+    q[0, 0, :3] = d["q"]
+    idx = np.array(d["idx"], dtype=np.int32)[None, :]
+    out, lse = oracle.sparse_attn_kv_e4m3(q, codes, scales, rope, idx, 1.0)
+    e = math.e
+    # values are the first 512 latent dims: dim 2 carries row 2's 0.5 as well
+    np.testing.assert_allclose(out[0, 0, :3], [e / (1 + 2 * e), 1 / (1 + 2 * e),
+                                               0.5 * e / (1 + 2 * e)], rtol=1e-15)
+    assert (out[0, 0, 3:] == 0).all()
+    np.testing.assert_allclose(lse[0, 0], d["lse"][0], rtol=1e-15)
+    # a group scale of 2 doubles that group's values: logits of q on group 0 double
+    out2, lse2 = oracle.sparse_attn_kv_e4m3(q, codes, scales * 2, rope, idx, 0.5)
+    np.testing.assert_allclose(out2[0, 0, :2], 2 * out[0, 0, :2], rtol=1e-14)
+    # rope dims take part in the logits but not in the values
+    rope2 = rope.copy()
+    rope2[1, 0] = 1.0
+    q2 = q.copy()
+    q2[0, 0, 512] = math.log(3.0)
+    out3, _ = oracle.sparse_attn_kv_e4m3(q2, codes, scales, rope2, idx, 1.0)
+    w = np.array([1.0, 3 * e, e])   # rows 0, 1, 2: z = 0, 1 + log 3, 1
+    want = (w[1] * np.array([1, 0]) + w[0] * np.array([0, 1])) / w.sum()
+    np.testing.assert_allclose(out3[0, 0, :2], want, rtol=1e-14)
+
+
 def test_attn_single_index_returns_that_value_row():
     g = np.random.default_rng(11)
     R, H, Dk, Dv, L, k = 5, 3, 12, 8, 20, 6
