@@ -62,8 +62,8 @@ struct IdxTcArgs {
 // k of them; max is the largest.
 constexpr int FUSED_CB = 8192;                         // candidate buffer of a CTA
 constexpr size_t FUSED_SLOT_BYTES = 64 + 8 * FUSED_CB;
-constexpr int FUSED_NSTG = 24;                         // staged tiles of scores
 constexpr int FUSED_SELW = 4;                          // selector warps
+constexpr int FUSED_XINTS = 104;                       // selector scratch ints
 
 template <bool FP8, int TPM, bool FUSED = false>
 struct IdxCfg {
@@ -79,7 +79,7 @@ struct IdxCfg {
   static constexpr int Q_BYTES = N * ROWB;         // the query block
   // the fused top-k's staging ring and candidate buffer take the shared memory
   // of some key ring stages
-  static constexpr int STAGES = FP8 ? 8 : 4;
+  static constexpr int STAGES = FP8 ? (FUSED ? 6 : 8) : 4;
   static constexpr int NACC = (TPM == 4) ? 2 : 6;  // TMEM accumulators in the ring
   static constexpr int TMEM_COLS = (NACC * N <= 256) ? 256 : 512;
   static constexpr int EPG = (TPM == 4) ? 2 : 1;   // epilogue warps per TMEM lane quadrant
@@ -108,7 +108,7 @@ struct IdxCfg {
   // use of a staging slot falls to the same epilogue set)
   static constexpr int NSEL = FUSED ? FUSED_SELW : 0;
   static constexpr int SEL_W0 = EPI_W0 + NEPI;
-  static constexpr int NSTG = FUSED ? FUSED_NSTG : 0;
+  static constexpr int NSTG = FUSED ? (FP8 ? 24 : 12) : 0;
   static constexpr int THREADS = 32 * (EPI_W0 + NEPI + NSEL);
   // TMEM columns an epilogue thread loads at a time: 16, so that the head
   // weights of both its tokens fit in registers beside them
@@ -119,14 +119,16 @@ struct IdxCfg {
   static constexpr int W_FLOATS = NEPI * TOK_PER_EW * 64;
   static constexpr int OFF_BAR = OFF_W + W_FLOATS * 4;
   static constexpr int NBAR = 2 * STAGES + 2 * NACC + 3 + 2 * NSTG + (FUSED ? 2 : 0);
-  // fused top-k: the staging ring (NSTG x 128 fp32 scores), the candidate buffer
-  // of FUSED_CB selection keys, a 256-bin radix histogram and 64 ints of scratch
+  // fused top-k: the staging ring (per tile, each epilogue warp's candidate
+  // selection keys, packed, and their count), the candidate buffer of FUSED_CB
+  // selection keys, a 256-bin radix histogram and FUSED_XINTS ints of scratch
   static constexpr int CB = FUSED ? FUSED_CB : 0;
   static constexpr int OFF_STG = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;
-  static constexpr int OFF_CBUF = OFF_STG + NSTG * BM * 4;
+  static constexpr int OFF_SCNT = OFF_STG + NSTG * BM * 8;
+  static constexpr int OFF_CBUF = OFF_SCNT + NSTG * 16;
   static constexpr int OFF_CHIST = OFF_CBUF + CB * 8;
   static constexpr int OFF_CX = OFF_CHIST + (FUSED ? 256 * 4 : 0);
-  static constexpr int OFF_MISC = OFF_CX + (FUSED ? 96 * 4 : 0);
+  static constexpr int OFF_MISC = OFF_CX + (FUSED ? FUSED_XINTS * 4 : 0);
   static constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;  // + alignment slack
   static_assert(!FUSED || (TPM == 1 && NSTG % NSETS == 0 && SETW == 4),
                 "the fused top-k runs in the one-token instance");
@@ -165,28 +167,33 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------------ fused top-k
-// The epilogue warps leave each tile's 128 scores in a staging ring; 4 selector
-// warps (one thread per key of a tile) walk the tiles in order and keep, for the
-// row they are working on, a shared-memory buffer of selection keys with a
-// rising threshold tau: a key enters when its selection key is >= tau; when the
-// buffer fills up, a radix descent finds a new tau with at least k and at most
-// `target` buffered keys >= tau, and the buffer is compacted to those.  Keys
-// below tau have at least k larger keys in the same CTA's share of the row, so
-// they cannot be among the row's top k: the buffer always holds every
-// candidate.  At the end of the row (or of the CTA's work) the buffer goes to its
-// slot in global memory.  Selection runs beside the tensor-core pipeline: a
-// compaction only delays the selectors, which the staging ring absorbs.
+// The epilogue warps leave each tile's 128 scores in a staging ring, with one
+// 32-bit mask per warp of the keys that may be candidates; one streaming selector
+// warp walks the tiles in order and appends those keys' selection keys, in index
+// order, to a shared-memory buffer for the row it is working on.  The buffer has
+// a rising threshold tau: it holds every key of the CTA's share of the row seen so
+// far whose selection key is >= tau (and possibly some below).  When it fills
+// up, the streaming warp and three helper warps find by a radix descent a new
+// tau with at least k and at most `target` buffered keys >= tau, and compact the
+// buffer to those, keeping their order.  A key below tau has at least k larger
+// keys in the same share of the row, so it cannot be among the row's top k.  The
+// streaming warp publishes tau's score key, tagged with the row, and the epilogue
+// leaves keys whose score key is below it out of the masks (a stale value only
+// lets more keys through).  At the end of the row (or of the CTA's work) the
+// buffer goes to the row's slot in global memory.  Selection runs beside the
+// tensor-core pipeline: a compaction only delays the selectors, which the staging
+// ring absorbs.
 //
-// The selectors meet on named barrier 1.  Every selector warp reaches every
-// barrier: the only wait on another role (a staged tile) is bounded, and a warp
-// whose wait gave up raises the `dead` flag and still arrives; the selectors read
-// the flag right after the barrier and leave together.
+// The four selector warps meet on an mbarrier (one arrival per warp) that each
+// waits on by polling, bounded in time and by the CTA's abort flag; a warp whose
+// wait gave up returns false and the selectors leave.
 struct CandSet {
   uint64_t* buf;   // [FUSED_CB]
   uint32_t* hist;  // [256]
-  int* x;          // [96]: 0..7 warp sums and 8..15 chosen bin (by round parity),
-                   // 16..23 per-round counts, 48..63 per-warp min and max (8 uint64),
-                   // 64.. the streamer's request (op, count, target, tau as uint64)
+  int* x;          // [FUSED_XINTS]: 0..7 warp sums and 8..15 the chosen bin (by
+                   // round parity), 16..79 per-round counts of a compaction (by
+                   // round parity, 8 x 4 each), 96.. the streamer's request (op,
+                   // count, target, -, tau and the buffer's largest key as uint64)
   uint32_t bar;    // group barrier (mbarrier, 4 arrivals: lane 0 of each selector warp)
   uint32_t phase;  // its phase parity, the same in every selector thread
   volatile int* abort;
@@ -198,76 +205,52 @@ struct CandSet {
     phase ^= 1u;
     return ok;
   }
-  __device__ __forceinline__ uint64_t* mm() const { return reinterpret_cast<uint64_t*>(x + 48); }
 };
 
-// Min and max of the buffered keys (every thread gets them).
-__device__ __forceinline__ bool cand_minmax(CandSet& cs, int cnt, int t, uint64_t& mn,
-                                            uint64_t& mx) {
-  const int lane = t & 31, wid = t >> 5;
-  mn = ~0ull;
-  mx = 0ull;
-  for (int i = t; i < cnt; i += 128) {
-    const uint64_t c = cs.buf[i];
-    mn = c < mn ? c : mn;
-    mx = c > mx ? c : mx;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const uint64_t a = __shfl_xor_sync(0xffffffffu, mn, o);
-    const uint64_t b = __shfl_xor_sync(0xffffffffu, mx, o);
-    mn = a < mn ? a : mn;
-    mx = b > mx ? b : mx;
-  }
-  if (lane == 0) {
-    cs.mm()[wid] = mn;
-    cs.mm()[4 + wid] = mx;
-  }
-  if (!cs.sync()) return false;
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    const uint64_t a = cs.mm()[w], b = cs.mm()[4 + w];
-    mn = a < mn ? a : mn;
-    mx = b > mx ? b : mx;
-  }
-  return true;
-}
-
 // The new threshold and the compaction.  Every selector thread calls it with the
-// same cnt and tau (kept in registers, identical in every thread) and t = its
-// index (0..127).  The radix rounds start below the bits that every buffered key
-// shares, with 8-bit digits, and count with one shared atomic per distinct bin
-// per warp; the survivors are moved down in place, 128 entries per round (a
-// round's reads precede its writes, which land below the next round's reads).
-__device__ __noinline__ bool cand_compact(CandSet& cs, int& cnt_io, uint64_t& tau, int k,
-                                          int target, int t) {
+// same cnt, tau and hi (kept in registers, identical in every thread) and t = its
+// index (0..127).  hi is the largest buffered key; the buffer holds at least k
+// keys >= tau when tau != 0, so the k-th largest lies in [tau, hi] and the radix
+// rounds start below the bits those two share, with 8-bit digits.  The survivors
+// move down in place, 1024 entries per round in their original order (a round's
+// reads precede its writes, which land below the next round's reads).
+struct CompactResult {
+  uint64_t tau;
+  int cnt;
+  uint32_t phase;  // the group barrier's parity afterwards
+  bool ok;
+};
+__device__ __noinline__ CompactResult cand_compact(CandSet cs, const int cnt, uint64_t tau,
+                                                   uint64_t hi, int k, int target, int t) {
   const int lane = t & 31, wid = t >> 5;
-  const int cnt = cnt_io;
-  if (!cs.sync()) return false;  // the streamer's keys are in the buffer
-  uint64_t mn, mx;
-  if (!cand_minmax(cs, cnt, t, mn, mx)) return false;
-  int pbits = (mn == mx) ? 63 : __clzll(static_cast<long long>(mn ^ mx));
-  uint64_t prefix = pbits == 0 ? 0ull : (mn >> (64 - pbits));
+  CompactResult fail{tau, cnt, 0u, false};
+  if (!cs.sync()) return fail;  // the streamer's keys are in the buffer
+  int pbits = (tau >= hi) ? 63 : __clzll(static_cast<long long>(tau ^ hi));
+  uint64_t prefix = pbits == 0 ? 0ull : (tau >> (64 - pbits));
   int need = k, above = 0;
   uint64_t tnew;
   for (int round = 0;; ++round) {
     const int bits = (64 - pbits) < 8 ? 64 - pbits : 8;
     const int shift = 64 - pbits - bits;
+    const uint64_t dmask = (1ull << bits) - 1ull;
     cs.hist[t] = 0u;
     cs.hist[t + 128] = 0u;
-    if (!cs.sync()) return false;
-    for (int base = 0; base < cnt; base += 128) {
-      const int i = base + t;
-      int bin = -1;
-      if (i < cnt) {
-        const uint64_t c = cs.buf[i];
-        if (pbits == 0 || (c >> (64 - pbits)) == prefix)
-          bin = static_cast<int>((c >> shift) & ((1ull << bits) - 1ull));
+    if (!cs.sync()) return fail;
+    for (int base = 0; base < cnt; base += 1024) {
+      uint64_t c[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + 128 * j + t;
+        c[j] = i < cnt ? cs.buf[i] : 0ull;
       }
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cs.hist[bin], __popc(peers));
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + 128 * j + t;
+        if (i < cnt && (pbits == 0 || (c[j] >> (64 - pbits)) == prefix))
+          atomicAdd(&cs.hist[static_cast<int>((c[j] >> shift) & dmask)], 1u);
+      }
     }
-    if (!cs.sync()) return false;
+    if (!cs.sync()) return fail;
     // thread t owns bins 2t and 2t + 1; count the keys in higher bins
     const int h1 = static_cast<int>(cs.hist[2 * t + 1]), h0 = static_cast<int>(cs.hist[2 * t]);
     const int v = h0 + h1;
@@ -278,7 +261,7 @@ __device__ __noinline__ bool cand_compact(CandSet& cs, int& cnt_io, uint64_t& ta
       if (lane + o < 32) incl += y;
     }
     if (lane == 0) cs.x[4 * (round & 1) + wid] = incl;
-    if (!cs.sync()) return false;
+    if (!cs.sync()) return fail;
     int higher = 0;
     for (int w = wid + 1; w < 4; ++w) higher += cs.x[4 * (round & 1) + w];
     const int gt1 = higher + incl - v, gt0 = gt1 + h1;
@@ -293,7 +276,7 @@ __device__ __noinline__ bool cand_compact(CandSet& cs, int& cnt_io, uint64_t& ta
       xb[1] = gt0;
       xb[2] = h0;
     }
-    if (!cs.sync()) return false;
+    if (!cs.sync()) return fail;
     const uint64_t pre = (prefix << bits) | static_cast<uint64_t>(xb[0] & 255);
     const int gt = xb[1], inb = xb[2];
     pbits += bits;
@@ -305,31 +288,50 @@ __device__ __noinline__ bool cand_compact(CandSet& cs, int& cnt_io, uint64_t& ta
     need -= gt;
     prefix = pre;
   }
+  // entry base + 128 j + t is thread t's j-th of the round; a survivor's place
+  // counts the survivors of the earlier (j, warp) groups, in that order
   int wpos = 0;
-  for (int base = 0, par = 0; base < cnt; base += 128, par ^= 1) {
-    const int i = base + t;
-    uint64_t c = 0;
-    bool keep = false;
-    if (i < cnt) {
-      c = cs.buf[i];
-      keep = c >= tnew;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = 0, par = 0; base < cnt; base += 1024, par ^= 1) {
+    uint64_t c[8];
+    unsigned m[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = base + 128 * j + t;
+      c[j] = i < cnt ? cs.buf[i] : 0ull;
+      m[j] = __ballot_sync(0xffffffffu, i < cnt && c[j] >= tnew);
     }
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) cs.x[16 + 4 * par + wid] = __popc(m);
-    if (!cs.sync()) return false;
-    int off = 0, tot = 0;
-    for (int w = 0; w < 4; ++w) {
-      const int n = cs.x[16 + 4 * par + w];
-      off += (w < wid) ? n : 0;
-      tot += n;
+    int* rc = cs.x + 16 + 32 * par;
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) rc[4 * j + wid] = __popc(m[j]);
     }
-    const int dst = wpos + off + __popc(m & ((1u << lane) - 1u));
-    if (keep && dst < FUSED_CB) cs.buf[dst] = c;
-    wpos += tot;
+    if (!cs.sync()) return fail;
+    int acc = 0;
+    int off[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int4 n = *reinterpret_cast<const int4*>(rc + 4 * j);
+      const int nw[4] = {n.x, n.y, n.z, n.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        if (w == wid) off[j] = acc;
+        acc += nw[w];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if ((m[j] >> lane) & 1u) {
+        const int d = wpos + off[j] + __popc(m[j] & lt);
+        if (d < FUSED_CB) cs.buf[d] = c[j];
+      }
+    }
+    wpos += acc;
   }
-  cnt_io = wpos < FUSED_CB ? wpos : FUSED_CB;
-  if (tnew > tau) tau = tnew;
-  return cs.sync();
+  CompactResult r{tnew > tau ? tnew : tau, wpos < FUSED_CB ? wpos : FUSED_CB, 0u, false};
+  r.ok = cs.sync();
+  r.phase = cs.phase;
+  return r;
 }
 
 template <bool FP8, int TPM, bool FUSED>
@@ -362,6 +364,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* start = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+  // fused: the streaming selector's threshold, (row + 1) << 32 | tau's score key
+  volatile uint64_t* tau_pub = reinterpret_cast<volatile uint64_t*>(smem + C::OFF_MISC + 16);
   float* w_smem = reinterpret_cast<float*>(smem + C::OFF_W);
   const uint32_t a_base = smem_u32(smem + C::OFF_A);
   const uint32_t q_base = smem_u32(smem + C::OFF_Q);
@@ -390,7 +394,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
         }
         mbar_init(selreq_bar, 1);
         mbar_init(selgrp_bar, C::NSEL);
-        for (int j = 0; j < 96; ++j) reinterpret_cast<int*>(smem + C::OFF_CX)[j] = 0;
+        for (int j = 0; j < FUSED_XINTS; ++j) reinterpret_cast<int*>(smem + C::OFF_CX)[j] = 0;
+        *tau_pub = 0ull;
       }
       *abort_flag = 0;
       fence_barrier_init();
@@ -557,7 +562,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
       for (int t = 0; t < C::TOK_PER_EW; ++t)
 #pragma unroll
         for (int h = 0; h < 64; ++h) wr[t][h] = 0.f;
-      float* stg = reinterpret_cast<float*>(smem + C::OFF_STG);  // fused: staged scores
+      uint64_t* stg = reinterpret_cast<uint64_t*>(smem + C::OFF_STG);  // fused: staged keys
+      int* scnt = reinterpret_cast<int*>(smem + C::OFF_SCNT);             // and counts
       for (long i = 0; i < nitems; ++i) {
         if (C::NSETS > 1 && acc % C::NSETS != set) {  // another set's slot
           if (++acc == C::NACC) {
@@ -632,14 +638,24 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(accempty_bar(acc));
         if constexpr (FUSED) {
-          // the tile's scores (the same fp32 values the unfused store writes) go to
-          // staging slot i % NSTG, which only this set uses, for the selectors
+          // the selection keys of the keys in range whose score (the same fp32
+          // value the unfused store writes) reaches the row's published threshold go,
+          // packed in index order, to staging slot i % NSTG, which only this set uses
+          const uint64_t ck = select_key(res[0] * ks, static_cast<uint32_t>(s));
+          const uint64_t pub = *tau_pub;
+          const uint32_t tf =
+              (static_cast<uint32_t>(pub >> 32) == static_cast<uint32_t>(it.qb) + 1u)
+                  ? static_cast<uint32_t>(pub)
+                  : 0u;
+          const bool cand = key_ok && s <= a.pos0 && static_cast<uint32_t>(ck >> 32) >= tf;
+          const unsigned cm = __ballot_sync(0xffffffffu, cand);
           const int sl = static_cast<int>(i % C::NSTG);
           const uint32_t use = static_cast<uint32_t>(i / C::NSTG);
           if (!__all_sync(0xffffffffu, mbar_wait(stgempty_bar(sl), (use & 1u) ^ 1u, abort_flag,
                                                  kErrTimeoutEpilogue)))
             break;
-          stg[sl * C::BM + qd * 32 + lane] = res[0] * ks;
+          if (cand) stg[sl * C::BM + qd * 32 + __popc(cm & ((1u << lane) - 1u))] = ck;
+          if (lane == 0) scnt[sl * 4 + qd] = __popc(cm);
           __syncwarp();
           if (lane == 0) mbar_arrive(stgfull_bar(sl));
         } else if (key_ok) {
@@ -661,95 +677,112 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
       }
     } else {
       // ------------------------------------------------------------ selectors (fused)
-      // The first selector warp streams: it takes every tile's 128 scores from the
-      // staging ring (4 keys per lane) and appends the candidates to the buffer,
-      // warp-synchronously.  The other three sleep until it asks them to compact the
-      // buffer with it (or to leave).
+      // The first selector warp streams: it takes every tile's candidate keys from
+      // the staging ring and appends them to the buffer in index order.  The other three wait until it asks them to compact
+      // the buffer with it (or to leave).
       if constexpr (FUSED) {
         const int wid = warp - C::SEL_W0, t = wid * 32 + lane;
         CandSet cs{reinterpret_cast<uint64_t*>(smem + C::OFF_CBUF),
                    reinterpret_cast<uint32_t*>(smem + C::OFF_CHIST),
                    reinterpret_cast<int*>(smem + C::OFF_CX), selgrp_bar, 0u, abort_flag};
-        int* req = cs.x + 64;  // op (1 compact, 2 leave), count, target; tau at req + 4
+        int* req = cs.x + 96;  // op (1 compact, 2 leave), count, target; tau, hi at req + 4, + 6
         if (wid == 0) {
-          const float* stg = reinterpret_cast<const float*>(smem + C::OFF_STG);
+          const uint64_t* stg = reinterpret_cast<const uint64_t*>(smem + C::OFF_STG);
+          const int* scnt = reinterpret_cast<const int*>(smem + C::OFF_SCNT);
+          uint64_t* const cbuf = reinterpret_cast<uint64_t*>(smem + C::OFF_CBUF);
           WorkIt<TPM> it{start[0], start[1], qb_tiles<TPM>(a, start[0])};
           int ccnt = 0, crow = -1;
-          uint64_t ctau = 0;
-          long crow_first = 0;  // first CTA of the current row
-          bool ok = true;
-          auto compact = [&](int target) {  // with the helpers
-            if (!ok) return;
-            if (lane == 0) {
-              req[0] = 1;
-              req[1] = ccnt;
-              req[2] = target;
-              *reinterpret_cast<uint64_t*>(req + 4) = ctau;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(selreq_bar);
-            ok = cand_compact(cs, ccnt, ctau, a.topk, target, t);
-          };
-          // the buffer to the row's slot (header: count, tau, largest key), emptied;
-          // more than 2k keys are first compacted to at most k + 256
-          auto flush = [&](int row) {
-            if (ccnt > 2 * a.topk) compact(a.topk + 256);
-            if (!ok) return;
-            const long piece = static_cast<long>(blockIdx.x) - crow_first;
-            uint8_t* slot = a.cslots + (static_cast<long>(row) * a.maxp + piece) *
-                                           static_cast<long>(FUSED_SLOT_BYTES);
-            uint64_t* dst = reinterpret_cast<uint64_t*>(slot + 64);
-            uint64_t mx = 0;
-            for (int j = lane; j < ccnt; j += 32) {
-              const uint64_t c = cs.buf[j];
-              dst[j] = c;
-              mx = c > mx ? c : mx;
-            }
+          uint64_t ctau = 0, kmx = 0;  // kmx: this lane's largest appended key
+          long crow_first = 0;         // first CTA of the current row
+          int sl = 0;                  // staging slot of tile i, and its use parity
+          uint32_t sph = 0;
+          // (the loop state stays in registers: no helper takes its address)
+          for (long i = 0;; ++i) {
+            // before tile i: the buffer goes to the row's slot when the row (or the
+            // work) ends, first compacted to at most k + 256 keys if it holds more
+            // than 2k; otherwise it is compacted to 3/8 of its size when the next
+            // tile might not fit
+            const bool row_end = crow >= 0 && (i == nitems || it.qb != crow);
+            int target = 0;
+            if (row_end && ccnt > 2 * a.topk) target = a.topk + 256;
+            if (!row_end && ccnt > FUSED_CB - C::BM) target = 3 * FUSED_CB / 8;
+            if (target > 0) {  // with the helpers
+              uint64_t hi = kmx;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              const uint64_t y = __shfl_xor_sync(0xffffffffu, mx, o);
-              mx = y > mx ? y : mx;
+              for (int o = 16; o > 0; o >>= 1) {
+                const uint64_t y = __shfl_xor_sync(0xffffffffu, hi, o);
+                hi = y > hi ? y : hi;
+              }
+              if (lane == 0) {
+                req[0] = 1;
+                req[1] = ccnt;
+                req[2] = target;
+                *reinterpret_cast<uint64_t*>(req + 4) = ctau;
+                *reinterpret_cast<uint64_t*>(req + 6) = hi;
+              }
+              __syncwarp();
+              if (lane == 0) mbar_arrive(selreq_bar);
+              const CompactResult r = cand_compact(cs, ccnt, ctau, hi, a.topk, target, t);
+              if (!r.ok) break;
+              ccnt = r.cnt;
+              ctau = r.tau;
+              cs.phase = r.phase;
+              if (lane == 0)
+                *tau_pub = (static_cast<uint64_t>(static_cast<uint32_t>(crow) + 1u) << 32) |
+                           (ctau >> 32);
             }
-            if (lane == 0) {
-              *reinterpret_cast<int*>(slot) = ccnt;
-              *reinterpret_cast<uint64_t*>(slot + 8) = ctau;
-              *reinterpret_cast<uint64_t*>(slot + 16) = mx;
+            if (row_end) {  // header: count, tau, largest key
+              const long piece = static_cast<long>(blockIdx.x) - crow_first;
+              uint8_t* slot = a.cslots + (static_cast<long>(crow) * a.maxp + piece) *
+                                             static_cast<long>(FUSED_SLOT_BYTES);
+              uint64_t* dst = reinterpret_cast<uint64_t*>(slot + 64);
+              for (int j = lane; j < ccnt; j += 32) dst[j] = cbuf[j];
+              uint64_t mx = kmx;
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) {
+                const uint64_t y = __shfl_xor_sync(0xffffffffu, mx, o);
+                mx = y > mx ? y : mx;
+              }
+              if (lane == 0) {
+                *reinterpret_cast<int*>(slot) = ccnt;
+                *reinterpret_cast<uint64_t*>(slot + 8) = ctau;
+                *reinterpret_cast<uint64_t*>(slot + 16) = mx;
+              }
+              __syncwarp();
+              ccnt = 0;
+              ctau = 0;
+              kmx = 0;
             }
-            __syncwarp();
-            ccnt = 0;
-            ctau = 0;
-          };
-          for (long i = 0; i < nitems && ok; ++i) {
+            if (i == nitems) break;
             if (it.qb != crow) {
-              if (crow >= 0) flush(crow);
               crow = it.qb;
               crow_first = ((g0 + i - it.kt) * gridDim.x + gridDim.x - 1) / a.total_tiles;
             }
-            const int sl = static_cast<int>(i % C::NSTG);
-            const uint32_t use = static_cast<uint32_t>(i / C::NSTG);
-            if (!__all_sync(0xffffffffu, mbar_wait_poll(stgfull_bar(sl), use & 1u, abort_flag,
-                                                        kErrTimeoutEpilogue))) {
-              ok = false;
+            if (!__all_sync(0xffffffffu, mbar_wait_poll(stgfull_bar(sl), sph, abort_flag,
+                                                        kErrTimeoutEpilogue)))
               break;
-            }
-            const float4 v = *reinterpret_cast<const float4*>(stg + sl * C::BM + 4 * lane);
+            const int4 n4 = *reinterpret_cast<const int4*>(scnt + sl * 4);
+            const int nq[4] = {n4.x, n4.y, n4.z, n4.w};
+            uint64_t kv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) kv[q] = lane < nq[q] ? stg[sl * C::BM + q * 32 + lane] : 0ull;
             __syncwarp();
             if (lane == 0) mbar_arrive(stgempty_bar(sl));
-            // keys 4 lane .. 4 lane + 3 of the tile: one query per sequence, at pos0
-            const float sv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int s = it.kt * C::BM + 4 * lane + e;
-              const uint64_t ck = select_key(sv[e], static_cast<uint32_t>(s));
-              const bool cand = s < a.Lk && s <= a.pos0 && ck >= ctau;
-              const unsigned m = __ballot_sync(0xffffffffu, cand);
-              if (cand) cs.buf[ccnt + __popc(m & ((1u << lane) - 1u))] = ck;
-              ccnt += __popc(m);
+            if (++sl == C::NSTG) {
+              sl = 0;
+              sph ^= 1u;
             }
-            if (ccnt > FUSED_CB - C::BM) compact(3 * FUSED_CB / 8);
+            // warp q's keys follow warp q - 1's: the tile's candidates in index order
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (lane < nq[q]) {
+                cbuf[ccnt + lane] = kv[q];
+                kmx = kv[q] > kmx ? kv[q] : kmx;
+              }
+              ccnt += nq[q];
+            }
             it.advance(a);
           }
-          if (crow >= 0 && ok) flush(crow);
           // the helpers leave
           __syncwarp();
           if (lane == 0) {
@@ -761,23 +794,26 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
           for (;;) {
             // wait for a request: bounded by a long limit (the streamer always ends
             // with one), or the CTA's abort
-            bool got = mbar_try_wait(selreq_bar, rph);
+            bool got = mbar_test(selreq_bar, rph);
             const uint64_t t0 = globaltimer();
             while (!got) {
+              __nanosleep(64);
               if (*abort_flag) break;
               if (globaltimer() - t0 > 30ull * IC_WAIT_NS) {
                 *abort_flag = 1;
                 record_error(kErrTimeoutEpilogue);
                 break;
               }
-              got = mbar_try_wait(selreq_bar, rph);
+              got = mbar_test(selreq_bar, rph);
             }
             if (!__all_sync(0xffffffffu, got)) break;
             rph ^= 1u;
             if (req[0] != 1) break;
-            int cnt = req[1];
-            uint64_t tau = *reinterpret_cast<const uint64_t*>(req + 4);
-            if (!cand_compact(cs, cnt, tau, a.topk, req[2], t)) break;
+            const CompactResult r =
+                cand_compact(cs, req[1], *reinterpret_cast<const uint64_t*>(req + 4),
+                             *reinterpret_cast<const uint64_t*>(req + 6), a.topk, req[2], t);
+            if (!r.ok) break;
+            cs.phase = r.phase;
           }
         }
       }

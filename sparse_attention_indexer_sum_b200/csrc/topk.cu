@@ -594,21 +594,21 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
 
 // ------------------------------------------------------------------ fused top-k merge
 // The second half of the fused indexer -> top-k (indexer_tc.cu, one query per
-// sequence): every (row, CTA piece, epilogue set) left a slot holding every key
-// of its share of the row whose selection key (score key << 32 | ~index) is >=
-// the slot's tau, and, when tau != 0, at least k of them.  So the row's k largest
+// sequence): every (row, CTA piece) left a slot holding, in ascending index
+// order, every key of its share of the row whose selection key (score key << 32
+// | ~index) is >= the slot's tau, and, when tau != 0, at least k of them; the
+// pieces of a row follow one another in index order.  So the row's k largest
 // selection keys are all in the slots and all >= the largest tau.  One CTA per
 // row gathers the slot keys >= that tau into shared memory (narrowing the bound
 // by radix digits over the slots if too many pass), finds the exact k-th largest
-// selection key by 12-bit radix rounds, and writes the k selected indices in
-// ascending order (bitonic sort).  Selection keys are unique within a row, so
-// exactly k keys are >= the k-th: ties need no separate handling.
+// selection key by 12-bit radix rounds, and writes the indices of the slot keys
+// >= it in slot order, which is ascending.  Selection keys are unique within a
+// row, so exactly k keys are >= the k-th: ties need no separate handling.
 constexpr int TM_CAP = 8192;  // selection keys gathered into shared memory
 
 struct MergeSmem {
   uint64_t cand[TM_CAP];
   int hist[TK_NBINS];
-  int sel[TK_MAXK];
   int scnt[512];        // keys per slot (clamped)
   int soff[513];        // prefix of scnt
   int scan_tmp[TK_NW];
@@ -795,42 +795,61 @@ __global__ void __launch_bounds__(TK_THREADS) topk_merge_kernel(
     need -= gt;
   }
 
-  // the k keys >= T, their indices sorted ascending
-  int P = 1;
-  while (P < k) P <<= 1;
-  for (int j = tid; j < P; j += TK_THREADS) sm.sel[j] = 0x7fffffff;
-  if (tid == 0) sm.counter = 0;
-  __syncthreads();
-  for (int i0 = 0; i0 < C; i0 += TK_THREADS) {
-    const int i = i0 + tid;
-    const uint64_t c = i < C ? sm.cand[i] : 0ull;
-    const bool take = i < C && c >= T;
-    const unsigned m = __ballot_sync(0xffffffffu, take);
-    if (m) {
-      int p = 0;
-      if (lane == 0) p = atomicAdd(&sm.counter, __popc(m));
-      p = __shfl_sync(0xffffffffu, p, 0) + __popc(m & ((1u << lane) - 1u));
-      if (take && p < TK_MAXK) sm.sel[p] = static_cast<int>(~static_cast<uint32_t>(c));
-    }
-  }
-  __syncthreads();
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < P / 2; i += TK_THREADS) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const int x = sm.sel[lo], y = sm.sel[hi];
-        if ((x > y) == ((lo & size) == 0)) {
-          sm.sel[lo] = y;
-          sm.sel[hi] = x;
-        }
+  // the k keys >= T in slot order (ascending index): each round takes 8 x 512
+  // slot keys, key f0 + 512 u + thread; a key's place counts the selected keys of
+  // the earlier (u, warp) groups (scanned by warp 0) and of the lower lanes
+  const int tot = sm.soff[nslot];
+  const int warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  int wbase = 0;
+  for (int f0 = 0; f0 < tot; f0 += 8 * TK_THREADS) {
+    uint64_t c[8];
+    unsigned m[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int fi = f0 + u * TK_THREADS + tid;
+      c[u] = 0;
+      if (fi < tot) {
+        int j = 0;
+        while (sm.soff[j + 1] <= fi) ++j;
+        c[u] = __ldg(reinterpret_cast<const unsigned long long*>(base + j * slot_bytes + 64) +
+                     (fi - sm.soff[j]));
       }
-      __syncthreads();
+      m[u] = __ballot_sync(0xffffffffu, fi < tot && c[u] >= T);
     }
+    if (lane == 0) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sm.hist[u * TK_NW + warp] = __popc(m[u]);
+    }
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan of the 8 x TK_NW group counts, 4 per lane
+      static_assert(8 * TK_NW == 128, "four group counts per lane");
+      const int4 v = *reinterpret_cast<const int4*>(sm.hist + 4 * lane);
+      const int sum = v.x + v.y + v.z + v.w;
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int ex = incl - sum;
+      *reinterpret_cast<int4*>(sm.hist + 4 * lane) =
+          make_int4(ex, ex + v.x, ex + v.x + v.y, ex + v.x + v.y + v.z);
+      if (lane == 31) sm.counter = incl;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if ((m[u] >> lane) & 1u) {
+        const int p = wbase + sm.hist[u * TK_NW + warp] + __popc(m[u] & lt);
+        if (p < k) out[p] = static_cast<int>(~static_cast<uint32_t>(c[u]));
+      }
+    }
+    wbase += sm.counter;
+    __syncthreads();
   }
-  const int got = sm.counter < k ? sm.counter : k;
-  if (sm.counter != k && tid == 0) record_error(kErrTopkOverflow);  // cannot happen
-  for (int j = tid; j < k; j += TK_THREADS) out[j] = (j < got) ? sm.sel[j] : -1;
+  if (wbase != k && tid == 0) record_error(kErrTopkOverflow);  // cannot happen
+  for (int j = wbase + tid; j < k; j += TK_THREADS) out[j] = -1;
 }
 
 ic_status launch_topk_merge(const uint8_t* slots, long rows, long nt, long total, int G, int maxp,
