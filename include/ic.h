@@ -95,6 +95,7 @@ ic_status ic_device_status(void* stream);
 #define IC_K_INDEXER_TOPK_E4M3 12
 #define IC_K_ATTN_MLA_KV8 13
 #define IC_K_PACK_KV 14
+#define IC_K_FILL_VALID 15
 ic_status ic_trace_begin(void* stream, int capacity);
 long ic_trace_end(float* ms, int* kinds, double* work, int capacity);
 
@@ -357,9 +358,14 @@ ic_status ic_layer_stack_rows(const char* pattern, const ic_stack_desc* desc,
  * the whole routing loop on its own keys at positions 0..L_i - 1, as
  * ic_layer_stack would with desc->L = L_i.  cu_seqlens: host int64 [nseq + 1],
  * cu_seqlens[0] = 0, nondecreasing, every L_i <= desc->L (desc->L sizes the
- * workspace: ic_stack_workspace_size(desc) covers any batch).  The sequences run
- * one after another on `stream`.  Errors as ic_layer_stack, with the sequence
- * named.
+ * workspace: ic_stack_workspace_size(desc) covers any batch).
+ * bf16 / e4m3 stacks share their launches between sequences: an F layer walks the
+ * packed query rows in blocks of as many score rows as the workspace holds
+ * (desc->L floats plus one int32 each), each block touching at most 64 sequences,
+ * with one indexer, one valid-length and one top-k launch per block (each row
+ * scored against its own sequence's keys); every layer's attention runs once per
+ * group of up to 64 whole sequences.  The fp32 forms run the sequences one after
+ * another.  Errors as ic_layer_stack (the fp32 forms name the sequence).
  */
 ic_status ic_layer_stack_varlen(const char* pattern, const ic_stack_desc* desc,
                                 const ic_layer_io* layers, int nlayers, const long* cu_seqlens,

@@ -162,7 +162,7 @@ def ic_device_status(stream=None):
 KIND_NAMES = {1: "indexer_tc_bf16", 2: "indexer_tc_e4m3", 3: "indexer_f32", 4: "fill_masked",
               5: "topk", 6: "attn_mla", 7: "attn_combine", 8: "attn_f32", 9: "quant_e4m3",
               10: "topk_merge", 11: "indexer_topk_bf16", 12: "indexer_topk_e4m3",
-              13: "attn_mla_kv8", 14: "pack_kv_e4m3"}
+              13: "attn_mla_kv8", 14: "pack_kv_e4m3", 15: "fill_valid"}
 
 
 def ic_trace_begin(capacity: int = 4096, stream=None):

@@ -275,6 +275,116 @@ static ic_status run_stack(const char* pattern, const ic_stack_desc* d, const ic
   return IC_OK;
 }
 
+// Packed sequences (cu: host [nseq + 1]) of a bf16 / e4m3 stack in shared launches.
+// F layers walk the packed query rows in blocks that fit the score workspace and
+// touch at most IC_MAXSEG sequences: one indexer launch over the block's segments
+// (each row against its own sequence's keys), one valid-length fill and one top-k
+// launch; attention runs over groups of at most IC_MAXSEG whole sequences.  The
+// launch count depends on the rows and the number of groups, not on nseq.
+static ic_status run_stack_varlen_shared(const std::vector<char>& kinds, const ic_stack_desc* d,
+                                         const ic_layer_io* layers, int nlayers, const long* cu,
+                                         int nseq, int* t_cache, void* workspace, size_t ws_bytes,
+                                         cudaStream_t stream) {
+  const long total = cu[nseq];
+  if (total == 0) return IC_OK;
+  for (int l = 0; l < nlayers; ++l) {
+    const ic_layer_io& io = layers[l];
+    if (kinds[l] == 'F') {
+      ic_status st = check_indexer(io.q_idx, io.q_scale, io.k_idx, io.k_scale, io.w, d->idx_dtype,
+                                   1, d->H, d->D, static_cast<int>(total),
+                                   static_cast<int>(total), 0, nullptr, total, false);
+      if (st) return fail(st, "layer %d: %s", l, ic_last_error());
+    }
+    ic_status st = check_attn(io.q, io.kv, d->ld_kv, io.v, t_cache, d->attn_dtype, 1,
+                              static_cast<int>(total), d->heads, d->dk, d->dv, d->L, d->k, io.out);
+    if (st) return fail(st, "layer %d: %s", l, ic_last_error());
+  }
+  // score rows of L floats plus one valid length each
+  const long ld = d->L;
+  long rb = static_cast<long>(ws_bytes / (static_cast<size_t>(ld) * sizeof(float) + sizeof(int)));
+  if (rb > total) rb = total;
+  if (rb >= 4 && rb < total) rb &= ~3L;
+  if (!workspace || rb < 1)
+    return fail(IC_ERR_WORKSPACE, "varlen: workspace of %zu bytes holds no score row of %ld floats",
+                ws_bytes, ld);
+  float* scores = static_cast<float*>(workspace);
+  int* valid = reinterpret_cast<int*>(scores + rb * ld);
+  const bool kv8 = d->attn_dtype == IC_E4M3;
+  const size_t qe = 2;
+  const size_t arow_b = static_cast<size_t>(d->heads) * d->dk * qe;
+  const size_t orow_b = static_cast<size_t>(d->heads) * d->dv * qe;
+  std::vector<IdxSeg> segs;
+  std::vector<AttnSeg> asegs;
+  for (int l = 0; l < nlayers; ++l) {
+    const ic_layer_io& io = layers[l];
+    if (kinds[l] == 'F') {
+      int sf = 0;  // first sequence with rows at or after u0
+      for (long u0 = 0; u0 < total;) {
+        while (sf < nseq && cu[sf + 1] <= u0) ++sf;
+        long u1 = u0 + rb < total ? u0 + rb : total;
+        const int sl = sf + IC_MAXSEG < nseq ? sf + IC_MAXSEG : nseq;
+        if (cu[sl] < u1) u1 = cu[sl];  // at most IC_MAXSEG sequences in the block
+        segs.clear();
+        for (int sq = sf; sq < sl && cu[sq] < u1; ++sq) {
+          const long c0 = cu[sq], c1 = cu[sq + 1];
+          const long a0 = c0 > u0 ? c0 : u0, a1 = c1 < u1 ? c1 : u1;
+          if (a1 <= a0) continue;
+          IdxSeg g;
+          g.qrow0 = a0;
+          g.krow0 = c0;
+          g.orow0 = a0 - u0;
+          g.pos0 = a0 - c0;
+          g.R = static_cast<int>(a1 - a0);
+          g.Lk = static_cast<int>(c1 - c0);
+          g.qb0 = 0;
+          g.pad = 0;
+          segs.push_back(g);
+        }
+        const long nu = u1 - u0;
+        ic_status st = launch_indexer_tc_segs(d->idx_dtype == IC_E4M3, io.q_idx, io.q_scale,
+                                              io.k_idx, io.k_scale, io.w, segs.data(),
+                                              static_cast<int>(segs.size()), total, total, scores,
+                                              ld, stream);
+        if (st) return st;
+        st = launch_fill_valid_len(segs.data(), static_cast<int>(segs.size()), nu, valid, stream);
+        if (st) return st;
+        st = launch_topk(scores, nu, static_cast<int>(ld), ld, 0, d->k, t_cache + u0 * d->k, stream,
+                         valid);
+        if (st) return st;
+        u0 = u1;
+      }
+    }
+    // attention over groups of whole sequences
+    for (int g0 = 0; g0 < nseq; g0 += IC_MAXSEG) {
+      const int g1 = g0 + IC_MAXSEG < nseq ? g0 + IC_MAXSEG : nseq;
+      const long r0 = cu[g0], nr = cu[g1] - cu[g0];
+      if (nr == 0) continue;
+      asegs.clear();
+      long long valid_entries = 0;
+      for (int sq = g0; sq < g1; ++sq) {
+        const long n = cu[sq + 1] - cu[sq];
+        if (n == 0) continue;
+        AttnSeg a;
+        a.q0 = cu[sq] - r0;
+        a.k0 = cu[sq];
+        a.len = static_cast<int>(n);
+        a.pad = 0;
+        asegs.push_back(a);
+        valid_entries += causal_pairs(n, d->k, 0);
+      }
+      ic_status st = launch_attn_mla(static_cast<const uint8_t*>(io.q) + r0 * arow_b, io.kv,
+                                     d->ld_kv, t_cache + r0 * d->k, 1, static_cast<int>(nr), d->L,
+                                     d->k, d->scale,
+                                     static_cast<uint8_t*>(io.out) + r0 * orow_b,
+                                     io.lse ? io.lse + r0 * d->heads : nullptr, workspace, ws_bytes,
+                                     valid_entries, stream, kv8, asegs.data(),
+                                     static_cast<int>(asegs.size()));
+      if (st) return st;
+    }
+  }
+  return IC_OK;
+}
+
 }  // namespace ic
 
 using namespace ic;
@@ -464,6 +574,22 @@ ic_status ic_layer_stack_varlen(const char* pattern, const ic_stack_desc* desc,
                   cu_seqlens[i + 1] - cu_seqlens[i], desc->L);
   if (nlayers < 1 || nlayers > 4096 || !layers)
     return fail(IC_ERR_INVALID_ARG, "varlen: bad layers / nlayers");
+  if (desc->idx_dtype != IC_F32 && desc->attn_dtype != IC_F32 && !desc->decode) {
+    ic_status st = check_desc(desc, false);
+    if (st) return st;
+    std::vector<char> kinds;
+    st = parse_pattern(pattern, &kinds);
+    if (st) return st;
+    if (static_cast<int>(kinds.size()) != nlayers)
+      return fail(IC_ERR_INVALID_ARG, "pattern has %zu layers, nlayers is %d", kinds.size(),
+                  nlayers);
+    if (!t_cache) return fail(IC_ERR_INVALID_ARG, "varlen: NULL t_cache");
+    if (cu_seqlens[nseq] * 64 > 0x7fffffffL)
+      return fail(IC_ERR_UNSUPPORTED, "varlen: too many rows for 32-bit TMA coordinates");
+    return run_stack_varlen_shared(kinds, desc, layers, nlayers, cu_seqlens, nseq, t_cache,
+                                   workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+  }
+  // fp32 forms (small shapes): the sequences run one after another
   const size_t qrow_b = static_cast<size_t>(desc->H) * desc->D * elem_bytes(desc->idx_dtype);
   const size_t krow_b = static_cast<size_t>(desc->D) * elem_bytes(desc->idx_dtype);
   // q, v and out are fp32 (MQA) or bf16 (MLA, also over an e4m3 cache, whose ld_kv is

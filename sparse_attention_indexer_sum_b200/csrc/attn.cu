@@ -94,7 +94,30 @@ struct AttnArgs {
   int kv8;
   const uint8_t* kv8p;
   long ld_kv8;
+  // packed sequences (nseg > 0): query row r belongs to the last segment with
+  // seg.q0 <= r, whose latent rows start at row seg.k0 and number seg.len
+  int nseg;
+  AttnSeg seg[IC_MAXSEG];
 };
+
+// Latent rows of query row qrow: the first row's offset (in rows) and how many.
+__device__ __forceinline__ void attn_kv_range(const AttnArgs& a, long qrow, long& row0, int& len) {
+  if (a.nseg == 0) {
+    row0 = (qrow / a.R) * static_cast<long>(a.Lkv);
+    len = a.Lkv;
+    return;
+  }
+  int lo = 0, hi = a.nseg - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.seg[mid].q0 <= qrow)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  row0 = a.seg[lo].k0;
+  len = a.seg[lo].len;
+}
 
 // Dequantises the fp8 rows of one tile stage that belong to producer warp pw (rows
 // 8pw..8pw+7 with their bit set in `valid`) in place: a raw row (656 bytes at slot
@@ -278,9 +301,11 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
   for (long it = 0; it < nj; ++it, ib ^= 1) {
     const AttnItem x = attn_item(a, it);
     const int cnt = x.end - x.beg;
-    const long b = x.qrow / a.R;
-    const __nv_bfloat16* kvb = a.kv + b * static_cast<long>(a.Lkv) * a.ld_kv;
-    const uint8_t* kvb8 = a.kv8p + b * static_cast<long>(a.Lkv) * a.ld_kv8;
+    long kr0;
+    int lkv;
+    attn_kv_range(a, x.qrow, kr0, lkv);
+    const __nv_bfloat16* kvb = a.kv + kr0 * a.ld_kv;
+    const uint8_t* kvb8 = a.kv8p + kr0 * a.ld_kv8;
     // every producer is done with the previous item (and its index list)
     if (lane == 0) mbar_arrive(smem_u32(&sm.pitem));
     if (!mbar_wait(smem_u32(&sm.pitem), static_cast<uint32_t>(nitem & 1), abort, kErrTimeoutProducer))
@@ -302,7 +327,7 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
     int lv = -1;
     for (int j = lane; j < cnt; j += 32) {
       const int s = ilist[j];
-      if (s >= 0 && s < a.Lkv) lv = j;
+      if (s >= 0 && s < lkv) lv = j;
     }
     lv = __reduce_max_sync(0xffffffffu, lv);
     const int ntiles = (lv >= 0) ? lv / AT_BK + 1 : 0;
@@ -327,7 +352,7 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
       }
       const int j = t * AT_BK + lane;
       int s = (t < ntiles && j < cnt) ? ilist[j] : -1;
-      if (s >= a.Lkv) s = -1;
+      if (s >= lkv) s = -1;
       const unsigned valid = __ballot_sync(0xffffffffu, s >= 0);
       if (pw == 0 && lane == 0) {
         sm.vmask[stage] = valid;
@@ -596,7 +621,7 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
   }
 }
 
-__global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t at_smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(
       (reinterpret_cast<uintptr_t>(at_smem_raw) + 127) & ~static_cast<uintptr_t>(127));
@@ -735,8 +760,10 @@ size_t attn_mla_ws_bytes(int batch, int rows, int k) {
 ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* idx, int batch,
                           int rows, int Lkv, int k, float scale, void* out, float* lse, void* ws,
                           size_t ws_bytes, long long valid_entries, cudaStream_t stream,
-                          bool kv8) {
+                          bool kv8, const AttnSeg* segs, int nseg) {
   const long items = static_cast<long>(batch) * rows;
+  if (nseg < 0 || nseg > IC_MAXSEG || (nseg > 0 && (batch != 1 || !segs)))
+    return fail(IC_ERR_INVALID_ARG, "attn: bad segment list (%d)", nseg);
   if (items == 0) return IC_OK;
   SplitPlan p = split_plan(items, k);
   const size_t need = static_cast<size_t>(items) * p.maxp * AT_H * (AT_DV + 2) * sizeof(float);
@@ -766,6 +793,8 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
   a.idx_bulk = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
   a.part_o = p.split ? static_cast<float*>(ws) : nullptr;
   a.part_ml = p.split ? static_cast<float*>(ws) + items * p.maxp * AT_H * AT_DV : nullptr;
+  a.nseg = nseg;
+  for (int j = 0; j < nseg; ++j) a.seg[j] = segs[j];
   const int smem = static_cast<int>(sizeof(AttnSmem)) + 128;
   ic_status st = cuda_check(
       cudaFuncSetAttribute(attn_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),

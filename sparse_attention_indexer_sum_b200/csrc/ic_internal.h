@@ -58,6 +58,7 @@ enum LaunchKind : int {
   kKindIndexerTopkE4m3 = 12,
   kKindAttnMlaKv8 = 13,
   kKindPackKv = 14,
+  kKindFillValid = 15,
 };
 // Called after every kernel launch: when tracing is on for this host thread,
 // records an event on `stream` with the launch's kind and algorithmic work
@@ -67,6 +68,28 @@ void trace_launch(int kind, cudaStream_t stream, double work);
 long long causal_pairs(long R, long Lk, long pos0);
 
 // Indexer on tensor cores (H = 64, D = 128).  fp8 = e4m3 inputs with scales.
+// Packed sequences of different lengths: at most IC_MAXSEG per launch.  An
+// indexer segment is described beside IdxTcArgs (indexer_tc.cu); an attention
+// segment's query rows q0.. (up to the next segment's q0) attend over latent rows
+// k0 .. k0 + len - 1, which their index lists address as 0 .. len - 1.
+constexpr int IC_MAXSEG = 64;
+struct IdxSeg {
+  long qrow0, krow0, orow0, pos0;
+  int R, Lk, qb0, pad;
+};
+struct AttnSeg {
+  long q0, k0;
+  int len, pad;
+};
+// The multi-token tensor-core indexer over nseg packed segments in one launch
+// (q_rows, k_rows: rows of the packed query and key tensors).
+ic_status launch_indexer_tc_segs(bool fp8, const void* q, const float* q_scale, const void* k,
+                                 const float* k_scale, const float* w, const IdxSeg* segs,
+                                 int nseg, long q_rows, long k_rows, float* scores, long ld,
+                                 cudaStream_t stream);
+// valid_len[r] of the rows of a block of packed segments (their positions + 1).
+ic_status launch_fill_valid_len(const IdxSeg* segs, int nseg, long rows, int* out,
+                                cudaStream_t stream);
 ic_status launch_indexer_tc(bool fp8, const void* q, const float* q_scale, const void* k,
                             const float* k_scale, const float* w, int batch, int rows, int Lk,
                             long pos0, float* scores, long ld, bool fill_tail,
@@ -94,10 +117,12 @@ ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0,
 // it (the causal stack does), else -1 (rows * k is assumed for tracing only).
 // kv8: kv holds fp8 latent rows (KV8_ROW_BYTES, ld_kv in bytes), else bf16 rows
 // (ld_kv in elements).
+// segs (nseg <= IC_MAXSEG, host array): packed sequences, with batch = 1 and rows =
+// all their query rows; Lkv is then ignored.
 ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* idx, int batch,
                           int rows, int Lkv, int k, float scale, void* out, float* lse,
                           void* ws, size_t ws_bytes, long long valid_entries, cudaStream_t stream,
-                          bool kv8 = false);
+                          bool kv8 = false, const AttnSeg* segs = nullptr, int nseg = 0);
 size_t attn_mla_ws_bytes(int batch, int rows, int k);
 ic_status launch_attn_f32(const float* q, const float* kv, long ld_kv, const float* v,
                           const int* idx, int batch, int rows, int heads, int dk, int dv,

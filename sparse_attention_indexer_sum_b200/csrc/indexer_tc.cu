@@ -49,11 +49,18 @@ struct IdxTcArgs {
   int qb_per_batch;      // ceil(R / TPM)
   int nqb;               // B * qb_per_batch
   long total_tiles;
-  // Fused top-k (one query per sequence): every (row, CTA piece, epilogue set)
-  // leaves its candidates in a slot of `cslots`; topk_merge_kernel selects.
+  // Fused top-k (one query per sequence): every (row, CTA piece) leaves its
+  // candidates in a slot of `cslots`; topk_merge_kernel selects.
   uint8_t* cslots;
-  int maxp;              // CTA pieces per row (slots per row = maxp * NSETS)
+  int maxp;              // CTA pieces per row
   int topk;              // k of the selection
+  // Segments (packed sequences of different lengths; 0 = the uniform batch above).
+  // Segment j holds seg[j].R query rows at positions seg[j].pos0.. over seg[j].Lk
+  // keys: its query rows are rows qrow0.. of q / w / q_scale, its keys rows krow0..
+  // of k / k_scale, its score rows rows orow0.. of scores; its query blocks are
+  // qb0 .. qb0 + ceil(R / TPM) - 1.  Used by the multi-token instances only.
+  int nseg;
+  IdxSeg seg[IC_MAXSEG];
 };
 
 // Fused top-k slot: a 64-byte header {int count; int pad; uint64 tau; uint64 max}
@@ -139,23 +146,63 @@ struct IdxCfg {
   static_assert(NACC % NSETS == 0, "each epilogue set owns whole accumulator slots");
 };
 
-template <int TPM>
+// Where query block qb lies: its first query row's index in its segment (ql *
+// TPM), the segment's rows, positions and keys, and the row offsets of its query,
+// key and score rows.
+struct QbInfo {
+  long qrow0, krow0, orow0, pos0;
+  int R, Lk, ql;
+};
+template <int TPM, bool SEGS>
+__host__ __device__ __forceinline__ QbInfo qb_info(const IdxTcArgs& a, int qb) {
+  QbInfo x;
+  if (SEGS) {
+    int lo = 0, hi = a.nseg - 1;  // the last segment with qb0 <= qb
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.seg[mid].qb0 <= qb)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    const IdxSeg& g = a.seg[lo];
+    x.ql = qb - g.qb0;
+    x.qrow0 = g.qrow0;
+    x.krow0 = g.krow0;
+    x.orow0 = g.orow0;
+    x.pos0 = g.pos0;
+    x.R = g.R;
+    x.Lk = g.Lk;
+  } else {
+    const int b = qb / a.qb_per_batch;
+    x.ql = qb - b * a.qb_per_batch;
+    x.qrow0 = static_cast<long>(b) * a.R;
+    x.orow0 = x.qrow0;
+    x.krow0 = static_cast<long>(b) * a.Lk;
+    x.pos0 = a.pos0;
+    x.R = a.R;
+    x.Lk = a.Lk;
+  }
+  return x;
+}
+
+template <int TPM, bool SEGS>
 __host__ __device__ __forceinline__ int qb_tiles(const IdxTcArgs& a, int qb) {
-  int ql = qb % a.qb_per_batch;
-  int r_last = min(ql * TPM + TPM, a.R) - 1;
-  long keys = a.pos0 + r_last + 1;
-  if (keys > a.Lk) keys = a.Lk;
+  const QbInfo x = qb_info<TPM, SEGS>(a, qb);
+  const int r_last = min(x.ql * TPM + TPM, x.R) - 1;
+  long keys = x.pos0 + r_last + 1;
+  if (keys > x.Lk) keys = x.Lk;
   return static_cast<int>((keys + 127) / 128);
 }
 
-template <int TPM>
+template <int TPM, bool SEGS>
 struct WorkIt {
   int qb, kt, nt;
   __device__ __forceinline__ void advance(const IdxTcArgs& a) {
     if (++kt >= nt) {
       kt = 0;
       ++qb;
-      nt = (qb < a.nqb) ? qb_tiles<TPM>(a, qb) : 0;
+      nt = (qb < a.nqb) ? qb_tiles<TPM, SEGS>(a, qb) : 0;
     }
   }
 };
@@ -334,10 +381,10 @@ __device__ __noinline__ CompactResult cand_compact(CandSet cs, const int cnt, ui
   return r;
 }
 
-template <bool FP8, int TPM, bool FUSED>
+template <bool FP8, int TPM, bool FUSED, bool SEGS>
 __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmQ, const IdxTcArgs a) {
+                      const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ IdxTcArgs a) {
   using C = IdxCfg<FP8, TPM, FUSED>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -407,7 +454,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
     long cum = 0;
     for (int base = 0; base < a.nqb; base += 32) {
       const int qb = base + lane;
-      const long t = (qb < a.nqb) ? qb_tiles<TPM>(a, qb) : 0;
+      const long t = (qb < a.nqb) ? qb_tiles<TPM, SEGS>(a, qb) : 0;
       long incl = t;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -442,7 +489,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
-        WorkIt<TPM> it{start[0], start[1], qb_tiles<TPM>(a, start[0])};
+        WorkIt<TPM, SEGS> it{start[0], start[1], qb_tiles<TPM, SEGS>(a, start[0])};
         int stage = 0;
         uint32_t ph = 0;
         int qloads = 0, cur_qb = -1;
@@ -452,8 +499,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
             if (qloads > 0 &&
                 !mbar_wait(qempty_bar, (qloads - 1) & 1, abort_flag, kErrTimeoutProducer))
               break;
-            const int b = it.qb / a.qb_per_batch, ql = it.qb % a.qb_per_batch;
-            const int qrow = (b * a.R + ql * TPM) * 64;
+            const QbInfo x = qb_info<TPM, SEGS>(a, it.qb);
+            const int qrow = static_cast<int>((x.qrow0 + x.ql * TPM) * 64);
             mbar_arrive_expect_tx(qfull_bar, C::Q_BYTES);
 #pragma unroll
             for (int kb = 0; kb < C::KBLK; ++kb)
@@ -462,8 +509,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
             cur_qb = it.qb;
           }
           if (!mbar_wait(empty_bar(stage), ph ^ 1, abort_flag, kErrTimeoutProducer)) break;
-          const int b = it.qb / a.qb_per_batch;
-          const int krow = b * a.Lk + it.kt * C::BM;
+          const int krow = static_cast<int>(qb_info<TPM, SEGS>(a, it.qb).krow0 + it.kt * C::BM);
           mbar_arrive_expect_tx(full_bar(stage), C::A_BYTES);
 #pragma unroll
           for (int kb = 0; kb < C::KBLK; ++kb)
@@ -500,7 +546,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
         for (int kk = 0; kk < C::KSTEPS; ++kk)
           bdesc[kk] = sdesc_k_sw128(q_base + (kk / 4) * (C::N * 128) + (kk % 4) * 32);
         const uint64_t adesc0 = sdesc_k_sw128(a_base);
-        WorkIt<TPM> it{start[0], start[1], qb_tiles<TPM>(a, start[0])};
+        WorkIt<TPM, SEGS> it{start[0], start[1], qb_tiles<TPM, SEGS>(a, start[0])};
         int stage = 0, acc = 0;
         uint32_t ph = 0, aph = 0;
         int qwaits = 0, cur_qb = -1;
@@ -527,7 +573,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
             tc_commit(empty_bar(stage));
             tc_commit(accfull_bar(acc));
           }
-          WorkIt<TPM> nx = it;
+          WorkIt<TPM, SEGS> nx = it;
           nx.advance(a);
           if (i + 1 == nitems || nx.qb != it.qb) tc_commit(qempty_bar);
           it = nx;
@@ -551,7 +597,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
       const int set = e / C::SETW;  // accumulator slots a with a % NSETS == set
       const int member = (e % C::SETW) / 4;  // which tokens of the block this warp reduces
       float* wsl = w_smem + e * C::TOK_PER_EW * 64;
-      WorkIt<TPM> it{start[0], start[1], qb_tiles<TPM>(a, start[0])};
+      WorkIt<TPM, SEGS> it{start[0], start[1], qb_tiles<TPM, SEGS>(a, start[0])};
       int acc = 0;
       uint32_t aph = 0;
       int cur_qb = -1;
@@ -573,15 +619,15 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
           it.advance(a);
           continue;
         }
-        const int b = it.qb / a.qb_per_batch, ql = it.qb % a.qb_per_batch;
-        const int r0 = ql * TPM + member * C::TOK_PER_EW;
+        const QbInfo qi = qb_info<TPM, SEGS>(a, it.qb);
+        const int r0 = qi.ql * TPM + member * C::TOK_PER_EW;
         if (it.qb != cur_qb) {
           __syncwarp();
           for (int x = lane; x < C::TOK_PER_EW * 64; x += 32) {
             const int r = r0 + x / 64;
             float v = 0.f;
-            if (r < a.R) {
-              const long o = (static_cast<long>(b) * a.R + r) * 64 + (x % 64);
+            if (r < qi.R) {
+              const long o = (qi.qrow0 + r) * 64 + (x % 64);
               v = a.w[o];
               if constexpr (FP8) v *= a.q_scale[o];
             }
@@ -599,9 +645,9 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
         // this lane's key; its fp8 scale is fetched before the wait so the load's
         // latency hides behind it
         const int s = it.kt * C::BM + qd * 32 + lane;
-        const bool key_ok = s < a.Lk && b < a.B;
+        const bool key_ok = s < qi.Lk;
         float ks = 1.f;
-        if constexpr (FP8) ks = key_ok ? a.k_scale[static_cast<long>(b) * a.Lk + s] : 0.f;
+        if constexpr (FP8) ks = key_ok ? a.k_scale[qi.krow0 + s] : 0.f;
         // every lane leaves together, so the warp never splits before tcgen05.ld
         const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(accfull_bar(acc), aph, abort_flag,
                                                               kErrTimeoutEpilogue));
@@ -647,7 +693,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
               (static_cast<uint32_t>(pub >> 32) == static_cast<uint32_t>(it.qb) + 1u)
                   ? static_cast<uint32_t>(pub)
                   : 0u;
-          const bool cand = key_ok && s <= a.pos0 && static_cast<uint32_t>(ck >> 32) >= tf;
+          const bool cand = key_ok && s <= qi.pos0 && static_cast<uint32_t>(ck >> 32) >= tf;
           const unsigned cm = __ballot_sync(0xffffffffu, cand);
           const int sl = static_cast<int>(i % C::NSTG);
           const uint32_t use = static_cast<uint32_t>(i / C::NSTG);
@@ -662,9 +708,9 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
 #pragma unroll
           for (int tk = 0; tk < C::TOK_PER_EW; ++tk) {
             const int r = r0 + tk;
-            if (r < a.R) {
-              const long pos = a.pos0 + r;
-              a.scores[(static_cast<long>(b) * a.R + r) * a.ld + s] =
+            if (r < qi.R) {
+              const long pos = qi.pos0 + r;
+              a.scores[(qi.orow0 + r) * a.ld + s] =
                   (s <= pos) ? res[tk] * ks : -INFINITY;
             }
           }
@@ -690,7 +736,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
           const uint64_t* stg = reinterpret_cast<const uint64_t*>(smem + C::OFF_STG);
           const int* scnt = reinterpret_cast<const int*>(smem + C::OFF_SCNT);
           uint64_t* const cbuf = reinterpret_cast<uint64_t*>(smem + C::OFF_CBUF);
-          WorkIt<TPM> it{start[0], start[1], qb_tiles<TPM>(a, start[0])};
+          WorkIt<TPM, SEGS> it{start[0], start[1], qb_tiles<TPM, SEGS>(a, start[0])};
           int ccnt = 0, crow = -1;
           uint64_t ctau = 0, kmx = 0;  // kmx: this lane's largest appended key
           long crow_first = 0;         // first CTA of the current row
@@ -899,8 +945,9 @@ static ic_status launch_tpl(const void* q, const float* q_scale, const void* k,
   a.cslots = cslots;
   a.maxp = maxp;
   a.topk = topk;
+  a.nseg = 0;
   long total = 0;
-  for (int qb = 0; qb < a.qb_per_batch; ++qb) total += qb_tiles<TPM>(a, qb);
+  for (int qb = 0; qb < a.qb_per_batch; ++qb) total += qb_tiles<TPM, false>(a, qb);
   total *= batch;  // every batch has the same triangle
   a.total_tiles = total;
   if (total == 0) return IC_OK;
@@ -911,12 +958,12 @@ static ic_status launch_tpl(const void* q, const float* q_scale, const void* k,
   st = make_map(&tmQ, q, FP8, static_cast<uint64_t>(batch) * rows * 64, C::N);
   if (st) return st;
 
-  st = cuda_check(cudaFuncSetAttribute(indexer_tc_kernel<FP8, TPM, FUSED>,
+  st = cuda_check(cudaFuncSetAttribute(indexer_tc_kernel<FP8, TPM, FUSED, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
                   "cudaFuncSetAttribute(indexer)");
   if (st) return st;
   const long grid = total < num_sms() ? total : num_sms();
-  st = cuda_check(launch_dep(indexer_tc_kernel<FP8, TPM, FUSED>, dim3(static_cast<unsigned>(grid)),
+  st = cuda_check(launch_dep(indexer_tc_kernel<FP8, TPM, FUSED, false>, dim3(static_cast<unsigned>(grid)),
                              dim3(C::THREADS), C::SMEM_BYTES, stream, 1, tmK, tmQ, a),
                   "indexer_tc_kernel launch");
   if (st) return st;
@@ -925,6 +972,73 @@ static ic_status launch_tpl(const void* q, const float* q_scale, const void* k,
   trace_launch(kind, stream,
                2.0 * 64 * 128 * static_cast<double>(causal_pairs(rows, Lk, pos0)) * batch);
   return IC_OK;
+}
+
+// The multi-token instance over packed segments (see IdxTcArgs): one launch for
+// every segment; q_rows and k_rows are the rows of the packed query and key tensors.
+template <bool FP8>
+static ic_status launch_segs(const void* q, const float* q_scale, const void* k,
+                             const float* k_scale, const float* w, const IdxSeg* segs, int nseg,
+                             long q_rows, long k_rows, float* scores, long ld,
+                             cudaStream_t stream) {
+  constexpr int TPM = 4;
+  using C = IdxCfg<FP8, TPM, false>;
+  IdxTcArgs a;
+  a.w = w;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.scores = scores;
+  a.ld = ld;
+  a.B = 1;
+  a.R = 0;
+  a.Lk = 0;
+  a.pos0 = 0;
+  a.qb_per_batch = 1;
+  a.cslots = nullptr;
+  a.maxp = 0;
+  a.topk = 0;
+  a.nseg = nseg;
+  int nqb = 0;
+  double flop = 0.0;
+  for (int j = 0; j < nseg; ++j) {
+    a.seg[j] = segs[j];
+    a.seg[j].qb0 = nqb;
+    nqb += (segs[j].R + TPM - 1) / TPM;
+    flop += 2.0 * 64 * 128 * static_cast<double>(causal_pairs(segs[j].R, segs[j].Lk, segs[j].pos0));
+  }
+  a.nqb = nqb;
+  long total = 0;
+  for (int qb = 0; qb < nqb; ++qb) total += qb_tiles<TPM, true>(a, qb);
+  a.total_tiles = total;
+  if (total == 0) return IC_OK;
+
+  CUtensorMap tmK, tmQ;
+  ic_status st = make_map(&tmK, k, FP8, static_cast<uint64_t>(k_rows), C::BM);
+  if (st) return st;
+  st = make_map(&tmQ, q, FP8, static_cast<uint64_t>(q_rows) * 64, C::N);
+  if (st) return st;
+  st = cuda_check(cudaFuncSetAttribute(indexer_tc_kernel<FP8, TPM, false, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
+                  "cudaFuncSetAttribute(indexer)");
+  if (st) return st;
+  const long grid = total < num_sms() ? total : num_sms();
+  st = cuda_check(launch_dep(indexer_tc_kernel<FP8, TPM, false, true>, dim3(static_cast<unsigned>(grid)),
+                             dim3(C::THREADS), C::SMEM_BYTES, stream, 1, tmK, tmQ, a),
+                  "indexer_tc_kernel launch");
+  if (st) return st;
+  trace_launch(FP8 ? kKindIndexerE4m3 : kKindIndexerBf16, stream, flop);
+  return IC_OK;
+}
+
+ic_status launch_indexer_tc_segs(bool fp8, const void* q, const float* q_scale, const void* k,
+                                 const float* k_scale, const float* w, const IdxSeg* segs,
+                                 int nseg, long q_rows, long k_rows, float* scores, long ld,
+                                 cudaStream_t stream) {
+  if (nseg < 1 || nseg > IC_MAXSEG) return fail(IC_ERR_INVALID_ARG, "indexer: %d segments", nseg);
+  return fp8 ? launch_segs<true>(q, q_scale, k, k_scale, w, segs, nseg, q_rows, k_rows, scores, ld,
+                                 stream)
+             : launch_segs<false>(q, q_scale, k, k_scale, w, segs, nseg, q_rows, k_rows, scores,
+                                  ld, stream);
 }
 
 // Plan of the fused indexer -> top-k for `batch` sequences of one query each at

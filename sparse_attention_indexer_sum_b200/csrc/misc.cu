@@ -157,4 +157,45 @@ ic_status launch_indexer_f32(const float* q, const float* k, const float* w, int
   return st;
 }
 
+// ------------------------------------------------------------------ packed rows
+// valid_len[r] = position + 1 of score row r of a block of packed sequences: the
+// block's rows of segment j are rows orow0.. at positions pos0.. (IdxSeg).
+struct ValidSegs {
+  int nseg;
+  long orow0[IC_MAXSEG];
+  long pos0[IC_MAXSEG];
+};
+__global__ void fill_valid_len_kernel(const __grid_constant__ ValidSegs v, long rows, int* out) {
+  grid_dep_wait();
+  const long r = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  int lo = 0, hi = v.nseg - 1;  // the last segment starting at or before row r
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (v.orow0[mid] <= r)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  out[r] = static_cast<int>(v.pos0[lo] + (r - v.orow0[lo]) + 1);
+}
+
+ic_status launch_fill_valid_len(const IdxSeg* segs, int nseg, long rows, int* out,
+                                cudaStream_t stream) {
+  if (rows <= 0) return IC_OK;
+  if (nseg < 1 || nseg > IC_MAXSEG) return fail(IC_ERR_INVALID_ARG, "valid_len: %d segments", nseg);
+  ValidSegs v;
+  v.nseg = nseg;
+  for (int j = 0; j < nseg; ++j) {
+    v.orow0[j] = segs[j].orow0;
+    v.pos0[j] = segs[j].pos0;
+  }
+  ic_status st = cuda_check(launch_dep(fill_valid_len_kernel,
+                                       dim3(static_cast<unsigned>((rows + 255) / 256)), dim3(256), 0,
+                                       stream, 1, v, rows, out),
+                            "fill_valid_len_kernel launch");
+  if (!st) trace_launch(kKindFillValid, stream, 4.0 * static_cast<double>(rows));
+  return st;
+}
+
 }  // namespace ic

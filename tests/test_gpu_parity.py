@@ -14,8 +14,9 @@ import torch
 import oracle
 from sparse_attention_indexer_sum_b200 import binding as ic
 from sparse_attention_indexer_sum_b200 import synth
-from tests.paritylib import (assert_attn_close, assert_fp8_scores_close_to_unquantised,
-                             assert_scores_close, check_index_row)
+from tests.paritylib import (IDX_ATOL, IDX_RTOL_BF16, assert_attn_close,
+                             assert_fp8_scores_close_to_unquantised, assert_scores_close,
+                             check_index_row)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -532,6 +533,124 @@ def test_stack_varlen_batch_matches_the_oracle_per_sequence():
                                        rtol=1e-4)
             np.testing.assert_allclose(packed[l]["lse"][o0:o1].cpu().numpy(), rl, atol=1e-5,
                                        rtol=1e-5)
+
+
+def _varlen_mla_case(lens, pattern, fp8, seed):
+    """Per-sequence bf16 MLA stack inputs (shapes of prefill_8k) for `lens`, packed
+    along the rows; fp8: e4m3 indexer inputs and an fp8 latent cache."""
+    wl0 = synth.variant("prefill_8k", L=max(max(lens), 1), pattern=pattern)
+    per = []
+    for i, n in enumerate(lens):
+        wl = synth.variant("prefill_8k", L=max(n, 1), pattern=pattern)
+        lay = []
+        for l in range(wl.layers):
+            d = synth.indexer_inputs(wl, l, seed=seed + i)
+            d.update(synth.attn_inputs(wl, l, seed=seed + i))
+            lay.append({k: v[:n] for k, v in d.items()})
+        per.append(lay)
+    packed = []
+    for l in range(wl0.layers):
+        e = {k: torch.cat([p[l][k] for p in per]).to(DEV) for k in per[0][l]}
+        if fp8:
+            e["q_idx"], e["q_scale"] = ic.ic_quant_e4m3_rows(e["q_idx"])
+            e["k_idx"], e["k_scale"] = ic.ic_quant_e4m3_rows(e["k_idx"])
+            e["kv"] = ic.ic_pack_kv_e4m3(e["kv"])
+        tot = sum(lens)
+        e["out"] = torch.empty(tot, wl0.Hq, wl0.Dv, dtype=torch.bfloat16, device=DEV)
+        e["lse"] = torch.empty(tot, wl0.Hq, device=DEV)
+        packed.append(e)
+    dt = ic.IC_E4M3 if fp8 else ic.IC_BF16
+    desc = ic.make_desc(L=wl0.L, k=wl0.k, H=wl0.H, D=wl0.D, idx_dtype=dt, heads=wl0.Hq, dk=wl0.Dk,
+                        dv=wl0.Dv, attn_dtype=dt, scale=wl0.scale,
+                        ld_kv=ic.KV8_ROW_BYTES if fp8 else None)
+    return wl0, per, packed, desc
+
+
+def _check_varlen_sequence(wl0, packed, T, o0, n, rows, fp8, pattern):
+    """Sampled rows of one packed sequence: its F layers' index sets against the
+    oracle's scores over the sequence's own keys, every layer's attention against the
+    oracle on those rows (on the dequantised cache rows for fp8)."""
+    kinds = pattern.split(",")
+    seq = slice(o0, o0 + n)
+    Ti = T[o0:o0 + n]
+    for l, kind in enumerate(kinds):
+        e = packed[l]
+        if kind == "F":
+            if fp8:
+                ref = oracle.indexer_scores_e4m3(e["q_idx"][seq].cpu().numpy(),
+                                                 e["q_scale"][seq].cpu().numpy(),
+                                                 e["k_idx"][seq].cpu().numpy(),
+                                                 e["k_scale"][seq].cpu().numpy(),
+                                                 e["w"][seq].cpu().numpy(), rows_sel=rows)
+                atol, rtol = 1e-3, 1e-3   # same e4m3 codes: only summation order differs
+            else:
+                ref = oracle.indexer_scores(e["q_idx"][seq].float().cpu().numpy(),
+                                            e["k_idx"][seq].float().cpu().numpy(),
+                                            e["w"][seq].cpu().numpy(), rows_sel=rows)
+                atol, rtol = IDX_ATOL, IDX_RTOL_BF16
+            for j, r in enumerate(rows):
+                check_index_row(Ti[r], ref[j], wl0.k, r + 1, atol=atol, rtol=rtol)
+        q = e["q"][seq][torch.from_numpy(rows).to(DEV)].float().cpu().numpy()
+        if fp8:
+            codes, scales, rope = _unpack_kv8(e["kv"][seq].cpu().numpy())
+            ro, rl = oracle.sparse_attn_kv_e4m3(q, codes, scales, rope, Ti[rows], wl0.scale)
+        else:
+            ro, rl = oracle.sparse_attn(q, e["kv"][seq].float().cpu().numpy(), Ti[rows], wl0.scale,
+                                        dv=512)
+        got = e["out"][seq][torch.from_numpy(rows).to(DEV)]
+        assert_attn_close(_np(got), ro, what="layer %d" % l)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_stack_varlen_shared_launches(fp8):
+    """bf16 / e4m3 stack over packed sequences of 300, 0, 1, 2, 517, 64, 2100, 5 and 1300
+    tokens, pattern F,S: one indexer, one valid-length fill, one top-k and one
+    attention launch per layer cover every sequence (the trace counts them), and each
+    sequence's index sets and outputs match the oracle on that sequence alone."""
+    lens = [300, 0, 1, 2, 517, 64, 2100, 5, 1300]
+    pattern = "F,S"
+    wl0, per, packed, desc = _varlen_mla_case(lens, pattern, fp8, seed=11)
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    # room for every packed row's scores (and valid length): one block
+    ws = torch.empty(sum(lens) * (wl0.L + 1) + 64, device=DEV)
+    t = torch.full((sum(lens), wl0.k), -7, dtype=torch.int32, device=DEV)
+    ic.ic_trace_begin(256)
+    ic.ic_layer_stack_varlen(pattern, desc, packed, cu, t, ws)
+    n_launch, tr = ic.ic_trace_end(256)
+    _sync()
+    names = [x[0] for x in tr]
+    assert names.count("topk") == 1 and names.count("fill_valid") == 1, names
+    assert n_launch <= 6, names  # F: indexer, fill, top-k, attention; S: attention (+merges)
+    T = t.cpu().numpy()
+    for i, n in enumerate(lens):
+        if n == 0:
+            continue
+        rows = np.unique(np.clip(np.array([0, 1, n // 2, n - 2, n - 1, 2047, 2048, 2049]), 0, n - 1))
+        _check_varlen_sequence(wl0, packed, T, cu[i], n, rows, fp8, pattern)
+
+
+def test_stack_varlen_many_sequences_and_small_blocks():
+    """70 packed sequences of 0..180 tokens (more than one launch group) with a
+    workspace of 700 score rows, so that row blocks cut through sequences: every
+    sequence's index sets (all earlier tokens, k = 2048) and both layers' outputs
+    match the oracle on that sequence alone."""
+    g = np.random.default_rng(5)
+    lens = g.integers(0, 181, size=70).tolist()
+    lens[3] = 0
+    lens[10] = 1
+    pattern = "F,S"
+    wl0, per, packed, desc = _varlen_mla_case(lens, pattern, False, seed=40)
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    ws = torch.empty((700 * wl0.L * 4 + 700 * 4) // 4 + 64, device=DEV)
+    t = torch.full((sum(lens), wl0.k), -7, dtype=torch.int32, device=DEV)
+    ic.ic_layer_stack_varlen(pattern, desc, packed, cu, t, ws)
+    _sync()
+    T = t.cpu().numpy()
+    for i, n in enumerate(lens):
+        if n == 0:
+            continue
+        rows = np.unique(np.array([0, n // 3, n - 1]))
+        _check_varlen_sequence(wl0, packed, T, cu[i], n, rows, False, pattern)
 
 
 def test_decode_step_parity():
