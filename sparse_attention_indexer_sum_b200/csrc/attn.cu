@@ -98,6 +98,11 @@ struct AttnArgs {
   // seg.q0 <= r, whose latent rows start at row seg.k0 and number seg.len
   int nseg;
   AttnSeg seg[IC_MAXSEG];
+  // early: q, kv and idx are not written by the previous kernel of the stream (an
+  // S layer of the stack: its index set is the F layer's, two or more launches
+  // back), so the producers gather without waiting for that kernel and the
+  // consumers wait for it only before their first global write
+  int early;
 };
 
 // Latent rows of query row qrow: the first row's offset (in rows) and how many.
@@ -579,6 +584,7 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
     }
 
     // ---- item epilogue: head h's final max and sum live in warp h/2
+    if (a.early && it == 0) grid_dep_wait();  // the previous kernel's reads are done
     named_bar_sync(1, AT_CONSUMERS);  // every warp's P V of the item is done
     if ((lane & 15) == 0) {
       sm.fin_m[sh] = m_run;
@@ -646,7 +652,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const __grid_co
     z[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   __syncthreads();
-  grid_dep_wait();  // set-up above touches no global memory
+  grid_dep_signal();
+  if (!a.early) grid_dep_wait();  // set-up above touches no global memory
   if (threadIdx.x >= AT_CONSUMERS)
     attn_producer(sm, a);
   else
@@ -660,6 +667,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const __grid_co
 // them with shuffles; every thread accumulates its output dims over the pieces.
 __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, int maxp, long tot,
                                     int tq, int G, __nv_bfloat16* out, float* lse) {
+  grid_dep_signal();
   grid_dep_wait();
   const long qrow = blockIdx.x;
   const int h = blockIdx.y;
@@ -760,7 +768,7 @@ size_t attn_mla_ws_bytes(int batch, int rows, int k) {
 ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* idx, int batch,
                           int rows, int Lkv, int k, float scale, void* out, float* lse, void* ws,
                           size_t ws_bytes, long long valid_entries, cudaStream_t stream,
-                          bool kv8, const AttnSeg* segs, int nseg) {
+                          bool kv8, const AttnSeg* segs, int nseg, bool early) {
   const long items = static_cast<long>(batch) * rows;
   if (nseg < 0 || nseg > IC_MAXSEG || (nseg > 0 && (batch != 1 || !segs)))
     return fail(IC_ERR_INVALID_ARG, "attn: bad segment list (%d)", nseg);
@@ -795,6 +803,7 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
   a.part_ml = p.split ? static_cast<float*>(ws) + items * p.maxp * AT_H * AT_DV : nullptr;
   a.nseg = nseg;
   for (int j = 0; j < nseg; ++j) a.seg[j] = segs[j];
+  a.early = early ? 1 : 0;
   const int smem = static_cast<int>(sizeof(AttnSmem)) + 128;
   ic_status st = cuda_check(
       cudaFuncSetAttribute(attn_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),

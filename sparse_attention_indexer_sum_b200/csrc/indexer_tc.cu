@@ -601,11 +601,13 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
       int acc = 0;
       uint32_t aph = 0;
       int cur_qb = -1;
-      // head weights of this warp's tokens, kept in registers while the query
-      // block lasts (the values are then read from TMEM 16 columns at a time)
-      float wr[C::TOK_PER_EW][64];
+      // head weights of this warp's tokens: the warp's shared copy (wsl), written
+      // when a query block starts; the multi-token instance keeps them in registers
+      // (wr), the one-token instances read them with one broadcast load per 4 heads
+      constexpr bool WREG = TPM > 1;
+      float wr[WREG ? C::TOK_PER_EW : 1][64];
 #pragma unroll
-      for (int t = 0; t < C::TOK_PER_EW; ++t)
+      for (int t = 0; t < (WREG ? C::TOK_PER_EW : 1); ++t)
 #pragma unroll
         for (int h = 0; h < 64; ++h) wr[t][h] = 0.f;
       uint64_t* stg = reinterpret_cast<uint64_t*>(smem + C::OFF_STG);  // fused: staged keys
@@ -634,7 +636,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
             wsl[x] = v;
           }
           __syncwarp();
-          if constexpr (!FUSED) {
+          if constexpr (WREG) {
 #pragma unroll
             for (int t = 0; t < C::TOK_PER_EW; ++t)
 #pragma unroll
@@ -654,31 +656,72 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
         if (!acc_ok) break;
         float res[C::TOK_PER_EW];
         tc_fence_after();
-#pragma unroll
-        for (int tk = 0; tk < C::TOK_PER_EW; ++tk) {
-          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
-                                 static_cast<uint32_t>(acc * C::N + (member * C::TOK_PER_EW + tk) * 64);
+        // sum_h w_h relu(x_h) of each token, heads h = j mod 4 into s_j in head order
+        auto head_sum = [&](const float* v, int tk) {
           float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-          for (int part = 0; part < 64 / C::EPI_COLS; ++part) {  // heads in chunks of EPI_COLS
-            float v[C::EPI_COLS];
-            tmem_ld16(taddr + C::EPI_COLS * part, v);
+          for (int h = 0; h < 64; h += 4) {
+            const float4 wv = *reinterpret_cast<const float4*>(wsl + tk * 64 + h);
+            s0 = fmaf(wv.x, fmaxf(v[h + 0], 0.f), s0);
+            s1 = fmaf(wv.y, fmaxf(v[h + 1], 0.f), s1);
+            s2 = fmaf(wv.z, fmaxf(v[h + 2], 0.f), s2);
+            s3 = fmaf(wv.w, fmaxf(v[h + 3], 0.f), s3);
+          }
+          return (s0 + s1) + (s2 + s3);
+        };
+        auto tok_addr = [&](int tk) {
+          return tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
+                 static_cast<uint32_t>(acc * C::N + (member * C::TOK_PER_EW + tk) * 64);
+        };
+        if constexpr (WREG) {
+          // 16 columns per TMEM round trip, weights in registers
+#pragma unroll
+          for (int tk = 0; tk < C::TOK_PER_EW; ++tk) {
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {
+              float v[16];
+              tmem_ld16(tok_addr(tk) + 16 * part, v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int h4 = 0; h4 < 4; ++h4) {
+                const int h = 16 * part + 4 * h4;
+                s0 = fmaf(wr[tk][h], fmaxf(v[4 * h4 + 0], 0.f), s0);
+                s1 = fmaf(wr[tk][h + 1], fmaxf(v[4 * h4 + 1], 0.f), s1);
+                s2 = fmaf(wr[tk][h + 2], fmaxf(v[4 * h4 + 2], 0.f), s2);
+                s3 = fmaf(wr[tk][h + 3], fmaxf(v[4 * h4 + 3], 0.f), s3);
+              }
+            }
+            res[tk] = (s0 + s1) + (s2 + s3);
+          }
+        } else if constexpr (!FUSED) {
+          // one token: its 64 columns are loaded before one wait, a single TMEM
+          // round trip per tile
+          float v[64];
+#pragma unroll
+          for (int part = 0; part < 4; ++part)
+            tmem_ld16(tok_addr(0) + 16 * part, *reinterpret_cast<float(*)[16]>(&v[16 * part]));
+          tmem_ld_wait();
+          res[0] = head_sum(v, 0);
+        } else {
+          // 16 columns at a time, leaving the registers to the selection
+          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+          for (int part = 0; part < 4; ++part) {
+            float v[16];
+            tmem_ld16(tok_addr(0) + 16 * part, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int h4 = 0; h4 < C::EPI_COLS / 4; ++h4) {
-              const int h = C::EPI_COLS * part + 4 * h4;
-              // the fused instance reads the weights from the warp's shared copy (one
-              // broadcast load per 4 heads), leaving the registers to the selection
-              const float4 wv =
-                  FUSED ? *reinterpret_cast<const float4*>(wsl + tk * 64 + h)
-                        : make_float4(wr[tk][h], wr[tk][h + 1], wr[tk][h + 2], wr[tk][h + 3]);
+            for (int h4 = 0; h4 < 4; ++h4) {
+              const int h = 16 * part + 4 * h4;
+              const float4 wv = *reinterpret_cast<const float4*>(wsl + h);
               s0 = fmaf(wv.x, fmaxf(v[4 * h4 + 0], 0.f), s0);
               s1 = fmaf(wv.y, fmaxf(v[4 * h4 + 1], 0.f), s1);
               s2 = fmaf(wv.z, fmaxf(v[4 * h4 + 2], 0.f), s2);
               s3 = fmaf(wv.w, fmaxf(v[4 * h4 + 3], 0.f), s3);
             }
           }
-          res[tk] = (s0 + s1) + (s2 + s3);
+          res[0] = (s0 + s1) + (s2 + s3);
         }
         tc_fence_before();
         __syncwarp();
