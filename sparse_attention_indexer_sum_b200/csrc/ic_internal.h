@@ -107,7 +107,7 @@ ic_status launch_indexer_topk_fused(bool fp8, const void* q, const float* q_scal
                                     cudaStream_t stream);
 size_t indexer_topk_fused_ws_bytes(int batch, int Lk, long pos0);
 ic_status launch_topk_merge(const uint8_t* slots, long rows, long nt, long total, int G, int maxp,
-                            int nsets, size_t slot_bytes, int cb, int nv, int k, int* idx,
+                            size_t slot_bytes, int cb, int nv, int k, int* idx,
                             cudaStream_t stream);
 // valid_len (device int32 [rows], or NULL): row r's candidate count, clamped to
 // [0, n]; NULL means min(n, pos0 + r + 1), or n when pos0 < 0.

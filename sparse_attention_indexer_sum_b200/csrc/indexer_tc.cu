@@ -89,7 +89,10 @@ struct IdxCfg {
   static constexpr int STAGES = FP8 ? (FUSED ? 6 : 8) : 4;
   static constexpr int NACC = (TPM == 4) ? 2 : 6;  // TMEM accumulators in the ring
   static constexpr int TMEM_COLS = (NACC * N <= 256) ? 256 : 512;
-  static constexpr int EPG = (TPM == 4) ? 2 : 1;   // epilogue warps per TMEM lane quadrant
+  // epilogue warps per TMEM lane quadrant: with fp8 keys the tiles come twice as
+  // fast and four warps per quadrant (one token each) hide more of the TMEM round
+  // trips than two (measured 5% faster on long e4m3 rows, 6% slower with bf16)
+  static constexpr int EPG = (TPM == 4) ? (FP8 ? 4 : 2) : 1;
   // Epilogue warp sets: set j takes the accumulator slots a with a % NSETS == j, so
   // each set sees every use of its slots in order.  One-token blocks (decode) have
   // little epilogue work per tile; several sets overlap consecutive tiles.
@@ -111,8 +114,8 @@ struct IdxCfg {
   static_assert(NACC % MMAW == 0, "every use of an accumulator falls to one MMA warp");
   static constexpr int EPI_W0 = 1 + MMAW;  // first epilogue warp
   // fused top-k: selector warps after the epilogue warps consume the tiles'
-  // scores from a staging ring of NSTG tiles (a multiple of NSETS, so that every
-  // use of a staging slot falls to the same epilogue set)
+  // candidate keys from a staging ring of NSTG tiles (a multiple of NSETS, so that
+  // every use of a staging slot falls to the same epilogue set)
   static constexpr int NSEL = FUSED ? FUSED_SELW : 0;
   static constexpr int SEL_W0 = EPI_W0 + NEPI;
   static constexpr int NSTG = FUSED ? (FP8 ? 24 : 12) : 0;
@@ -602,9 +605,9 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
       uint32_t aph = 0;
       int cur_qb = -1;
       // head weights of this warp's tokens: the warp's shared copy (wsl), written
-      // when a query block starts; the multi-token instance keeps them in registers
-      // (wr), the one-token instances read them with one broadcast load per 4 heads
-      constexpr bool WREG = TPM > 1;
+      // when a query block starts; a warp with several tokens keeps them in registers
+      // (wr), a one-token warp reads them with one broadcast load per 4 heads
+      constexpr bool WREG = C::TOK_PER_EW > 1;
       float wr[WREG ? C::TOK_PER_EW : 1][64];
 #pragma unroll
       for (int t = 0; t < (WREG ? C::TOK_PER_EW : 1); ++t)
@@ -694,7 +697,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
             }
             res[tk] = (s0 + s1) + (s2 + s3);
           }
-        } else if constexpr (!FUSED) {
+        } else if constexpr (!FUSED && TPM == 1) {
           // one token: its 64 columns are loaded before one wait, a single TMEM
           // round trip per tile
           float v[64];
@@ -703,6 +706,26 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
             tmem_ld16(tok_addr(0) + 16 * part, *reinterpret_cast<float(*)[16]>(&v[16 * part]));
           tmem_ld_wait();
           res[0] = head_sum(v, 0);
+        } else if constexpr (!FUSED) {
+          // one token of a multi-token block (fewer registers per warp): 32 columns
+          // per round trip
+          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld16(tok_addr(0) + 32 * half, *reinterpret_cast<float(*)[16]>(&v[0]));
+            tmem_ld16(tok_addr(0) + 32 * half + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+            tmem_ld_wait();
+#pragma unroll
+            for (int h = 0; h < 32; h += 4) {
+              const float4 wv = *reinterpret_cast<const float4*>(wsl + 32 * half + h);
+              s0 = fmaf(wv.x, fmaxf(v[h + 0], 0.f), s0);
+              s1 = fmaf(wv.y, fmaxf(v[h + 1], 0.f), s1);
+              s2 = fmaf(wv.z, fmaxf(v[h + 2], 0.f), s2);
+              s3 = fmaf(wv.w, fmaxf(v[h + 3], 0.f), s3);
+            }
+          }
+          res[0] = (s0 + s1) + (s2 + s3);
         } else {
           // 16 columns at a time, leaving the registers to the selection
           float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
@@ -1132,7 +1155,7 @@ ic_status launch_indexer_topk_fused(bool fp8, const void* q, const float* q_scal
                                                     pos0, nullptr, Lk, stream, slots, p.maxp, topk);
     if (st) return st;
   }
-  return launch_topk_merge(slots, batch, p.nt, p.total, p.G, p.maxp, 1, FUSED_SLOT_BYTES,
+  return launch_topk_merge(slots, batch, p.nt, p.total, p.G, p.maxp, FUSED_SLOT_BYTES,
                            FUSED_CB, static_cast<int>(nv), topk, idx, stream);
 }
 

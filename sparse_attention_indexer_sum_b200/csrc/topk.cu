@@ -667,7 +667,7 @@ __device__ __forceinline__ void for_slot_keys(const MergeSmem& sm, const uint8_t
 }
 
 __global__ void __launch_bounds__(TK_THREADS) topk_merge_kernel(
-    const uint8_t* __restrict__ slots, long nt, long total, int G, int maxp, int nsets,
+    const uint8_t* __restrict__ slots, long nt, long total, int G, int maxp,
     long slot_bytes, int cb, int nv, int k, int* __restrict__ idx) {
   extern __shared__ __align__(16) uint8_t tm_smem_raw[];
   MergeSmem& sm = *reinterpret_cast<MergeSmem*>(tm_smem_raw);
@@ -681,9 +681,9 @@ __global__ void __launch_bounds__(TK_THREADS) topk_merge_kernel(
   }
   const long first = (row * nt * G + G - 1) / total;
   const long last = ((row * nt + nt - 1) * G + G - 1) / total;
-  int nslot = static_cast<int>(last - first + 1) * nsets;
+  int nslot = static_cast<int>(last - first + 1);
   if (nslot > 512) nslot = 512;  // cannot happen for a plan of <= 170 pieces per row
-  const uint8_t* base = slots + row * static_cast<long>(maxp) * nsets * slot_bytes;
+  const uint8_t* base = slots + row * static_cast<long>(maxp) * slot_bytes;
   if (tid == 0) {
     sm.tau = 0ull;
     sm.kmax = 0ull;
@@ -853,7 +853,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_merge_kernel(
 }
 
 ic_status launch_topk_merge(const uint8_t* slots, long rows, long nt, long total, int G, int maxp,
-                            int nsets, size_t slot_bytes, int cb, int nv, int k, int* idx,
+                            size_t slot_bytes, int cb, int nv, int k, int* idx,
                             cudaStream_t stream) {
   if (rows == 0) return IC_OK;
   const int smem = static_cast<int>(sizeof(MergeSmem));
@@ -862,7 +862,7 @@ ic_status launch_topk_merge(const uint8_t* slots, long rows, long nt, long total
       "cudaFuncSetAttribute(topk_merge)");
   if (st) return st;
   st = cuda_check(launch_dep(topk_merge_kernel, dim3(static_cast<unsigned>(rows)),
-                             dim3(TK_THREADS), smem, stream, 1, slots, nt, total, G, maxp, nsets,
+                             dim3(TK_THREADS), smem, stream, 1, slots, nt, total, G, maxp,
                              static_cast<long>(slot_bytes), cb, nv, k, idx),
                   "topk_merge_kernel launch");
   if (st) return st;
