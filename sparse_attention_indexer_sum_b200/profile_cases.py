@@ -5,6 +5,7 @@
     python -m sparse_attention_indexer_sum_b200.profile_cases attn_tail4k
     python -m sparse_attention_indexer_sum_b200.profile_cases decode_indexer
     python -m sparse_attention_indexer_sum_b200.profile_cases decode_attn
+    python -m sparse_attention_indexer_sum_b200.profile_cases decode_step
 
 Each case builds its inputs once, on the GPU, with seeded generators. It runs the
 kernels through the C ABI, 2 warm-up rounds then 3 traced rounds, and prints
@@ -25,6 +26,11 @@ name captures a warm launch. Every case fits in a few GB of device memory.
                     over 2048 random distinct rows of its own 20000-row latent KV
                     (1.5 GB in all, far beyond L2); split over the SMs, partials
                     merged by the combine kernel.
+  decode_step       the whole F,S,S,S decode step of 64 sequences x 1 query over
+                    200000 tokens (ic_decode_step: e4m3 indexer, top-k, four
+                    attention layers with their merges).  The four layers share
+                    one 14.7 GB latent cache and one key cache (each layer has its
+                    own queries), ~17 GB in all; for a launch list only.
 """
 from __future__ import annotations
 
@@ -152,9 +158,34 @@ def decode_attn():
     _rounds(lambda: ic.ic_sparse_attn(q, kv, idx, wl.scale, out=out, workspace=ws))
 
 
+def decode_step():
+    dev = "cuda"
+    wl = synth.WORKLOADS["decode_200k"]
+    B, L, k = wl.batch, wl.L, wl.k
+    d = synth.indexer_inputs(wl, 0, device=dev)
+    q8, qs = ic.ic_quant_e4m3_rows(d["q_idx"])
+    k8, ks = ic.ic_quant_e4m3_rows(d.pop("k_idx"))
+    kv = synth.attn_inputs(wl, 0, device=dev)["kv"]
+    torch.cuda.empty_cache()
+    g = torch.Generator(device=dev).manual_seed(1)
+    layers = []
+    for _ in range(wl.layers):
+        q = torch.randn(B, 1, wl.Hq, wl.Dk, device=dev, generator=g).to(torch.bfloat16)
+        layers.append({"q_idx": q8, "q_scale": qs, "k_idx": k8, "k_scale": ks, "w": d["w"],
+                       "q": q, "kv": kv,
+                       "out": torch.empty(B, 1, wl.Hq, wl.Dv, dtype=torch.bfloat16, device=dev),
+                       "lse": torch.empty(B, 1, wl.Hq, device=dev)})
+    desc = ic.make_desc(L=L, k=k, H=wl.H, D=wl.D, idx_dtype=ic.IC_E4M3, heads=wl.Hq, dk=wl.Dk,
+                        dv=wl.Dv, attn_dtype=ic.IC_BF16, scale=wl.scale, batch=B, decode=True)
+    ws = torch.empty(ic.ic_stack_workspace_size(desc) // 4 + 1, device=dev)
+    t_cache = torch.empty(B, k, dtype=torch.int32, device=dev)
+    _rounds(lambda: ic.ic_decode_step(wl.pattern, desc, layers, t_cache, ws))
+
+
 CASES = {"indexer_longrows": indexer_longrows, "indexer_longrows_e4m3": indexer_longrows_e4m3,
          "attn_tail4k": attn_tail4k,
-         "decode_indexer": decode_indexer, "decode_attn": decode_attn}
+         "decode_indexer": decode_indexer, "decode_attn": decode_attn,
+         "decode_step": decode_step}
 
 
 def main(argv=None) -> int:
