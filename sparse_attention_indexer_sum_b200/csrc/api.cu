@@ -146,11 +146,10 @@ static ic_status check_attn(const void* q, const void* kv, long ld_kv, const voi
 static ic_status run_attn(const void* q, const void* kv, long ld_kv, const void* v,
                           const int* idx, ic_dtype dt, int batch, int rows, int heads, int dk,
                           int dv, int Lkv, int k, float scale, void* out, float* lse, void* ws,
-                          size_t ws_bytes, long long valid_entries, cudaStream_t stream,
-                          bool early = false) {
+                          size_t ws_bytes, long long valid_entries, cudaStream_t stream) {
   if (!v)
     return launch_attn_mla(q, kv, ld_kv, idx, batch, rows, Lkv, k, scale, out, lse, ws, ws_bytes,
-                           valid_entries, stream, dt == IC_E4M3, nullptr, 0, early);
+                           valid_entries, stream, dt == IC_E4M3);
   return launch_attn_f32(static_cast<const float*>(q), static_cast<const float*>(kv), ld_kv,
                          static_cast<const float*>(v), idx, batch, rows, heads, dk, dv, Lkv, k,
                          scale, static_cast<float*>(out), lse, stream);
@@ -269,11 +268,8 @@ static ic_status run_stack(const char* pattern, const ic_stack_desc* d, const ic
     // out_l <- SparseAttn_l(T_cache); the score workspace is free again here
     const long long valid = decode ? static_cast<long long>(B) * (d->k < d->L ? d->k : d->L)
                                    : causal_pairs(R, d->k, row0);
-    // an S layer's inputs come from launches before the previous one: its gathers
-    // start before that kernel ends
     st = run_attn(io.q, io.kv, d->ld_kv, io.v, t_cache, d->attn_dtype, B, R, d->heads, d->dk,
-                  d->dv, d->L, d->k, d->scale, io.out, io.lse, workspace, ws_bytes, valid, stream,
-                  kinds[l] == 'S');
+                  d->dv, d->L, d->k, d->scale, io.out, io.lse, workspace, ws_bytes, valid, stream);
     if (st) return st;
   }
   return IC_OK;

@@ -28,6 +28,8 @@
 //     (query, range) piece leaves an unnormalised partial in the workspace, and
 //     attn_combine_kernel merges them.
 // Shared rows are padded to 1168 B so that ldmatrix is bank-conflict free.
+#include <type_traits>
+
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
@@ -88,40 +90,45 @@ struct AttnArgs {
   float* lse;               // [B, R, 16] or null (not split)
   float* part_o;            // [items * maxp, 16, 512] (split)
   float* part_ml;           // [items * maxp, 16, 2]   (split)
-  // fp8 latent cache (kv8): rows of 656 bytes (512 e4m3 codes, 4 fp32 group scales,
-  // 64 bf16 rope dims) at kv8p + row * ld_kv8 bytes; dequantised in shared memory
-  // to the bf16 row layout the consumers read
-  int kv8;
-  const uint8_t* kv8p;
-  long ld_kv8;
-  // packed sequences (nseg > 0): query row r belongs to the last segment with
-  // seg.q0 <= r, whose latent rows start at row seg.k0 and number seg.len
-  int nseg;
-  AttnSeg seg[IC_MAXSEG];
-  // early: q, kv and idx are not written by the previous kernel of the stream (an
-  // S layer of the stack: its index set is the F layer's, two or more launches
-  // back), so the producers gather without waiting for that kernel and the
-  // consumers wait for it only before their first global write
-  int early;
+  // (the fp8 latent cache instance reads kv as rows of ld_kv bytes, each holding a
+  // 656-byte row: 512 e4m3 codes, 4 fp32 group scales, 64 bf16 rope dims; it
+  // dequantises them in shared memory to the bf16 row layout the consumers read)
 };
 
+// Packed sequences: query row r of the launch belongs to the last segment with
+// seg.q0 <= r, whose latent rows start at row seg.k0 and number seg.len.  A kernel
+// parameter of its own, so that AttnArgs stays small (the kernel reads it as
+// instruction operands; a larger or addressable AttnArgs measured ~1 % slower
+// each on the prefill attention).
+struct AttnSegs {
+  int nseg;
+  AttnSeg seg[IC_MAXSEG];
+};
+struct AttnNoSegs {
+  int unused;
+};
+template <bool SEGS>
+using AttnSegParam = typename std::conditional<SEGS, AttnSegs, AttnNoSegs>::type;
+
 // Latent rows of query row qrow: the first row's offset (in rows) and how many.
-__device__ __forceinline__ void attn_kv_range(const AttnArgs& a, long qrow, long& row0, int& len) {
-  if (a.nseg == 0) {
+template <bool SEGS>
+__device__ __forceinline__ void attn_kv_range(const AttnArgs& a, const AttnSegParam<SEGS>& sg,
+                                              long qrow, long& row0, int& len) {
+  if constexpr (!SEGS) {
     row0 = (qrow / a.R) * static_cast<long>(a.Lkv);
     len = a.Lkv;
-    return;
+  } else {
+    int lo = 0, hi = sg.nseg - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sg.seg[mid].q0 <= qrow)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    row0 = sg.seg[lo].k0;
+    len = sg.seg[lo].len;
   }
-  int lo = 0, hi = a.nseg - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.seg[mid].q0 <= qrow)
-      lo = mid;
-    else
-      hi = mid - 1;
-  }
-  row0 = a.seg[lo].k0;
-  len = a.seg[lo].len;
 }
 
 // Dequantises the fp8 rows of one tile stage that belong to producer warp pw (rows
@@ -267,7 +274,11 @@ __device__ __forceinline__ void attn_load_indices(AttnSmem& sm, const AttnArgs& 
 // every tile -- one warp's bulk copies issue one lane at a time, so spreading a
 // tile over four warps quadruples the gather issue rate.  Producer 0 also owns
 // the per-item work: the next index list, the queries, the stage flags.
-__device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
+// KV8: fp8 latent rows; SEGS: packed sequences (separate instances, so that the
+// bf16 form of one batch compiles without either)
+template <bool KV8, bool SEGS>
+__device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a,
+                                              const AttnSegParam<SEGS>& sg) {
   const int lane = threadIdx.x & 31;
   const int pw = (threadIdx.x - AT_CONSUMERS) >> 5;
   volatile int* abort = &sm.abort;
@@ -308,9 +319,9 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
     const int cnt = x.end - x.beg;
     long kr0;
     int lkv;
-    attn_kv_range(a, x.qrow, kr0, lkv);
+    attn_kv_range<SEGS>(a, sg, x.qrow, kr0, lkv);
     const __nv_bfloat16* kvb = a.kv + kr0 * a.ld_kv;
-    const uint8_t* kvb8 = a.kv8p + kr0 * a.ld_kv8;
+    const uint8_t* kvb8 = reinterpret_cast<const uint8_t*>(a.kv) + kr0 * a.ld_kv;
     // every producer is done with the previous item (and its index list)
     if (lane == 0) mbar_arrive(smem_u32(&sm.pitem));
     if (!mbar_wait(smem_u32(&sm.pitem), static_cast<uint32_t>(nitem & 1), abort, kErrTimeoutProducer))
@@ -363,7 +374,7 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
         sm.vmask[stage] = valid;
         sm.last[stage] = (t == nt - 1);
       }
-      if (a.kv8) {
+      if constexpr (KV8) {
         // the raw fp8 row lands in the slot's last 656 bytes; the warp dequantises
         // its rows of the previous tile while these copies are in flight
         const uint32_t rb = smem_u32(&sm.rawf[stage]);
@@ -372,7 +383,7 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
         __syncwarp();
         if (mine && s >= 0)
           bulk_g2s(kv0 + (stage * AT_BK + lane) * AT_ROWB + (AT_ROWB - KV8_ROW_BYTES),
-                   kvb8 + static_cast<long>(s) * a.ld_kv8, KV8_ROW_BYTES, rb);
+                   kvb8 + static_cast<long>(s) * a.ld_kv, KV8_ROW_BYTES, rb);
         if (!dequant_pending()) {
           ok = false;
           break;
@@ -397,13 +408,13 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a) {
     }
     if (!ok) break;
   }
-  if (a.kv8 && !*abort) (void)dequant_pending();  // the last tile
+  if (KV8 && !*abort) (void)dequant_pending();  // the last tile
   if (*abort) {
     // let every copy still in flight land before the CTA exits
     volatile int never = 0;
     const long n = issued < AT_STAGES ? issued : AT_STAGES;
     for (long j = issued - n; j < issued; ++j)
-      (void)mbar_wait(smem_u32(a.kv8 ? &sm.rawf[j % AT_STAGES] : &sm.full[j % AT_STAGES]),
+      (void)mbar_wait(smem_u32(KV8 ? &sm.rawf[j % AT_STAGES] : &sm.full[j % AT_STAGES]),
                       static_cast<uint32_t>((j / AT_STAGES) & 1), &never, kErrTimeoutDrain);
     if (qloads > 0) (void)mbar_wait(smem_u32(&sm.qfull), (qloads - 1) & 1, &never, kErrTimeoutDrain);
     for (int b2 = 0; b2 < 2; ++b2)
@@ -584,7 +595,6 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
     }
 
     // ---- item epilogue: head h's final max and sum live in warp h/2
-    if (a.early && it == 0) grid_dep_wait();  // the previous kernel's reads are done
     named_bar_sync(1, AT_CONSUMERS);  // every warp's P V of the item is done
     if ((lane & 15) == 0) {
       sm.fin_m[sh] = m_run;
@@ -627,7 +637,9 @@ __device__ __forceinline__ void attn_consumer(AttnSmem& sm, const AttnArgs& a) {
   }
 }
 
-__global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const __grid_constant__ AttnArgs a) {
+template <bool KV8, bool SEGS>
+__global__ void __launch_bounds__(AT_THREADS, 1)
+    attn_mla_kernel(const AttnArgs a, const __grid_constant__ AttnSegParam<SEGS> sg) {
   extern __shared__ uint8_t at_smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(
       (reinterpret_cast<uintptr_t>(at_smem_raw) + 127) & ~static_cast<uintptr_t>(127));
@@ -641,7 +653,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const __grid_co
     mbar_init(smem_u32(&sm.ifull[0]), 1);
     mbar_init(smem_u32(&sm.ifull[1]), 1);
     mbar_init(smem_u32(&sm.pitem), AT_PRODUCERS);
-    for (int st = 0; st < AT_STAGES; ++st) mbar_init(smem_u32(&sm.rawf[st]), AT_PRODUCERS);
+    if (KV8)
+      for (int st = 0; st < AT_STAGES; ++st) mbar_init(smem_u32(&sm.rawf[st]), AT_PRODUCERS);
     sm.abort = 0;
     fence_barrier_init();
   }
@@ -652,10 +665,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const __grid_co
     z[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   __syncthreads();
-  grid_dep_signal();
-  if (!a.early) grid_dep_wait();  // set-up above touches no global memory
+  grid_dep_wait();  // set-up above touches no global memory
   if (threadIdx.x >= AT_CONSUMERS)
-    attn_producer(sm, a);
+    attn_producer<KV8, SEGS>(sm, a, sg);
   else
     attn_consumer(sm, a);
   __syncthreads();
@@ -667,7 +679,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_mla_kernel(const __grid_co
 // them with shuffles; every thread accumulates its output dims over the pieces.
 __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, int maxp, long tot,
                                     int tq, int G, __nv_bfloat16* out, float* lse) {
-  grid_dep_signal();
   grid_dep_wait();
   const long qrow = blockIdx.x;
   const int h = blockIdx.y;
@@ -765,10 +776,23 @@ size_t attn_mla_ws_bytes(int batch, int rows, int k) {
   return static_cast<size_t>(items) * p.maxp * AT_H * (AT_DV + 2) * sizeof(float);
 }
 
+template <bool KV8, bool SEGS>
+static ic_status launch_attn_inst(const AttnArgs& a, const AttnSegParam<SEGS>& sg, long grid,
+                                  cudaStream_t stream) {
+  const int smem = static_cast<int>(sizeof(AttnSmem)) + 128;
+  ic_status st = cuda_check(cudaFuncSetAttribute(attn_mla_kernel<KV8, SEGS>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                            "cudaFuncSetAttribute(attn)");
+  if (st) return st;
+  return cuda_check(launch_dep(attn_mla_kernel<KV8, SEGS>, dim3(static_cast<unsigned>(grid)),
+                               dim3(AT_THREADS), smem, stream, 1, a, sg),
+                    "attn_mla_kernel launch");
+}
+
 ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* idx, int batch,
                           int rows, int Lkv, int k, float scale, void* out, float* lse, void* ws,
                           size_t ws_bytes, long long valid_entries, cudaStream_t stream,
-                          bool kv8, const AttnSeg* segs, int nseg, bool early) {
+                          bool kv8, const AttnSeg* segs, int nseg) {
   const long items = static_cast<long>(batch) * rows;
   if (nseg < 0 || nseg > IC_MAXSEG || (nseg > 0 && (batch != 1 || !segs)))
     return fail(IC_ERR_INVALID_ARG, "attn: bad segment list (%d)", nseg);
@@ -780,11 +804,8 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
     p.split = false;
   AttnArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
-  a.kv = kv8 ? nullptr : static_cast<const __nv_bfloat16*>(kv);
-  a.ld_kv = kv8 ? 0 : ld_kv;
-  a.kv8 = kv8 ? 1 : 0;
-  a.kv8p = kv8 ? static_cast<const uint8_t*>(kv) : nullptr;
-  a.ld_kv8 = kv8 ? ld_kv : 0;
+  a.kv = static_cast<const __nv_bfloat16*>(kv);  // fp8 cache: rows of ld_kv bytes
+  a.ld_kv = ld_kv;
   a.idx = idx;
   a.B = batch;
   a.R = rows;
@@ -801,18 +822,19 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
   a.idx_bulk = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
   a.part_o = p.split ? static_cast<float*>(ws) : nullptr;
   a.part_ml = p.split ? static_cast<float*>(ws) + items * p.maxp * AT_H * AT_DV : nullptr;
-  a.nseg = nseg;
-  for (int j = 0; j < nseg; ++j) a.seg[j] = segs[j];
-  a.early = early ? 1 : 0;
-  const int smem = static_cast<int>(sizeof(AttnSmem)) + 128;
-  ic_status st = cuda_check(
-      cudaFuncSetAttribute(attn_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
-      "cudaFuncSetAttribute(attn)");
-  if (st) return st;
   const long grid = p.split ? p.G : (items < num_sms() ? items : num_sms());
-  st = cuda_check(launch_dep(attn_mla_kernel, dim3(static_cast<unsigned>(grid)), dim3(AT_THREADS),
-                             smem, stream, 1, a),
-                  "attn_mla_kernel launch");
+  ic_status st;
+  if (nseg > 0) {
+    AttnSegs sg;
+    sg.nseg = nseg;
+    for (int j = 0; j < nseg; ++j) sg.seg[j] = segs[j];
+    st = kv8 ? launch_attn_inst<true, true>(a, sg, grid, stream)
+             : launch_attn_inst<false, true>(a, sg, grid, stream);
+  } else {
+    const AttnNoSegs sg{0};
+    st = kv8 ? launch_attn_inst<true, false>(a, sg, grid, stream)
+             : launch_attn_inst<false, false>(a, sg, grid, stream);
+  }
   if (st) return st;
   // algorithmic bytes: each selected latent row gathered once, q read once, out written once
   const double ve = valid_entries >= 0 ? static_cast<double>(valid_entries)

@@ -118,13 +118,11 @@ ic_status launch_topk(const float* scores, long rows, int n, long ld, long pos0,
 // kv8: kv holds fp8 latent rows (KV8_ROW_BYTES, ld_kv in bytes), else bf16 rows
 // (ld_kv in elements).
 // segs (nseg <= IC_MAXSEG, host array): packed sequences, with batch = 1 and rows =
-// all their query rows; Lkv is then ignored.  early: q, kv and idx are not written
-// by the previous kernel of the stream (see AttnArgs::early).
+// all their query rows; Lkv is then ignored.
 ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* idx, int batch,
                           int rows, int Lkv, int k, float scale, void* out, float* lse,
                           void* ws, size_t ws_bytes, long long valid_entries, cudaStream_t stream,
-                          bool kv8 = false, const AttnSeg* segs = nullptr, int nseg = 0,
-                          bool early = false);
+                          bool kv8 = false, const AttnSeg* segs = nullptr, int nseg = 0);
 size_t attn_mla_ws_bytes(int batch, int rows, int k);
 ic_status launch_attn_f32(const float* q, const float* kv, long ld_kv, const float* v,
                           const int* idx, int batch, int rows, int heads, int dk, int dv,
