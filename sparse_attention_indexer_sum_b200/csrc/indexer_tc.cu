@@ -687,12 +687,18 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
               tmem_ld16(tok_addr(tk) + 16 * part, v);
               tmem_ld_wait();
 #pragma unroll
-              for (int h4 = 0; h4 < 4; ++h4) {
+              for (int h4 = 0; h4 < 4; ++h4) {  // chains (s0, s1) and (s2, s3) in pairs
                 const int h = 16 * part + 4 * h4;
-                s0 = fmaf(wr[tk][h], fmaxf(v[4 * h4 + 0], 0.f), s0);
-                s1 = fmaf(wr[tk][h + 1], fmaxf(v[4 * h4 + 1], 0.f), s1);
-                s2 = fmaf(wr[tk][h + 2], fmaxf(v[4 * h4 + 2], 0.f), s2);
-                s3 = fmaf(wr[tk][h + 3], fmaxf(v[4 * h4 + 3], 0.f), s3);
+                const float2 p01 = ffma2(make_float2(wr[tk][h], wr[tk][h + 1]),
+                                         make_float2(fmaxf(v[4 * h4 + 0], 0.f), fmaxf(v[4 * h4 + 1], 0.f)),
+                                         make_float2(s0, s1));
+                const float2 p23 = ffma2(make_float2(wr[tk][h + 2], wr[tk][h + 3]),
+                                         make_float2(fmaxf(v[4 * h4 + 2], 0.f), fmaxf(v[4 * h4 + 3], 0.f)),
+                                         make_float2(s2, s3));
+                s0 = p01.x;
+                s1 = p01.y;
+                s2 = p23.x;
+                s3 = p23.y;
               }
             }
             res[tk] = (s0 + s1) + (s2 + s3);
@@ -717,12 +723,18 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
             tmem_ld16(tok_addr(0) + 32 * half + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
             tmem_ld_wait();
 #pragma unroll
-            for (int h = 0; h < 32; h += 4) {
+            for (int h = 0; h < 32; h += 4) {  // chains (s0, s1) and (s2, s3) in pairs
               const float4 wv = *reinterpret_cast<const float4*>(wsl + 32 * half + h);
-              s0 = fmaf(wv.x, fmaxf(v[h + 0], 0.f), s0);
-              s1 = fmaf(wv.y, fmaxf(v[h + 1], 0.f), s1);
-              s2 = fmaf(wv.z, fmaxf(v[h + 2], 0.f), s2);
-              s3 = fmaf(wv.w, fmaxf(v[h + 3], 0.f), s3);
+              const float2 p01 =
+                  ffma2(make_float2(wv.x, wv.y),
+                        make_float2(fmaxf(v[h + 0], 0.f), fmaxf(v[h + 1], 0.f)), make_float2(s0, s1));
+              const float2 p23 =
+                  ffma2(make_float2(wv.z, wv.w),
+                        make_float2(fmaxf(v[h + 2], 0.f), fmaxf(v[h + 3], 0.f)), make_float2(s2, s3));
+              s0 = p01.x;
+              s1 = p01.y;
+              s2 = p23.x;
+              s3 = p23.y;
             }
           }
           res[0] = (s0 + s1) + (s2 + s3);
