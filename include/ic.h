@@ -35,6 +35,12 @@
  *  - Kernels never trap: a device-side wait that runs out of time (2 s)
  *    records a code in the device error word, abandons its work and returns;
  *    ic_device_status() reports it (IC_ERR_TIMEOUT).
+ *  - libic_b200_debug.so, the same library built with -DIC_DEBUG_BOUNDS, also
+ *    checks the indices its kernels compute (index-list entries against their
+ *    cache, TMA tile coordinates, top-k and merge output slots) before using
+ *    them; a failed check skips the access and ic_device_status() reports
+ *    IC_ERR_BOUNDS.  (Index-list entries outside the cache are skipped in every
+ *    build; only the debug build reports them.)
  */
 #ifndef IC_H_
 #define IC_H_
@@ -53,6 +59,7 @@ typedef int ic_status;
 #define IC_ERR_WORKSPACE (-3)   /* workspace missing or too small              */
 #define IC_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed           */
 #define IC_ERR_TIMEOUT (-5)     /* a device-side bounded wait gave up          */
+#define IC_ERR_BOUNDS (-6)      /* a debug-bounds build caught an index out of range */
 
 typedef enum { IC_F32 = 0, IC_BF16 = 1, IC_E4M3 = 2 } ic_dtype;
 
@@ -64,7 +71,8 @@ int ic_version(void);
 
 /* Synchronise `stream`, then read and clear the device error word.
  * Returns IC_OK, IC_ERR_TIMEOUT (a bounded device wait gave up since the last
- * check) or IC_ERR_CUDA. */
+ * check), IC_ERR_BOUNDS (debug-bounds build: an index check failed) or
+ * IC_ERR_CUDA. */
 ic_status ic_device_status(void* stream);
 
 /*

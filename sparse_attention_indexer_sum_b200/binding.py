@@ -14,7 +14,10 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libic_b200.so")
+# IC_DEBUG_BOUNDS=1 in the environment selects the debug-bounds build of the same
+# library (device-side index checks reported as IC_ERR_BOUNDS; see ic.h)
+LIB_PATH = os.path.join(_PKG, "libic_b200_debug.so" if os.environ.get("IC_DEBUG_BOUNDS") == "1"
+                        else "libic_b200.so")
 
 IC_OK = 0
 IC_ERR_INVALID_ARG = -1
@@ -22,6 +25,7 @@ IC_ERR_UNSUPPORTED = -2
 IC_ERR_WORKSPACE = -3
 IC_ERR_CUDA = -4
 IC_ERR_TIMEOUT = -5
+IC_ERR_BOUNDS = -6
 IC_F32, IC_BF16, IC_E4M3 = 0, 1, 2
 
 # names declared in include/ic.h (checked against the header by the tests)
@@ -155,7 +159,8 @@ def _contig(*ts):
 
 
 def ic_device_status(stream=None):
-    """Synchronises the stream; raises ICError(IC_ERR_TIMEOUT) if a device wait gave up."""
+    """Synchronises the stream; raises ICError(IC_ERR_TIMEOUT) if a device wait gave up
+    (IC_ERR_BOUNDS if a debug-bounds check failed)."""
     _check(lib().ic_device_status(_stream(stream)))
 
 

@@ -10,6 +10,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libic_b200.so")
+# the same sources with -DIC_DEBUG_BOUNDS: device-side index checks (see ic.h)
+LIB_DEBUG = os.path.join(PKG, "libic_b200_debug.so")
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
     "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
@@ -28,26 +30,29 @@ def sources() -> list[str]:
                   + glob.glob(os.path.join(CSRC, "*.h")) + [os.path.join(ROOT, "include", "ic.h")])
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and not stale():
-        return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc()] + NVCC_FLAGS + (extra or []) + ["-I", os.path.join(ROOT, "include"),
-                                                   "-o", tmp, os.path.join(CSRC, "libic.cu")]
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          debug_bounds: bool = False) -> str:
+    lib = LIB_DEBUG if debug_bounds else LIB
+    if not force and not stale(lib):
+        return lib
+    tmp = lib + ".tmp%d" % os.getpid()
+    cmd = [nvcc()] + NVCC_FLAGS + (["-DIC_DEBUG_BOUNDS"] if debug_bounds else []) + (extra or []) + [
+        "-I", os.path.join(ROOT, "include"), "-o", tmp, os.path.join(CSRC, "libic.cu")]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None)
+          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None,
+          debug_bounds="--debug-bounds" in sys.argv)

@@ -393,7 +393,7 @@ extern "C" {
 
 const char* ic_last_error(void) { return t_last_error.c_str(); }
 
-int ic_version(void) { return 101; }
+int ic_version(void) { return 102; }
 
 ic_status ic_device_status(void* stream) {
   ic_status st = cuda_check(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)),
@@ -406,6 +406,12 @@ ic_status ic_device_status(void* stream) {
     const int zero = 0;
     st = cuda_check(cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(int)), "clear device error word");
     if (st) return st;
+    if (v >= kErrBoundsFirst)
+      return fail(IC_ERR_BOUNDS, "device error word %d (a debug-bounds check failed: %s)", v,
+                  v == kErrBoundsGather ? "index-list entry outside the cache"
+                  : v == kErrBoundsTma  ? "TMA tile coordinate outside the tensor"
+                  : v == kErrBoundsTopk ? "top-k output slot outside the row"
+                                        : "merge slot or piece count out of range");
     return fail(IC_ERR_TIMEOUT, "device error word %d (a bounded device wait gave up)", v);
   }
   return IC_OK;

@@ -368,7 +368,7 @@ __device__ __forceinline__ void attn_producer(AttnSmem& sm, const AttnArgs& a,
       }
       const int j = t * AT_BK + lane;
       int s = (t < ntiles && j < cnt) ? ilist[j] : -1;
-      if (s >= lkv) s = -1;
+      if (!in_bounds(s >= -1 && s < lkv, kErrBoundsGather) || s >= lkv) s = -1;
       const unsigned valid = __ballot_sync(0xffffffffu, s >= 0);
       if (pw == 0 && lane == 0) {
         sm.vmask[stage] = valid;
@@ -683,7 +683,8 @@ __global__ void attn_combine_kernel(const float* part_o, const float* part_ml, i
   const long qrow = blockIdx.x;
   const int h = blockIdx.y;
   const long c0 = attn_cta_of(qrow * tq, tot, G);
-  const int np = static_cast<int>(attn_cta_of((qrow + 1) * tq - 1, tot, G) - c0 + 1);  // <= 64
+  int np = static_cast<int>(attn_cta_of((qrow + 1) * tq - 1, tot, G) - c0 + 1);  // <= 64
+  if (!in_bounds(np <= 64, kErrBoundsMerge)) np = 64;
   const long s0 = qrow * maxp;
   // Each thread owns 4 adjacent output dims.  The first CMB_PRE pieces' partial
   // outputs are loaded before the weights are known, so their latency overlaps

@@ -31,9 +31,32 @@ enum DevErr : int {
   kErrTimeoutEpilogue = 3,
   kErrTimeoutDrain = 4,
   kErrTopkOverflow = 5,
+  // debug-bounds builds only (codes >= kErrBoundsFirst)
+  kErrBoundsFirst = 16,
+  kErrBoundsGather = 16,  // an index-list entry outside [-1, rows of its cache)
+  kErrBoundsTma = 17,     // a TMA tile coordinate outside its tensor's rows
+  kErrBoundsTopk = 18,    // a top-k output slot or index outside its row
+  kErrBoundsMerge = 19,   // a merge output slot or piece count out of range
 };
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_dev_error, 0, code); }
+
+// Debug-bounds builds (nvcc -DIC_DEBUG_BOUNDS, libic_b200_debug.so) check indices
+// the kernels compute before they use them: a failed check records `code` in the
+// device error word (ic_device_status then returns IC_ERR_BOUNDS) and the access is
+// skipped.  In other builds the check compiles away and returns true.
+__device__ __forceinline__ bool in_bounds(bool ok, int code) {
+#ifdef IC_DEBUG_BOUNDS
+  if (!ok) {
+    record_error(code);
+    return false;
+  }
+#else
+  (void)ok;
+  (void)code;
+#endif
+  return true;
+}
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;

@@ -504,6 +504,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
               break;
             const QbInfo x = qb_info<TPM, SEGS>(a, it.qb);
             const int qrow = static_cast<int>((x.qrow0 + x.ql * TPM) * 64);
+            (void)in_bounds(qrow >= 0 && x.ql * TPM < x.R, kErrBoundsTma);  // loads stay legal
             mbar_arrive_expect_tx(qfull_bar, C::Q_BYTES);
 #pragma unroll
             for (int kb = 0; kb < C::KBLK; ++kb)
@@ -512,7 +513,9 @@ __global__ void __launch_bounds__(IdxCfg<FP8, TPM, FUSED>::THREADS, 1)
             cur_qb = it.qb;
           }
           if (!mbar_wait(empty_bar(stage), ph ^ 1, abort_flag, kErrTimeoutProducer)) break;
-          const int krow = static_cast<int>(qb_info<TPM, SEGS>(a, it.qb).krow0 + it.kt * C::BM);
+          const QbInfo kx = qb_info<TPM, SEGS>(a, it.qb);
+          const int krow = static_cast<int>(kx.krow0 + it.kt * C::BM);
+          (void)in_bounds(krow >= 0 && it.kt * C::BM < kx.Lk, kErrBoundsTma);
           mbar_arrive_expect_tx(full_bar(stage), C::A_BYTES);
 #pragma unroll
           for (int kb = 0; kb < C::KBLK; ++kb)

@@ -314,7 +314,7 @@ __device__ __noinline__ void topk_exact(TopkSmem& sm, const float* __restrict__ 
       const int mid = (lo + hi) >> 1;
       if (sm.u.ex.sel_idx[mid] < v) lo = mid + 1; else hi = mid;
     }
-    out[p + lo] = v;
+    if (in_bounds(p + lo < k, kErrBoundsTopk)) out[p + lo] = v;
   }
   for (int p = threadIdx.x; p < S; p += TK_THREADS) {
     const int v = sm.u.ex.sel_idx[p];
@@ -323,7 +323,7 @@ __device__ __noinline__ void topk_exact(TopkSmem& sm, const float* __restrict__ 
       const int mid = (lo + hi) >> 1;
       if (sm.u.ex.gt_idx[mid] < v) lo = mid + 1; else hi = mid;
     }
-    out[p + lo] = v;
+    if (in_bounds(p + lo < k, kErrBoundsTopk)) out[p + lo] = v;
   }
 }
 
@@ -585,7 +585,8 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
       uint32_t bits = sm.u.bitmap[w];
       while (bits) {
         const int b = __ffs(bits) - 1;
-        out[pos++] = (w << 5) + b;
+        if (in_bounds(pos < k, kErrBoundsTopk)) out[pos] = (w << 5) + b;
+        ++pos;
         bits &= bits - 1;
       }
     }
@@ -842,7 +843,8 @@ __global__ void __launch_bounds__(TK_THREADS) topk_merge_kernel(
     for (int u = 0; u < 8; ++u) {
       if ((m[u] >> lane) & 1u) {
         const int p = wbase + sm.hist[u * TK_NW + warp] + __popc(m[u] & lt);
-        if (p < k) out[p] = static_cast<int>(~static_cast<uint32_t>(c[u]));
+        if (in_bounds(p < k, kErrBoundsMerge) && p < k)
+          out[p] = static_cast<int>(~static_cast<uint32_t>(c[u]));
       }
     }
     wbase += sm.counter;

@@ -40,8 +40,17 @@ def test_library_exports_every_declared_symbol(lib):
     assert exported == set(_declared())
 
 
+def test_debug_bounds_library_exports_the_same_symbols():
+    # the -DIC_DEBUG_BOUNDS build of the same sources (device-side index checks)
+    path = build.build(debug_bounds=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True,
+                         check=True).stdout
+    assert set(re.findall(r"\s[TW]\s+(ic_\w+)$", out, flags=re.M)) == set(_declared())
+    assert ctypes.CDLL(path).ic_version() == binding.lib().ic_version()
+
+
 def test_version_and_empty_error(lib):
-    assert binding.ic_version() == 101
+    assert binding.ic_version() == 102
     assert isinstance(binding.ic_last_error(), str)
 
 
