@@ -217,22 +217,22 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------------ fused top-k
-// The epilogue warps leave each tile's 128 scores in a staging ring, with one
-// 32-bit mask per warp of the keys that may be candidates; one streaming selector
-// warp walks the tiles in order and appends those keys' selection keys, in index
-// order, to a shared-memory buffer for the row it is working on.  The buffer has
-// a rising threshold tau: it holds every key of the CTA's share of the row seen so
-// far whose selection key is >= tau (and possibly some below).  When it fills
-// up, the streaming warp and three helper warps find by a radix descent a new
-// tau with at least k and at most `target` buffered keys >= tau, and compact the
-// buffer to those, keeping their order.  A key below tau has at least k larger
+// Each epilogue warp leaves, per tile, the selection keys of its 32 keys that may
+// be candidates -- packed in index order -- and their count in a staging ring; one
+// streaming selector warp walks the tiles in order and appends them to a
+// shared-memory buffer for the row it is working on, keeping index order.  The
+// buffer has a rising threshold tau: it holds every key of the CTA's share of the
+// row seen so far whose selection key is >= tau (and possibly some below).  When
+// it fills up, the streaming warp and three helper warps find by a radix descent a
+// new tau with at least k and at most `target` buffered keys >= tau, and compact
+// the buffer to those, keeping their order.  A key below tau has at least k larger
 // keys in the same share of the row, so it cannot be among the row's top k.  The
 // streaming warp publishes tau's score key, tagged with the row, and the epilogue
-// leaves keys whose score key is below it out of the masks (a stale value only
-// lets more keys through).  At the end of the row (or of the CTA's work) the
-// buffer goes to the row's slot in global memory.  Selection runs beside the
-// tensor-core pipeline: a compaction only delays the selectors, which the staging
-// ring absorbs.
+// stages no key whose score key is below it (a stale value only lets more keys
+// through).  At the end of the row (or of the CTA's work) the buffer goes to the
+// row's slot in global memory.  Selection runs beside the tensor-core pipeline;
+// the staging ring absorbs short delays, but a compaction outlasts it and holds
+// the epilogue (and so the tensor pipe) until it ends.
 //
 // The four selector warps meet on an mbarrier (one arrival per warp) that each
 // waits on by polling, bounded in time and by the CTA's abort flag; a warp whose
