@@ -4,6 +4,7 @@
     python -m sparse_attention_indexer_sum_b200.profile_cases indexer_longrows_e4m3
     python -m sparse_attention_indexer_sum_b200.profile_cases attn_tail4k
     python -m sparse_attention_indexer_sum_b200.profile_cases decode_indexer
+    python -m sparse_attention_indexer_sum_b200.profile_cases decode_indexer_fused
     python -m sparse_attention_indexer_sum_b200.profile_cases decode_attn
     python -m sparse_attention_indexer_sum_b200.profile_cases decode_step
 
@@ -26,6 +27,9 @@ name captures a warm launch. Every case fits in a few GB of device memory.
                     over 2048 random distinct rows of its own 20000-row latent KV
                     (1.5 GB in all, far beyond L2); split over the SMs, partials
                     merged by the combine kernel.
+  decode_indexer_fused  the decode_indexer inputs through ic_indexer_topk (the
+                    fused indexer -> top-k: indexer_tc_kernel's fused instance, then
+                    topk_merge_kernel).
   decode_step       the whole F,S,S,S decode step of 64 sequences x 1 query over
                     200000 tokens (ic_decode_step: e4m3 indexer, top-k, four
                     attention layers with their merges).  The four layers share
@@ -143,6 +147,22 @@ def decode_indexer():
     _rounds(rnd)
 
 
+def decode_indexer_fused():
+    dev = "cuda"
+    B, L = 64, 200000
+    g = torch.Generator(device=dev).manual_seed(0)
+    q = (torch.randn(B, 1, 64, 128, device=dev, generator=g) / math.sqrt(128)).to(torch.bfloat16)
+    q8, qs = ic.ic_quant_e4m3_rows(q)
+    k8 = torch.empty(B, L, 128, dtype=torch.uint8, device=dev)
+    ks = torch.empty(B, L, dtype=torch.float32, device=dev)
+    for b in range(B):
+        kb = (torch.randn(L, 128, device=dev, generator=g) / math.sqrt(128)).to(torch.bfloat16)
+        ic.ic_quant_e4m3_rows(kb, codes=k8[b], scales=ks[b])
+    w = torch.rand(B, 1, 64, device=dev, generator=g) / 8
+    ws = torch.empty(ic.ic_indexer_topk_workspace_size(B, L, L - 1) // 4 + 4, device=dev)
+    _rounds(lambda: ic.ic_indexer_topk(q8, k8, w, 2048, ws, pos0=L - 1, q_scale=qs, k_scale=ks))
+
+
 def decode_attn():
     dev = "cuda"
     wl = synth.variant("decode_200k", L=20000)
@@ -184,7 +204,8 @@ def decode_step():
 
 CASES = {"indexer_longrows": indexer_longrows, "indexer_longrows_e4m3": indexer_longrows_e4m3,
          "attn_tail4k": attn_tail4k,
-         "decode_indexer": decode_indexer, "decode_attn": decode_attn,
+         "decode_indexer": decode_indexer, "decode_indexer_fused": decode_indexer_fused,
+         "decode_attn": decode_attn,
          "decode_step": decode_step}
 
 
