@@ -49,7 +49,7 @@ from . import synth
 
 def _report(trace):
     for name, ms, work in trace:
-        unit = "TFLOP/s" if name.startswith("indexer_tc") else "GB/s"
+        unit = "TFLOP/s" if name.startswith("indexer") else "GB/s"
         rate = work / ms / 1e9 if unit == "TFLOP/s" else work / ms / 1e6
         print("%-18s %9.3f ms  %10.1f %s" % (name, ms, rate, unit))
 
