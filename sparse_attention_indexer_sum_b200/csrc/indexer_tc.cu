@@ -96,7 +96,9 @@ struct IdxCfg {
   // Epilogue warp sets: set j takes the accumulator slots a with a % NSETS == j, so
   // each set sees every use of its slots in order.  One-token blocks (decode) have
   // little epilogue work per tile; several sets overlap consecutive tiles.
-  static constexpr int NSETS = (TPM == 4) ? 1 : 3;
+  // (the fused instance keeps two sets: with its selector warps, three sets would
+  // cap every thread at 96 registers and spill; two measured 4 % faster)
+  static constexpr int NSETS = (TPM == 4) ? 1 : (FUSED ? 2 : 3);
   static constexpr int SETW = 4 * EPG;             // warps per set
   static constexpr int NEPI = SETW * NSETS;
   static constexpr int TOK_PER_EW = TPM / EPG;     // tokens per epilogue warp
