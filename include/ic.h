@@ -369,13 +369,12 @@ ic_status ic_layer_stack_rows(const char* pattern, const ic_stack_desc* desc,
  * ic_layer_stack would with desc->L = L_i.  cu_seqlens: host int64 [nseq + 1],
  * cu_seqlens[0] = 0, nondecreasing, every L_i <= desc->L (desc->L sizes the
  * workspace: ic_stack_workspace_size(desc) covers any batch).
- * bf16 / e4m3 stacks share their launches between sequences: an F layer walks the
- * packed query rows in blocks of as many score rows as the workspace holds
- * (desc->L floats plus one int32 each), each block touching at most 64 sequences,
- * with one indexer, one valid-length and one top-k launch per block (each row
- * scored against its own sequence's keys); every layer's attention runs once per
- * group of up to 64 whole sequences.  The fp32 forms run the sequences one after
- * another.  Errors as ic_layer_stack (the fp32 forms name the sequence).
+ * The sequences share their launches: an F layer walks the packed query rows in
+ * blocks of as many score rows as the workspace holds (desc->L floats plus one
+ * int32 each), each block touching at most 64 sequences, with one indexer, one
+ * valid-length and one top-k launch per block (each row scored against its own
+ * sequence's keys); every layer's attention runs once per group of up to 64 whole
+ * sequences.  Errors as ic_layer_stack.
  */
 ic_status ic_layer_stack_varlen(const char* pattern, const ic_stack_desc* desc,
                                 const ic_layer_io* layers, int nlayers, const long* cu_seqlens,

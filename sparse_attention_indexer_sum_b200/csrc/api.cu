@@ -275,7 +275,7 @@ static ic_status run_stack(const char* pattern, const ic_stack_desc* d, const ic
   return IC_OK;
 }
 
-// Packed sequences (cu: host [nseq + 1]) of a bf16 / e4m3 stack in shared launches.
+// Packed sequences (cu: host [nseq + 1]) of a stack in shared launches.
 // F layers walk the packed query rows in blocks that fit the score workspace and
 // touch at most IC_MAXSEG sequences: one indexer launch over the block's segments
 // (each row against its own sequence's keys), one valid-length fill and one top-k
@@ -310,9 +310,11 @@ static ic_status run_stack_varlen_shared(const std::vector<char>& kinds, const i
   float* scores = static_cast<float*>(workspace);
   int* valid = reinterpret_cast<int*>(scores + rb * ld);
   const bool kv8 = d->attn_dtype == IC_E4M3;
-  const size_t qe = 2;
+  const bool f32_idx = d->idx_dtype == IC_F32, f32_attn = d->attn_dtype == IC_F32;
+  const size_t qe = f32_attn ? 4 : 2;  // q and out: fp32 (MQA) or bf16 (MLA)
   const size_t arow_b = static_cast<size_t>(d->heads) * d->dk * qe;
   const size_t orow_b = static_cast<size_t>(d->heads) * d->dv * qe;
+  const size_t qrow_b = static_cast<size_t>(d->H) * d->D * elem_bytes(d->idx_dtype);
   std::vector<IdxSeg> segs;
   std::vector<AttnSeg> asegs;
   for (int l = 0; l < nlayers; ++l) {
@@ -341,10 +343,16 @@ static ic_status run_stack_varlen_shared(const std::vector<char>& kinds, const i
           segs.push_back(g);
         }
         const long nu = u1 - u0;
-        ic_status st = launch_indexer_tc_segs(d->idx_dtype == IC_E4M3, io.q_idx, io.q_scale,
-                                              io.k_idx, io.k_scale, io.w, segs.data(),
-                                              static_cast<int>(segs.size()), total, total, scores,
-                                              ld, stream);
+        ic_status st =
+            f32_idx ? launch_indexer_f32_segs(
+                          reinterpret_cast<const float*>(static_cast<const uint8_t*>(io.q_idx) +
+                                                         u0 * qrow_b),
+                          static_cast<const float*>(io.k_idx), io.w + u0 * d->H, d->H, d->D,
+                          segs.data(), static_cast<int>(segs.size()), nu, scores, ld, stream)
+                    : launch_indexer_tc_segs(d->idx_dtype == IC_E4M3, io.q_idx, io.q_scale,
+                                             io.k_idx, io.k_scale, io.w, segs.data(),
+                                             static_cast<int>(segs.size()), total, total, scores,
+                                             ld, stream);
         if (st) return st;
         st = launch_fill_valid_len(segs.data(), static_cast<int>(segs.size()), nu, valid, stream);
         if (st) return st;
@@ -372,12 +380,18 @@ static ic_status run_stack_varlen_shared(const std::vector<char>& kinds, const i
         asegs.push_back(a);
         valid_entries += causal_pairs(n, d->k, 0);
       }
-      ic_status st = launch_attn_mla(static_cast<const uint8_t*>(io.q) + r0 * arow_b, io.kv,
-                                     d->ld_kv, t_cache + r0 * d->k, 1, static_cast<int>(nr), d->L,
-                                     d->k, d->scale,
-                                     static_cast<uint8_t*>(io.out) + r0 * orow_b,
-                                     io.lse ? io.lse + r0 * d->heads : nullptr, workspace, ws_bytes,
-                                     valid_entries, stream, kv8, asegs.data(),
+      const void* qg = static_cast<const uint8_t*>(io.q) + r0 * arow_b;
+      void* og = static_cast<uint8_t*>(io.out) + r0 * orow_b;
+      float* lg = io.lse ? io.lse + r0 * d->heads : nullptr;
+      ic_status st =
+          f32_attn ? launch_attn_f32(static_cast<const float*>(qg), static_cast<const float*>(io.kv),
+                                     d->ld_kv, static_cast<const float*>(io.v), t_cache + r0 * d->k,
+                                     1, static_cast<int>(nr), d->heads, d->dk, d->dv, d->L, d->k,
+                                     d->scale, static_cast<float*>(og), lg, stream, asegs.data(),
+                                     static_cast<int>(asegs.size()))
+                   : launch_attn_mla(qg, io.kv, d->ld_kv, t_cache + r0 * d->k, 1,
+                                     static_cast<int>(nr), d->L, d->k, d->scale, og, lg, workspace,
+                                     ws_bytes, valid_entries, stream, kv8, asegs.data(),
                                      static_cast<int>(asegs.size()));
       if (st) return st;
     }
@@ -580,59 +594,18 @@ ic_status ic_layer_stack_varlen(const char* pattern, const ic_stack_desc* desc,
                   cu_seqlens[i + 1] - cu_seqlens[i], desc->L);
   if (nlayers < 1 || nlayers > 4096 || !layers)
     return fail(IC_ERR_INVALID_ARG, "varlen: bad layers / nlayers");
-  if (desc->idx_dtype != IC_F32 && desc->attn_dtype != IC_F32 && !desc->decode) {
-    ic_status st = check_desc(desc, false);
-    if (st) return st;
-    std::vector<char> kinds;
-    st = parse_pattern(pattern, &kinds);
-    if (st) return st;
-    if (static_cast<int>(kinds.size()) != nlayers)
-      return fail(IC_ERR_INVALID_ARG, "pattern has %zu layers, nlayers is %d", kinds.size(),
-                  nlayers);
-    if (!t_cache) return fail(IC_ERR_INVALID_ARG, "varlen: NULL t_cache");
-    if (cu_seqlens[nseq] * 64 > 0x7fffffffL)
-      return fail(IC_ERR_UNSUPPORTED, "varlen: too many rows for 32-bit TMA coordinates");
-    return run_stack_varlen_shared(kinds, desc, layers, nlayers, cu_seqlens, nseq, t_cache,
-                                   workspace, ws_bytes, static_cast<cudaStream_t>(stream));
-  }
-  // fp32 forms (small shapes): the sequences run one after another
-  const size_t qrow_b = static_cast<size_t>(desc->H) * desc->D * elem_bytes(desc->idx_dtype);
-  const size_t krow_b = static_cast<size_t>(desc->D) * elem_bytes(desc->idx_dtype);
-  // q, v and out are fp32 (MQA) or bf16 (MLA, also over an e4m3 cache, whose ld_kv is
-  // in bytes)
-  const size_t qe = desc->attn_dtype == IC_F32 ? 4 : 2;
-  const size_t arow_b = static_cast<size_t>(desc->heads) * desc->dk * qe;
-  const size_t kvrow_b = static_cast<size_t>(desc->ld_kv) * elem_bytes(desc->attn_dtype);
-  const size_t vrow_b = static_cast<size_t>(desc->dv) * qe;
-  const size_t orow_b = static_cast<size_t>(desc->heads) * desc->dv * qe;
-  std::vector<ic_layer_io> sub(nlayers);
-  for (int i = 0; i < nseq; ++i) {
-    const long o = cu_seqlens[i], n = cu_seqlens[i + 1] - cu_seqlens[i];
-    if (n == 0) continue;
-    ic_stack_desc d = *desc;
-    d.L = static_cast<int>(n);
-    auto at = [o](const void* p, size_t row_b) -> void* {
-      return p ? const_cast<uint8_t*>(static_cast<const uint8_t*>(p)) + o * row_b : nullptr;
-    };
-    for (int l = 0; l < nlayers; ++l) {
-      const ic_layer_io& io = layers[l];
-      ic_layer_io& e = sub[l];
-      e.q_idx = at(io.q_idx, qrow_b);
-      e.q_scale = static_cast<const float*>(at(io.q_scale, desc->H * sizeof(float)));
-      e.k_idx = at(io.k_idx, krow_b);
-      e.k_scale = static_cast<const float*>(at(io.k_scale, sizeof(float)));
-      e.w = static_cast<const float*>(at(io.w, desc->H * sizeof(float)));
-      e.q = at(io.q, arow_b);
-      e.kv = at(io.kv, kvrow_b);
-      e.v = at(io.v, vrow_b);
-      e.out = at(io.out, orow_b);
-      e.lse = static_cast<float*>(at(io.lse, desc->heads * sizeof(float)));
-    }
-    ic_status st = run_stack(pattern, &d, sub.data(), nlayers, t_cache + o * desc->k, workspace,
-                             ws_bytes, stream, false);
-    if (st) return fail(st, "varlen: sequence %d: %s", i, ic_last_error());
-  }
-  return IC_OK;
+  ic_status st = check_desc(desc, false);
+  if (st) return st;
+  std::vector<char> kinds;
+  st = parse_pattern(pattern, &kinds);
+  if (st) return st;
+  if (static_cast<int>(kinds.size()) != nlayers)
+    return fail(IC_ERR_INVALID_ARG, "pattern has %zu layers, nlayers is %d", kinds.size(), nlayers);
+  if (!t_cache) return fail(IC_ERR_INVALID_ARG, "varlen: NULL t_cache");
+  if (cu_seqlens[nseq] * 64 > 0x7fffffffL)
+    return fail(IC_ERR_UNSUPPORTED, "varlen: too many rows for 32-bit TMA coordinates");
+  return run_stack_varlen_shared(kinds, desc, layers, nlayers, cu_seqlens, nseq, t_cache,
+                                 workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 ic_status ic_decode_step(const char* pattern, const ic_stack_desc* desc, const ic_layer_io* layers,

@@ -860,18 +860,36 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
 // ------------------------------------------------------------------ fp32 (MQA) form
 // One CTA per query row, CUDA cores: small shapes only (the fp32 workload has
 // 4 heads of dim 64 over k = 64 keys).
+template <bool SEGS>
 __global__ void attn_f32_kernel(const float* q, const float* kv, long ld_kv, const float* v,
-                                const int* idx, int R, int heads, int dk, int dv, int Lkv, int k,
-                                float scale, float* out, float* lse) {
+                                const int* idx, int R, int heads, int dk, int dv, int Lkv_, int k,
+                                float scale, float* out, float* lse,
+                                const __grid_constant__ AttnSegParam<SEGS> sg) {
   extern __shared__ float f32_smem[];
   float* qs = f32_smem;        // [dk]
   float* z = f32_smem + dk;    // [k]
   __shared__ float red[32];
   const long qrow = blockIdx.x;
-  const long b = qrow / R;
+  long r0;
+  int Lkv;
+  if constexpr (SEGS) {
+    int lo = 0, hi = sg.nseg - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sg.seg[mid].q0 <= qrow)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    r0 = sg.seg[lo].k0;
+    Lkv = sg.seg[lo].len;
+  } else {
+    r0 = (qrow / R) * static_cast<long>(Lkv_);
+    Lkv = Lkv_;
+  }
   const int* irow = idx + qrow * k;
-  const float* kvb = kv + b * static_cast<long>(Lkv) * ld_kv;
-  const float* vb = v + b * static_cast<long>(Lkv) * dv;
+  const float* kvb = kv + r0 * ld_kv;
+  const float* vb = v + r0 * dv;
   const int tid = threadIdx.x, nt = blockDim.x;
   for (int h = 0; h < heads; ++h) {
     const float* qh = q + (qrow * heads + h) * dk;
@@ -923,16 +941,32 @@ __global__ void attn_f32_kernel(const float* q, const float* kv, long ld_kv, con
 
 ic_status launch_attn_f32(const float* q, const float* kv, long ld_kv, const float* v,
                           const int* idx, int batch, int rows, int heads, int dk, int dv, int Lkv,
-                          int k, float scale, float* out, float* lse, cudaStream_t stream) {
+                          int k, float scale, float* out, float* lse, cudaStream_t stream,
+                          const AttnSeg* segs, int nseg) {
   const long items = static_cast<long>(batch) * rows;
   if (items == 0) return IC_OK;
+  if (nseg < 0 || nseg > IC_MAXSEG || (nseg > 0 && (batch != 1 || !segs)))
+    return fail(IC_ERR_INVALID_ARG, "attn: bad segment list (%d)", nseg);
   const int smem = (dk + k) * static_cast<int>(sizeof(float));
-  ic_status st = cuda_check(
-      cudaFuncSetAttribute(attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
-      "cudaFuncSetAttribute(attn_f32)");
-  if (st) return st;
-  attn_f32_kernel<<<static_cast<unsigned>(items), 128, smem, stream>>>(
-      q, kv, ld_kv, v, idx, rows, heads, dk, dv, Lkv, k, scale, out, lse);
+  ic_status st;
+  if (nseg > 0) {
+    AttnSegs sg;
+    sg.nseg = nseg;
+    for (int j = 0; j < nseg; ++j) sg.seg[j] = segs[j];
+    st = cuda_check(cudaFuncSetAttribute(attn_f32_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                    "cudaFuncSetAttribute(attn_f32)");
+    if (st) return st;
+    attn_f32_kernel<true><<<static_cast<unsigned>(items), 128, smem, stream>>>(
+        q, kv, ld_kv, v, idx, rows, heads, dk, dv, Lkv, k, scale, out, lse, sg);
+  } else {
+    st = cuda_check(cudaFuncSetAttribute(attn_f32_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                    "cudaFuncSetAttribute(attn_f32)");
+    if (st) return st;
+    attn_f32_kernel<false><<<static_cast<unsigned>(items), 128, smem, stream>>>(
+        q, kv, ld_kv, v, idx, rows, heads, dk, dv, Lkv, k, scale, out, lse, AttnNoSegs{0});
+  }
   st = cuda_check(cudaGetLastError(), "attn_f32_kernel launch");
   if (!st)
     trace_launch(kKindAttnF32, stream,

@@ -87,6 +87,11 @@ ic_status launch_indexer_tc_segs(bool fp8, const void* q, const float* q_scale, 
                                  const float* k_scale, const float* w, const IdxSeg* segs,
                                  int nseg, long q_rows, long k_rows, float* scores, long ld,
                                  cudaStream_t stream);
+// The fp32 indexer over packed segments: launch row r is row r of q and w and of
+// scores; the segments' orow0 / pos0 / krow0 / Lk place it (qrow0 is unused).
+ic_status launch_indexer_f32_segs(const float* q, const float* k, const float* w, int H, int D,
+                                  const IdxSeg* segs, int nseg, long rows, float* scores, long ld,
+                                  cudaStream_t stream);
 // valid_len[r] of the rows of a block of packed segments (their positions + 1).
 ic_status launch_fill_valid_len(const IdxSeg* segs, int nseg, long rows, int* out,
                                 cudaStream_t stream);
@@ -124,10 +129,11 @@ ic_status launch_attn_mla(const void* q, const void* kv, long ld_kv, const int* 
                           void* ws, size_t ws_bytes, long long valid_entries, cudaStream_t stream,
                           bool kv8 = false, const AttnSeg* segs = nullptr, int nseg = 0);
 size_t attn_mla_ws_bytes(int batch, int rows, int k);
+// segs: as launch_attn_mla's.
 ic_status launch_attn_f32(const float* q, const float* kv, long ld_kv, const float* v,
                           const int* idx, int batch, int rows, int heads, int dk, int dv,
                           int Lkv, int k, float scale, float* out, float* lse,
-                          cudaStream_t stream);
+                          cudaStream_t stream, const AttnSeg* segs = nullptr, int nseg = 0);
 ic_status launch_quant_e4m3(const void* x, bool bf16, long rows, int n, uint8_t* codes,
                             float* scales, cudaStream_t stream);
 // fp8 latent-KV cache rows (656 bytes: 512 e4m3 codes, 4 fp32 group scales, 64 bf16

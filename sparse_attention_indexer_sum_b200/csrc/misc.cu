@@ -3,6 +3,8 @@
 //    E4M3, with one fp32 scale per token, as the fp8 indexer variant takes them);
 //  * the indexer on CUDA cores for fp32 inputs (small head counts and dims:
 //    the fp32 workload has 4 heads of dim 32, far too small for tensor tiles).
+#include <type_traits>
+
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
@@ -114,21 +116,56 @@ ic_status launch_pack_kv_e4m3(const void* kv, long rows, long ld_kv, uint8_t* ou
 
 // I[b,r,s] = sum_h w[b,r,h] * max(0, q[b,r,h,:] . k[b,s,:]) on CUDA cores.
 // Grid (batch * rows, ceil(Lk / 128)); one key per thread, the query row in smem.
+// Packed segments for the fp32 indexer (the rows of a launch that belong to each).
+struct F32IdxSegs {
+  int nseg;
+  IdxSeg seg[IC_MAXSEG];
+};
+struct F32NoSegs {
+  int unused;
+};
+template <bool SEGS>
+using F32SegParam = typename std::conditional<SEGS, F32IdxSegs, F32NoSegs>::type;
+
+// One CTA per (query row, 128-key tile).  With segments, launch row r belongs to
+// the last segment j with seg[j].orow0 <= r: its position is seg.pos0 + (r -
+// seg.orow0) and its keys are rows seg.krow0 .. seg.krow0 + seg.Lk - 1 of k.
+template <bool SEGS>
 __global__ void indexer_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                                    const float* __restrict__ w, int R, int H, int D, int Lk,
-                                   long pos0, float* __restrict__ scores, long ld) {
+                                   long pos0, float* __restrict__ scores, long ld,
+                                   const __grid_constant__ F32SegParam<SEGS> sg) {
   extern __shared__ float qs[];  // [H * D] then w [H]
   const long row = blockIdx.x;   // b * R + r
-  const long b = row / R, r = row % R;
+  long kbase, pos;
+  int lk;
+  if constexpr (SEGS) {
+    int lo = 0, hi = sg.nseg - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sg.seg[mid].orow0 <= row)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    kbase = sg.seg[lo].krow0;
+    pos = sg.seg[lo].pos0 + (row - sg.seg[lo].orow0);
+    lk = sg.seg[lo].Lk;
+  } else {
+    const long b = row / R, r = row % R;
+    kbase = b * Lk;
+    pos = pos0 + r;
+    lk = Lk;
+  }
   float* ws = qs + H * D;
   for (int i = threadIdx.x; i < H * D; i += blockDim.x) qs[i] = q[row * H * D + i];
   for (int i = threadIdx.x; i < H; i += blockDim.x) ws[i] = w[row * H + i];
   __syncthreads();
   const long s = static_cast<long>(blockIdx.y) * blockDim.x + threadIdx.x;
-  if (s >= Lk) return;
+  if (s >= lk) return;
   float res = -INFINITY;
-  if (s <= pos0 + r) {
-    const float* ks = k + (b * Lk + s) * D;
+  if (s <= pos) {
+    const float* ks = k + (kbase + s) * D;
     res = 0.f;
     for (int h = 0; h < H; ++h) {
       float dot = 0.f;
@@ -145,15 +182,44 @@ ic_status launch_indexer_f32(const float* q, const float* k, const float* w, int
   if (static_cast<long>(batch) * rows == 0 || Lk == 0) return IC_OK;
   const int smem = (H * D + H) * static_cast<int>(sizeof(float));
   ic_status st = cuda_check(
-      cudaFuncSetAttribute(indexer_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+      cudaFuncSetAttribute(indexer_f32_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem),
       "cudaFuncSetAttribute(indexer_f32)");
   if (st) return st;
   dim3 grid(static_cast<unsigned>(static_cast<long>(batch) * rows), static_cast<unsigned>((Lk + 127) / 128));
-  indexer_f32_kernel<<<grid, 128, smem, stream>>>(q, k, w, rows, H, D, Lk, pos0, scores, ld);
+  indexer_f32_kernel<false><<<grid, 128, smem, stream>>>(q, k, w, rows, H, D, Lk, pos0, scores, ld,
+                                                         F32NoSegs{0});
   st = cuda_check(cudaGetLastError(), "indexer_f32_kernel launch");
   if (!st)
     trace_launch(kKindIndexerF32, stream,
                  2.0 * H * D * static_cast<double>(causal_pairs(rows, Lk, pos0)) * batch);
+  return st;
+}
+
+ic_status launch_indexer_f32_segs(const float* q, const float* k, const float* w, int H, int D,
+                                  const IdxSeg* segs, int nseg, long rows, float* scores, long ld,
+                                  cudaStream_t stream) {
+  if (rows == 0) return IC_OK;
+  if (nseg < 1 || nseg > IC_MAXSEG) return fail(IC_ERR_INVALID_ARG, "indexer: %d segments", nseg);
+  F32IdxSegs sg;
+  sg.nseg = nseg;
+  int lkmax = 0;
+  double flop = 0.0;
+  for (int j = 0; j < nseg; ++j) {
+    sg.seg[j] = segs[j];
+    lkmax = segs[j].Lk > lkmax ? segs[j].Lk : lkmax;
+    flop += 2.0 * H * D * static_cast<double>(causal_pairs(segs[j].R, segs[j].Lk, segs[j].pos0));
+  }
+  const int smem = (H * D + H) * static_cast<int>(sizeof(float));
+  ic_status st = cuda_check(
+      cudaFuncSetAttribute(indexer_f32_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem),
+      "cudaFuncSetAttribute(indexer_f32)");
+  if (st) return st;
+  dim3 grid(static_cast<unsigned>(rows), static_cast<unsigned>((lkmax + 127) / 128));
+  indexer_f32_kernel<true><<<grid, 128, smem, stream>>>(q, k, w, 1, H, D, lkmax, 0, scores, ld, sg);
+  st = cuda_check(cudaGetLastError(), "indexer_f32_kernel launch");
+  if (!st) trace_launch(kKindIndexerF32, stream, flop);
   return st;
 }
 

@@ -488,8 +488,9 @@ def test_stack_rows_zigzag_pieces_equal_the_whole_stack():
 
 
 def test_stack_varlen_batch_matches_the_oracle_per_sequence():
-    """Sequences of 300, 0, 517 and 64 tokens packed along the rows (fp32 config):
-    each one's index set and outputs match the oracle's stack on that sequence alone."""
+    """Sequences of 300, 0, 517 and 64 tokens packed along the rows (fp32 config), in
+    shared launches (one attention launch per layer for all of them): each one's index
+    set and outputs match the oracle's stack on that sequence alone."""
     lens = [300, 0, 517, 64]
     pattern = "F,S,S"
     seqs = [synth.variant("tiny_stack", L=max(n, 1), pattern=pattern) for n in lens]
@@ -514,8 +515,13 @@ def test_stack_varlen_batch_matches_the_oracle_per_sequence():
                         heads=wl0.Hq, dk=wl0.Dk, dv=wl0.Dv, attn_dtype=ic.IC_F32, scale=wl0.scale)
     ws = torch.empty(ic.ic_stack_workspace_size(desc) // 4 + 1, device=DEV)
     t = torch.full((sum(lens), wl0.k), -7, dtype=torch.int32, device=DEV)
+    ic.ic_trace_begin(256)
     ic.ic_layer_stack_varlen(pattern, desc, packed, cu, t, ws)
+    _, tr = ic.ic_trace_end(256)
     _sync()
+    names = [x[0] for x in tr]
+    assert names.count("attn_f32") == wl0.layers, names
+    assert names.count("indexer_f32") == names.count("topk") <= 2, names  # score-row blocks
     T = t.cpu().numpy()
     for i, n in enumerate(lens):
         if n == 0:
